@@ -1,0 +1,268 @@
+"""Seeded synthetic inputs for the GELU and row-softmax workloads.
+
+This module only draws random numbers and lays them out; it holds none of
+the operators' arithmetic.  It is the one piece shared by the CUDA-side
+callers (bench, tests) and the CPU oracle's callers, so that both see
+bit-identical inputs.
+
+Random source: numpy's PCG64.  Large inputs are generated in fixed chunks,
+each with its own generator derived from ``SeedSequence(seed,
+spawn_key=(chunk,))``, so the bits do not depend on how many host threads
+generate them (numpy releases the GIL while filling arrays).
+
+Workloads (shapes, distributions and structure of the lecture pages'
+workloads; every value is synthetic):
+
+=============  ==============================================================
+cfg1_softmax   fp32 [256, 1000], i.i.d. N(0, 3^2), seed 0
+cfg1_gelu      fp32 [256000], the same values as cfg1_softmax
+cfg2_gelu      fp32 [8388608] (32 MiB), N(0, 1); exactly round(0.01 n) = 83886
+               positions, chosen without replacement, redrawn U[-20, 20]; seed 1
+cfg3_softmax   fp32 [8192, 4096], N(0, 4^2); in every row exactly 410
+               (= round(0.1 * 4096)) positions, chosen without replacement, set
+               to -inf; seed 2
+cfg4_softmax   bf16 [1048576, 2048] = 32 x 16 heads of 2048 x 2048 attention
+               scores, N(0, 8^2) rounded to bf16 (nearest even); causal mask:
+               column j > (row mod 2048) is -inf; seed 3
+cfg5_softmax   fp32 [512, 131072] (256 MiB), N(0, 2^2), plus 50 added at one
+               uniformly drawn position per row; seed 4
+=============  ==============================================================
+
+bf16 arrays are returned as ``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass
+
+import numpy as np
+
+NEG_INF_BF16 = np.uint16(0xFF80)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    op: str          # "gelu" or "softmax"
+    dtype: str       # "f32" or "bf16"
+    shape: tuple     # (n,) for gelu, (rows, cols) for softmax
+    seed: int
+    recipe: str
+
+    @property
+    def numel(self) -> int:
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    @property
+    def itemsize(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """One read of the input plus one write of the output."""
+        return 2 * self.numel * self.itemsize
+
+
+WORKLOADS = {
+    w.name: w for w in [
+        Workload("cfg1_softmax", "softmax", "f32", (256, 1000), 0,
+                 "fp32 256x1000, iid N(0,3^2), seed 0"),
+        Workload("cfg1_gelu", "gelu", "f32", (256000,), 0,
+                 "fp32 256000, the cfg1_softmax values"),
+        Workload("cfg2_gelu", "gelu", "f32", (8388608,), 1,
+                 "fp32 8388608, N(0,1) with 83886 positions redrawn U[-20,20]"),
+        Workload("cfg3_softmax", "softmax", "f32", (8192, 4096), 2,
+                 "fp32 8192x4096, N(0,4^2), 410 -inf per row"),
+        Workload("cfg4_softmax", "softmax", "bf16", (32 * 16 * 2048, 2048), 3,
+                 "bf16 1048576x2048 (32x16 heads x 2048 queries), N(0,8^2), causal -inf"),
+        Workload("cfg5_softmax", "softmax", "f32", (512, 131072), 4,
+                 "fp32 512x131072, N(0,2^2), +50 at one position per row"),
+    ]
+}
+
+
+def _threads(threads: int | None) -> int:
+    if threads:
+        return threads
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def chunk_rng(seed: int, chunk: int) -> np.random.Generator:
+    """Independent generator for one chunk of a workload."""
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(chunk,))))
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Pack fp32 values into bf16 bit patterns, round to nearest even.
+    (Input preparation only; finite inputs.)"""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    bias = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    return ((u + bias) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to fp32 (exact)."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ------------------------------------------------------------------ cfg 1
+
+def _cfg1_values() -> np.ndarray:
+    g = np.random.default_rng(0)
+    return (g.standard_normal(256000) * 3.0).astype(np.float32)
+
+
+# ------------------------------------------------------------------ cfg 2
+
+def _cfg2(n: int = 8388608, seed: int = 1) -> np.ndarray:
+    g = np.random.default_rng(seed)
+    x = g.standard_normal(n, dtype=np.float32)
+    k = int(round(0.01 * n))
+    pos = g.choice(n, size=k, replace=False)
+    x[pos] = g.uniform(-20.0, 20.0, size=k).astype(np.float32)
+    return x
+
+
+# ------------------------------------------------------------------ cfg 3
+
+CFG3_ROWS_PER_CHUNK = 64
+
+
+def _cfg3_chunk(out: np.ndarray, chunk: int, seed: int, n_inf: int) -> None:
+    rows, cols = out.shape
+    g = chunk_rng(seed, chunk)
+    g.standard_normal(out=out, dtype=np.float32)
+    out *= np.float32(4.0)
+    for r in range(rows):
+        out[r, g.choice(cols, size=n_inf, replace=False)] = -np.inf
+
+
+def cfg3_rows(row_begin: int, row_end: int, cols: int = 4096, seed: int = 2) -> np.ndarray:
+    """Rows [row_begin, row_end) of cfg3 (chunk-aligned generation)."""
+    n_inf = int(round(0.1 * cols))
+    c0, c1 = row_begin // CFG3_ROWS_PER_CHUNK, (row_end - 1) // CFG3_ROWS_PER_CHUNK + 1
+    buf = np.empty(((c1 - c0) * CFG3_ROWS_PER_CHUNK, cols), np.float32)
+    for c in range(c0, c1):
+        _cfg3_chunk(buf[(c - c0) * CFG3_ROWS_PER_CHUNK:(c - c0 + 1) * CFG3_ROWS_PER_CHUNK], c, seed, n_inf)
+    off = c0 * CFG3_ROWS_PER_CHUNK
+    return buf[row_begin - off:row_end - off].copy()
+
+
+def _cfg3(rows: int = 8192, cols: int = 4096, seed: int = 2, threads=None) -> np.ndarray:
+    assert rows % CFG3_ROWS_PER_CHUNK == 0
+    n_inf = int(round(0.1 * cols))
+    x = np.empty((rows, cols), np.float32)
+    nchunks = rows // CFG3_ROWS_PER_CHUNK
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(lambda c: _cfg3_chunk(
+            x[c * CFG3_ROWS_PER_CHUNK:(c + 1) * CFG3_ROWS_PER_CHUNK], c, seed, n_inf), range(nchunks)))
+    return x
+
+
+# ------------------------------------------------------------------ cfg 4
+
+CFG4_T = 2048          # queries per head = keys per head
+CFG4_HEADS = 32 * 16   # batch x heads
+
+
+def _cfg4_head(out: np.ndarray, head: int, seed: int) -> None:
+    """One head: out is the uint16 [T, T] block of that head."""
+    t = out.shape[0]
+    g = chunk_rng(seed, head)
+    s = g.standard_normal((t, t), dtype=np.float32)
+    s *= np.float32(8.0)
+    out[...] = f32_to_bf16_bits(s)
+    for i in range(t - 1):                      # key j > query i is masked
+        out[i, i + 1:] = NEG_INF_BF16
+
+
+def cfg4_head(head: int, seed: int = 3, t: int = CFG4_T) -> np.ndarray:
+    out = np.empty((t, t), np.uint16)
+    _cfg4_head(out, head, seed)
+    return out
+
+
+def _cfg4(heads: int = CFG4_HEADS, t: int = CFG4_T, seed: int = 3, threads=None) -> np.ndarray:
+    x = np.empty((heads * t, t), np.uint16)
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(lambda h: _cfg4_head(x[h * t:(h + 1) * t], h, seed), range(heads)))
+    return x
+
+
+# ------------------------------------------------------------------ cfg 5
+
+CFG5_ROWS_PER_CHUNK = 8
+
+
+def _cfg5_chunk(out: np.ndarray, chunk: int, seed: int) -> None:
+    rows, cols = out.shape
+    g = chunk_rng(seed, chunk)
+    g.standard_normal(out=out, dtype=np.float32)
+    out *= np.float32(2.0)
+    pos = g.integers(0, cols, size=rows)
+    out[np.arange(rows), pos] += np.float32(50.0)
+
+
+def cfg5_rows(row_begin: int, row_end: int, cols: int = 131072, seed: int = 4) -> np.ndarray:
+    c0, c1 = row_begin // CFG5_ROWS_PER_CHUNK, (row_end - 1) // CFG5_ROWS_PER_CHUNK + 1
+    buf = np.empty(((c1 - c0) * CFG5_ROWS_PER_CHUNK, cols), np.float32)
+    for c in range(c0, c1):
+        _cfg5_chunk(buf[(c - c0) * CFG5_ROWS_PER_CHUNK:(c - c0 + 1) * CFG5_ROWS_PER_CHUNK], c, seed)
+    off = c0 * CFG5_ROWS_PER_CHUNK
+    return buf[row_begin - off:row_end - off].copy()
+
+
+def _cfg5(rows: int = 512, cols: int = 131072, seed: int = 4, threads=None) -> np.ndarray:
+    assert rows % CFG5_ROWS_PER_CHUNK == 0
+    x = np.empty((rows, cols), np.float32)
+    nchunks = rows // CFG5_ROWS_PER_CHUNK
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(lambda c: _cfg5_chunk(
+            x[c * CFG5_ROWS_PER_CHUNK:(c + 1) * CFG5_ROWS_PER_CHUNK], c, seed), range(nchunks)))
+    return x
+
+
+# ------------------------------------------------------------------ public
+
+def make(name: str, threads: int | None = None) -> np.ndarray:
+    """Full input of a named workload (fp32 array, or uint16 bf16 bits)."""
+    if name == "cfg1_softmax":
+        return _cfg1_values().reshape(256, 1000)
+    if name == "cfg1_gelu":
+        return _cfg1_values()
+    if name == "cfg2_gelu":
+        return _cfg2()
+    if name == "cfg3_softmax":
+        return _cfg3(threads=threads)
+    if name == "cfg4_softmax":
+        return _cfg4(threads=threads)
+    if name == "cfg5_softmax":
+        return _cfg5(threads=threads)
+    raise KeyError(name)
+
+
+def normal(shape, sigma: float, seed: int, dtype: str = "f32") -> np.ndarray:
+    """Generic i.i.d. N(0, sigma^2) test input (fp32, or bf16 bits)."""
+    g = np.random.default_rng(seed)
+    x = (g.standard_normal(shape) * sigma).astype(np.float32)
+    return x if dtype == "f32" else f32_to_bf16_bits(x)
+
+
+def causal_scores(heads: int, t: int, sigma: float, seed: int) -> np.ndarray:
+    """Attention-score-shaped bf16 bits: heads x [t, t], causal -inf mask."""
+    x = np.empty((heads * t, t), np.uint16)
+    for h in range(heads):
+        g = chunk_rng(seed, h)
+        s = g.standard_normal((t, t), dtype=np.float32) * np.float32(sigma)
+        b = f32_to_bf16_bits(s)
+        for i in range(t - 1):
+            b[i, i + 1:] = NEG_INF_BF16
+        x[h * t:(h + 1) * t] = b
+    return x

@@ -1,0 +1,174 @@
+"""CPU oracle for tanh-GELU and row softmax (double precision).
+
+TEST INFRASTRUCTURE ONLY.  This package is the independent checker for the
+CUDA library in ``memory_bound_fk_b200``; it shares no code with it and
+neither imports the other.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.
+
+The arithmetic lives in ``fk_oracle.c`` (plain C, IEEE double, no blocking or
+reordering); this module only marshals numpy arrays into it.
+
+Definitions followed:
+  * GELU (tanh form): lecture-6 notes of CS336 (kyc001.github.io), section 4.2,
+    0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+  * Row softmax: "Lecture 6: GPU Kernels and Triton" (cs336.sjfarmltd.com),
+    section 7.2 (standard two-pass form), and the lecture-6 notes, section 5.2
+    (row max, then exponentials and their sum, then normalise).
+
+Parity pins: every function here is pinned by tests in
+``tests/test_oracle_pins.py`` (closed forms, invariants, library routines
+of the same definition, brute force on tiny inputs).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        d, f, u16 = ctypes.c_double, ctypes.c_float, ctypes.c_uint16
+        p, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        lib.oracle_gelu_tanh.argtypes = [d]
+        lib.oracle_gelu_tanh.restype = d
+        lib.oracle_round_to_f32.argtypes = [d]
+        lib.oracle_round_to_f32.restype = f
+        lib.oracle_round_to_bf16.argtypes = [d]
+        lib.oracle_round_to_bf16.restype = u16
+        lib.oracle_bf16_to_f64.argtypes = [u16]
+        lib.oracle_bf16_to_f64.restype = d
+        for name in ("oracle_gelu_tanh_f64", "oracle_gelu_tanh_f32"):
+            getattr(lib, name).argtypes = [p, p, sz, i]
+            getattr(lib, name).restype = None
+        for name in ("oracle_softmax_rows_f64", "oracle_softmax_rows_f32",
+                     "oracle_softmax_rows_bf16"):
+            getattr(lib, name).argtypes = [p, p, sz, sz, i]
+            getattr(lib, name).restype = None
+        for name in ("oracle_round_to_f32_array", "oracle_round_to_bf16_array",
+                     "oracle_bf16_to_f64_array"):
+            getattr(lib, name).argtypes = [p, p, sz]
+            getattr(lib, name).restype = None
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+# ---------------------------------------------------------------- scalars
+
+def gelu_tanh(x: float) -> float:
+    """GELU (tanh form) of one double."""
+    return _load().oracle_gelu_tanh(float(x))
+
+
+def round_to_f32_scalar(v: float) -> np.float32:
+    return np.float32(_load().oracle_round_to_f32(float(v)))
+
+
+def round_to_bf16_scalar(v: float) -> int:
+    return int(_load().oracle_round_to_bf16(float(v)))
+
+
+# ---------------------------------------------------------------- arrays
+
+def gelu_tanh_f64(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """Elementwise GELU (tanh form), double in, double out."""
+    x = _c(x, np.float64)
+    y = np.empty_like(x)
+    _load().oracle_gelu_tanh_f64(_ptr(x), _ptr(y), x.size, nthreads or default_threads())
+    return y
+
+
+def gelu_tanh_f32(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """fp32 in; computed in double; rounded once to fp32 (nearest even)."""
+    x = _c(x, np.float32)
+    y = np.empty_like(x)
+    _load().oracle_gelu_tanh_f32(_ptr(x), _ptr(y), x.size, nthreads or default_threads())
+    return y
+
+
+def _rows_cols(x: np.ndarray):
+    if x.ndim != 2:
+        raise ValueError("softmax oracle expects a 2-D [rows, cols] array")
+    return x.shape
+
+
+def softmax_rows_f64(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """Softmax over the last axis of a [rows, cols] matrix, double in/out."""
+    x = _c(x, np.float64)
+    rows, cols = _rows_cols(x)
+    y = np.empty_like(x)
+    _load().oracle_softmax_rows_f64(_ptr(x), _ptr(y), rows, cols, nthreads or default_threads())
+    return y
+
+
+def softmax_rows_f32(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """fp32 rows in; computed in double; rounded once to fp32."""
+    x = _c(x, np.float32)
+    rows, cols = _rows_cols(x)
+    y = np.empty_like(x)
+    _load().oracle_softmax_rows_f32(_ptr(x), _ptr(y), rows, cols, nthreads or default_threads())
+    return y
+
+
+def softmax_rows_bf16(x_bits: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """bf16 rows given as uint16 bit patterns; computed in double; rounded
+    once to bf16 (nearest even).  Returns uint16 bit patterns."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = _rows_cols(x)
+    y = np.empty_like(x)
+    _load().oracle_softmax_rows_bf16(_ptr(x), _ptr(y), rows, cols, nthreads or default_threads())
+    return y
+
+
+def round_to_f32(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.float32)
+    _load().oracle_round_to_f32_array(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def round_to_bf16(v: np.ndarray) -> np.ndarray:
+    """double -> bf16 bit patterns (uint16), one rounding, nearest even."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    _load().oracle_round_to_bf16_array(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def bf16_to_f64(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> exact double values."""
+    b = _c(b, np.uint16)
+    out = np.empty(b.shape, np.float64)
+    _load().oracle_bf16_to_f64_array(_ptr(b), _ptr(out), b.size)
+    return out
+
+
+__all__ = [
+    "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32",
+    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16",
+    "round_to_f32", "round_to_bf16", "round_to_f32_scalar", "round_to_bf16_scalar",
+    "bf16_to_f64", "default_threads",
+]

@@ -1,0 +1,342 @@
+/*
+ * fk_oracle.c -- plain CPU oracle for the two fused memory-bound operators.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct
+ * reference that the CUDA library is checked against.  It shares no code,
+ * header, constant or helper with the CUDA library (memory_bound_fk_b200/),
+ * and the CUDA library never calls it.  Only tests/, the smoke check in
+ * __graft_entry__.py and the cpu_baseline / reference legs of bench.py may
+ * load it.
+ *
+ * Everything is computed in IEEE double precision, straight from the
+ * definitions, with no blocking, fusion or reordering:
+ *
+ *   GELU, tanh form -- "GPU Kernels" lecture-6 notes (kyc001.github.io,
+ *   CS336 lecture 6), section 4.2 "GELU":
+ *       GELU(x) = 0.5 x (1 + tanh( sqrt(2/pi) (x + 0.044715 x^3) ))
+ *   The constant 0.044715 is the decimal printed there; sqrt(2/pi) is
+ *   evaluated in double at run time.
+ *
+ *   Row softmax -- "Lecture 6: GPU Kernels and Triton" (cs336.sjfarmltd.com),
+ *   section 7.2 "Online Softmax", the two-pass form: first the row maximum
+ *   and the sum of exp(x - max), then exp(x - max) / sum; and the
+ *   lecture-6 notes (kyc001.github.io), section 5.2: one row at a time,
+ *   max, then exponentials and their sum, then normalise.
+ *
+ * Readings taken where the pages are silent (each also listed in the
+ * design notes):
+ *   - the softmax axis is the last one of a row-major [rows, cols] matrix;
+ *   - GELU(+inf) = +inf and GELU(-inf) = -0 (the limits); the literal
+ *     formula would give (-inf) * 0 = NaN at -inf;
+ *   - a row that is entirely -inf gives NaN everywhere (0/0); a row that
+ *     holds a NaN or a +inf gives NaN everywhere (inf - inf);
+ *   - the row sum uses Neumaier's compensated summation so that the double
+ *     result is accurate to a few units in the last place for any length;
+ *   - results are rounded once, double -> target type, round to nearest
+ *     even (the bf16 rounding works from the double bits directly, so there
+ *     is no intermediate fp32 rounding).
+ *
+ * Rows (and GELU element ranges) are split across POSIX threads; each row
+ * is computed by exactly one thread with the same sequential arithmetic,
+ * so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* Scalar definitions                                                  */
+/* ------------------------------------------------------------------ */
+
+/* GELU, tanh approximation, lecture-6 notes section 4.2. */
+double oracle_gelu_tanh(double x)
+{
+    if (isinf(x))
+        return x > 0.0 ? x : -0.0; /* limits at +-inf */
+    const double k = sqrt(2.0 / M_PI);
+    const double inner = k * (x + 0.044715 * x * x * x);
+    return 0.5 * x * (1.0 + tanh(inner));
+}
+
+/* Softmax of one row, in place of nothing: reads x[0..n), writes y[0..n).
+ * Two passes, as the lecture's section 7.2 states the standard algorithm. */
+static void softmax_row_f64(const double *x, double *y, size_t n)
+{
+    if (n == 0)
+        return;
+    /* pass 1a: row maximum (a NaN never compares greater, so it is skipped
+     * here and then poisons the sum below) */
+    double m = -INFINITY;
+    for (size_t j = 0; j < n; ++j)
+        if (x[j] > m)
+            m = x[j];
+    /* pass 1b: s = sum_j exp(x_j - m), Neumaier-compensated */
+    double s = 0.0, c = 0.0;
+    for (size_t j = 0; j < n; ++j) {
+        const double e = exp(x[j] - m);
+        y[j] = e;
+        const double t = s + e;
+        if (fabs(s) >= fabs(e))
+            c += (s - t) + e;
+        else
+            c += (e - t) + s;
+        s = t;
+    }
+    s = s + c;
+    /* pass 2: normalise */
+    for (size_t j = 0; j < n; ++j)
+        y[j] = y[j] / s;
+}
+
+/* ------------------------------------------------------------------ */
+/* Rounding helpers (double -> fp32 / bf16, round to nearest even)      */
+/* ------------------------------------------------------------------ */
+
+float oracle_round_to_f32(double v)
+{
+    /* C's double -> float conversion rounds to nearest even under the
+     * default floating-point environment. */
+    return (float)v;
+}
+
+/* bf16: 1 sign bit, 8 exponent bits (same range as fp32), 7 fraction bits.
+ * Normal numbers carry 8 significant bits; the subnormal quantum is 2^-133.
+ * Round the double directly to that grid, ties to even. */
+uint16_t oracle_round_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    const int neg = signbit(v) ? 1 : 0;
+    const double a = fabs(v);
+    uint16_t bits;
+    if (isinf(a)) {
+        bits = 0x7F80;
+    } else if (a == 0.0) {
+        bits = 0;
+    } else {
+        int e;
+        (void)frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) -> a in [2^(e-1), 2^e) */
+        int q_exp = (e - 1) - 7; /* quantum of an 8-significant-bit number */
+        if (q_exp < -133)
+            q_exp = -133; /* subnormal range */
+        const double scaled = ldexp(a, -q_exp); /* exact: power-of-two scale */
+        double r = floor(scaled);
+        const double frac = scaled - r; /* exact */
+        if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))
+            r += 1.0;
+        const double rounded = ldexp(r, q_exp); /* exact */
+        if (rounded >= 0x1p128) {
+            bits = 0x7F80; /* overflow to infinity */
+        } else {
+            /* rounded is representable in bf16, hence in fp32 exactly */
+            const float f = (float)rounded;
+            uint32_t u;
+            memcpy(&u, &f, sizeof u);
+            bits = (uint16_t)(u >> 16);
+        }
+    }
+    return (uint16_t)(bits | (neg ? 0x8000 : 0));
+}
+
+double oracle_bf16_to_f64(uint16_t b)
+{
+    const uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------ */
+/* Threading: split [0, count) into nthreads contiguous ranges          */
+/* ------------------------------------------------------------------ */
+
+typedef void (*range_fn)(void *ctx, size_t begin, size_t end);
+
+typedef struct {
+    range_fn fn;
+    void *ctx;
+    size_t begin, end;
+} range_job;
+
+static void *range_job_run(void *p)
+{
+    range_job *j = (range_job *)p;
+    j->fn(j->ctx, j->begin, j->end);
+    return NULL;
+}
+
+static void parallel_ranges(range_fn fn, void *ctx, size_t count, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((size_t)nthreads > count)
+        nthreads = count > 0 ? (int)count : 1;
+    if (nthreads == 1) {
+        fn(ctx, 0, count);
+        return;
+    }
+    pthread_t *tid = (pthread_t *)calloc((size_t)nthreads, sizeof *tid);
+    range_job *jobs = (range_job *)calloc((size_t)nthreads, sizeof *jobs);
+    int *started = (int *)calloc((size_t)nthreads, sizeof *started);
+    const size_t per = count / (size_t)nthreads, extra = count % (size_t)nthreads;
+    size_t at = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        const size_t len = per + ((size_t)t < extra ? 1 : 0);
+        jobs[t].fn = fn;
+        jobs[t].ctx = ctx;
+        jobs[t].begin = at;
+        jobs[t].end = at + len;
+        at += len;
+        started[t] = (pthread_create(&tid[t], NULL, range_job_run, &jobs[t]) == 0);
+        if (!started[t]) /* could not start a thread: do its share here */
+            fn(ctx, jobs[t].begin, jobs[t].end);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        if (started[t])
+            pthread_join(tid[t], NULL);
+    free(started);
+    free(jobs);
+    free(tid);
+}
+
+/* ------------------------------------------------------------------ */
+/* GELU over arrays                                                     */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const void *x;
+    void *y;
+} gelu_ctx;
+
+static void gelu_f64_range(void *p, size_t b, size_t e)
+{
+    gelu_ctx *c = (gelu_ctx *)p;
+    const double *x = (const double *)c->x;
+    double *y = (double *)c->y;
+    for (size_t i = b; i < e; ++i)
+        y[i] = oracle_gelu_tanh(x[i]);
+}
+
+static void gelu_f32_range(void *p, size_t b, size_t e)
+{
+    gelu_ctx *c = (gelu_ctx *)p;
+    const float *x = (const float *)c->x;
+    float *y = (float *)c->y;
+    for (size_t i = b; i < e; ++i)
+        y[i] = oracle_round_to_f32(oracle_gelu_tanh((double)x[i]));
+}
+
+/* double in, double out (no rounding) */
+void oracle_gelu_tanh_f64(const double *x, double *y, size_t n, int nthreads)
+{
+    gelu_ctx c = {x, y};
+    parallel_ranges(gelu_f64_range, &c, n, nthreads);
+}
+
+/* fp32 in, computed in double, rounded once to fp32 */
+void oracle_gelu_tanh_f32(const float *x, float *y, size_t n, int nthreads)
+{
+    gelu_ctx c = {x, y};
+    parallel_ranges(gelu_f32_range, &c, n, nthreads);
+}
+
+/* ------------------------------------------------------------------ */
+/* Row softmax over matrices                                            */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const void *x;
+    void *y;
+    size_t cols;
+} softmax_ctx;
+
+static void softmax_f64_range(void *p, size_t b, size_t e)
+{
+    softmax_ctx *c = (softmax_ctx *)p;
+    const double *x = (const double *)c->x;
+    double *y = (double *)c->y;
+    for (size_t r = b; r < e; ++r)
+        softmax_row_f64(x + r * c->cols, y + r * c->cols, c->cols);
+}
+
+static void softmax_f32_range(void *p, size_t b, size_t e)
+{
+    softmax_ctx *c = (softmax_ctx *)p;
+    const float *x = (const float *)c->x;
+    float *y = (float *)c->y;
+    double *xin = (double *)malloc(c->cols * sizeof(double) + 1);
+    double *yout = (double *)malloc(c->cols * sizeof(double) + 1);
+    for (size_t r = b; r < e; ++r) {
+        const float *xr = x + r * c->cols;
+        float *yr = y + r * c->cols;
+        for (size_t j = 0; j < c->cols; ++j)
+            xin[j] = (double)xr[j];
+        softmax_row_f64(xin, yout, c->cols);
+        for (size_t j = 0; j < c->cols; ++j)
+            yr[j] = oracle_round_to_f32(yout[j]);
+    }
+    free(yout);
+    free(xin);
+}
+
+static void softmax_bf16_range(void *p, size_t b, size_t e)
+{
+    softmax_ctx *c = (softmax_ctx *)p;
+    const uint16_t *x = (const uint16_t *)c->x;
+    uint16_t *y = (uint16_t *)c->y;
+    double *xin = (double *)malloc(c->cols * sizeof(double) + 1);
+    double *yout = (double *)malloc(c->cols * sizeof(double) + 1);
+    for (size_t r = b; r < e; ++r) {
+        const uint16_t *xr = x + r * c->cols;
+        uint16_t *yr = y + r * c->cols;
+        for (size_t j = 0; j < c->cols; ++j)
+            xin[j] = oracle_bf16_to_f64(xr[j]);
+        softmax_row_f64(xin, yout, c->cols);
+        for (size_t j = 0; j < c->cols; ++j)
+            yr[j] = oracle_round_to_bf16(yout[j]);
+    }
+    free(yout);
+    free(xin);
+}
+
+/* double in, double out */
+void oracle_softmax_rows_f64(const double *x, double *y, size_t rows, size_t cols, int nthreads)
+{
+    softmax_ctx c = {x, y, cols};
+    parallel_ranges(softmax_f64_range, &c, rows, nthreads);
+}
+
+/* fp32 in, computed in double, rounded once to fp32 */
+void oracle_softmax_rows_f32(const float *x, float *y, size_t rows, size_t cols, int nthreads)
+{
+    softmax_ctx c = {x, y, cols};
+    parallel_ranges(softmax_f32_range, &c, rows, nthreads);
+}
+
+/* bf16 (raw 16-bit patterns) in, computed in double, rounded once to bf16 */
+void oracle_softmax_rows_bf16(const uint16_t *x, uint16_t *y, size_t rows, size_t cols, int nthreads)
+{
+    softmax_ctx c = {x, y, cols};
+    parallel_ranges(softmax_bf16_range, &c, rows, nthreads);
+}
+
+/* array forms of the rounding helpers */
+void oracle_round_to_f32_array(const double *v, float *out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i)
+        out[i] = oracle_round_to_f32(v[i]);
+}
+
+void oracle_round_to_bf16_array(const double *v, uint16_t *out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i)
+        out[i] = oracle_round_to_bf16(v[i]);
+}
+
+void oracle_bf16_to_f64_array(const uint16_t *b, double *out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i)
+        out[i] = oracle_bf16_to_f64(b[i]);
+}

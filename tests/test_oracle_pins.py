@@ -1,0 +1,328 @@
+"""Pins for the CPU oracle, independent of the oracle's own formulas.
+
+Each check comes from something other than the oracle itself: the
+mathematics of the definitions (closed forms, invariants, special cases),
+library routines that implement the same definition (torch CPU float64),
+high-precision brute force (mpmath), or exhaustive enumeration (bf16).
+They are chosen so that a plausible slip in the oracle -- a dropped cubic
+term, a wrong constant, a sign error, a missing max subtraction, a wrong
+axis, a bad rounding rule -- fails at least one of them.
+
+Definitions:
+  GELU (tanh form): lecture-6 notes (kyc001.github.io), section 4.2.
+  Row softmax: lecture 6 (cs336.sjfarmltd.com), section 7.2; lecture-6
+  notes, section 5.2.
+"""
+import math
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+RNG = np.random.default_rng(12345)
+
+
+# ====================================================================== GELU
+
+def test_gelu_zero_and_signed_zero():
+    assert oracle.gelu_tanh(0.0) == 0.0
+    assert oracle.gelu_tanh(-0.0) == 0.0
+
+
+def test_gelu_odd_part_identity():
+    # tanh is odd, so 0.5x(1+t) - (0.5(-x)(1-t)) = x exactly in real
+    # arithmetic: GELU(x) - GELU(-x) = x.
+    x = np.concatenate([np.linspace(-20, 20, 40001), RNG.standard_normal(10000) * 5])
+    d = oracle.gelu_tanh_f64(x) - oracle.gelu_tanh_f64(-x)
+    assert np.all(np.abs(d - x) <= 4e-16 * np.maximum(np.abs(x), 1e-300) + 1e-300)
+
+
+def test_gelu_large_arguments_tend_to_identity_and_zero():
+    big = np.linspace(10, 1e4, 5001)
+    y = oracle.gelu_tanh_f64(big)
+    # tanh(u) == 1 in double once u > ~19; the fp32 rounding is then x itself
+    assert np.array_equal(oracle.round_to_f32(y), big.astype(np.float32))
+    neg = -big
+    yn = oracle.gelu_tanh_f64(neg)
+    assert np.all(np.abs(yn) < 1e-30)
+
+
+def test_gelu_special_values():
+    assert oracle.gelu_tanh(math.inf) == math.inf
+    r = oracle.gelu_tanh(-math.inf)
+    assert r == 0.0 and math.copysign(1.0, r) == -1.0
+    assert math.isnan(oracle.gelu_tanh(math.nan))
+    # cubic overflow to +-inf inside the tanh argument still gives the limits
+    assert oracle.gelu_tanh(1e200) == 1e200
+    assert oracle.gelu_tanh(-1e200) == 0.0
+
+
+def test_gelu_matches_torch_tanh_gelu_float64():
+    # torch.nn.functional.gelu(approximate='tanh') implements the same
+    # definition independently.
+    x = np.concatenate([np.linspace(-20, 20, 100001), RNG.standard_normal(100000) * 3])
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    y = oracle.gelu_tanh_f64(x)
+    assert np.max(np.abs(y - ref)) <= 1e-14
+
+
+def test_gelu_is_within_tanh_approximation_error_of_exact_gelu():
+    # x * Phi(x) with Phi from erf is the exact GELU; the tanh form is known to
+    # differ from it by at most ~4.7e-4 (largest near x = -2.7).  Dropping the
+    # cubic term pushes the gap above 1e-2; a different inner constant moves
+    # both the size and the place of the largest gap.
+    x = np.linspace(-10, 10, 200001)
+    exact = np.array([v * 0.5 * (1.0 + math.erf(v / math.sqrt(2.0))) for v in x])
+    gap = np.abs(oracle.gelu_tanh_f64(x) - exact)
+    assert 4.6e-4 < gap.max() < 4.8e-4
+    assert -2.75 < x[gap.argmax()] < -2.65
+
+
+def test_gelu_sigmoid_form():
+    # 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)) -- a second closed form
+    x = np.linspace(-12, 12, 24001)
+    u = math.sqrt(2 / math.pi) * (x + 0.044715 * x ** 3)
+    alt = x / (1.0 + np.exp(-2.0 * u))
+    y = oracle.gelu_tanh_f64(x)
+    assert np.max(np.abs(y - alt)) <= 1e-15 * 12
+
+
+def test_gelu_brute_force_mpmath():
+    mpmath.mp.dps = 50
+    xs = np.concatenate([np.linspace(-20, 20, 1201), RNG.standard_normal(800) * 4])
+    c = mpmath.sqrt(2 / mpmath.pi)
+    for x in xs:
+        xm = mpmath.mpf(float(x))
+        exact = mpmath.mpf("0.5") * xm * (1 + mpmath.tanh(c * (xm + mpmath.mpf("0.044715") * xm ** 3)))
+        got = oracle.gelu_tanh(float(x))
+        # double evaluation: a few roundings of relative size 2^-53 in the
+        # inputs of tanh and of the final product; bounded in absolute terms
+        assert abs(mpmath.mpf(got) - exact) <= 8e-16 * max(abs(float(x)), 1.0), x
+
+
+def test_gelu_f32_wrapper_rounds_the_double_result_once():
+    x = (RNG.standard_normal(100000) * 6).astype(np.float32)
+    via64 = oracle.round_to_f32(oracle.gelu_tanh_f64(x.astype(np.float64)))
+    assert np.array_equal(oracle.gelu_tanh_f32(x).view(np.uint32), via64.view(np.uint32))
+
+
+def test_gelu_thread_count_invariance():
+    x = RNG.standard_normal(100003) * 4
+    a = oracle.gelu_tanh_f64(x, nthreads=1)
+    b = oracle.gelu_tanh_f64(x, nthreads=7)
+    assert np.array_equal(a, b)
+
+
+# =================================================================== softmax
+
+@pytest.mark.parametrize("cols", [1, 2, 3, 1000, 4096, 131072])
+def test_softmax_rows_sum_to_one(cols):
+    rows = max(1, 2 ** 18 // cols)
+    x = RNG.standard_normal((rows, cols)) * 4
+    y = oracle.softmax_rows_f64(x)
+    s = y.sum(axis=1, dtype=np.float64)
+    assert np.max(np.abs(s - 1.0)) <= 1e-12
+
+
+def test_softmax_sums_along_rows_not_columns():
+    x = RNG.standard_normal((3, 7)) * 2
+    y = oracle.softmax_rows_f64(x)
+    assert np.allclose(y.sum(axis=1), 1.0, atol=1e-14)
+    assert not np.allclose(y.sum(axis=0), 1.0, atol=1e-3)
+
+
+def test_softmax_shift_invariance_bit_exact():
+    # multiples of 2^-10 in [-64, 64] plus an integer shift stay exact in
+    # double, so x_j - max(x) is the same number and the outputs are equal.
+    x = np.round(RNG.uniform(-64, 64, (64, 777)) * 1024) / 1024
+    for c in (1.0, -37.0, 1024.0):
+        assert np.array_equal(oracle.softmax_rows_f64(x), oracle.softmax_rows_f64(x + c))
+
+
+@pytest.mark.parametrize("n", [1, 1000, 4096, 131072])
+def test_softmax_constant_row_gives_one_over_n(n):
+    x = np.full((2, n), 3.25)
+    y = oracle.softmax_rows_f64(x)
+    assert np.all(y == 1.0 / n)
+
+
+def test_softmax_one_huge_entry_is_one_hot():
+    x = RNG.standard_normal((5, 300)) * 3
+    k = RNG.integers(0, 300, 5)
+    x[np.arange(5), k] += 1000.0
+    y = oracle.softmax_rows_f64(x)
+    expect = np.zeros_like(y)
+    expect[np.arange(5), k] = 1.0
+    assert np.array_equal(y, expect)
+
+
+def test_softmax_two_element_closed_form():
+    a = RNG.standard_normal(2000) * 10
+    b = RNG.standard_normal(2000) * 10
+    y = oracle.softmax_rows_f64(np.stack([a, b], axis=1))
+    sig = lambda d: 1.0 / (1.0 + np.exp(-d))  # noqa: E731
+    assert np.max(np.abs(y[:, 0] - sig(a - b))) <= 2e-16
+    assert np.max(np.abs(y[:, 1] - sig(b - a))) <= 2e-16
+
+
+def test_softmax_ratio_of_outputs_is_exp_of_difference():
+    x = RNG.standard_normal((10, 50)) * 3
+    y = oracle.softmax_rows_f64(x)
+    r = y[:, 1:] / y[:, :1]
+    assert np.allclose(r, np.exp(x[:, 1:] - x[:, :1]), rtol=1e-14, atol=0)
+
+
+def test_softmax_permutation_equivariance():
+    x = RNG.standard_normal((8, 513)) * 5
+    p = RNG.permutation(513)
+    assert np.allclose(oracle.softmax_rows_f64(x[:, p]), oracle.softmax_rows_f64(x)[:, p],
+                       rtol=0, atol=1e-16)
+
+
+def test_softmax_neg_inf_entries_are_exact_zeros_and_causal_row():
+    x = RNG.standard_normal((4, 64)) * 4
+    x[:, ::3] = -np.inf
+    y = oracle.softmax_rows_f64(x)
+    assert np.all(y[:, ::3] == 0.0)
+    assert np.allclose(y.sum(axis=1), 1.0, atol=1e-14)
+    # causal mask, query 0: only key 0 is visible -> exactly [1, 0, ..., 0]
+    t = 16
+    s = RNG.standard_normal((t, t)) * 8
+    s[np.triu_indices(t, 1)] = -np.inf
+    ys = oracle.softmax_rows_f64(s)
+    assert ys[0, 0] == 1.0 and np.all(ys[0, 1:] == 0.0)
+    assert np.all(ys[np.triu_indices(t, 1)] == 0.0)
+
+
+def test_softmax_degenerate_rows_are_nan():
+    x = np.zeros((3, 5))
+    x[0, :] = -np.inf         # all -inf: 0/0
+    x[1, 2] = np.nan          # any NaN
+    x[2, 4] = np.inf          # a +inf: inf - inf
+    y = oracle.softmax_rows_f64(x)
+    assert np.all(np.isnan(y))
+
+
+def test_softmax_matches_torch_float64():
+    for cols in (1, 7, 1000, 4096):
+        x = RNG.standard_normal((64, cols)) * 6
+        x[:, ::5] = -np.inf if cols > 1 else x[:, ::5]
+        ref = torch.softmax(torch.from_numpy(x), dim=-1).numpy()
+        # torch's vectorised exp and summation order differ from libm's by a
+        # few double ulps; outputs are <= 1, so 1e-14 is ~50 ulps of 1.0
+        assert np.max(np.abs(oracle.softmax_rows_f64(x) - ref)) <= 1e-14
+
+
+def test_softmax_brute_force_mpmath():
+    mpmath.mp.dps = 50
+    for n in (1, 2, 5, 17, 100):
+        for _ in range(4):
+            x = RNG.standard_normal(n) * 6
+            xm = [mpmath.mpf(float(v)) for v in x]
+            den = mpmath.fsum(mpmath.exp(v) for v in xm)
+            exact = [mpmath.exp(v) / den for v in xm]
+            y = oracle.softmax_rows_f64(x.reshape(1, n))[0]
+            m = float(np.max(x))
+            for got, ex, xj in zip(y, exact, x):
+                # error bound of the double evaluation: rounding x_j - m costs
+                # |x_j - m| * 2^-53 in the exponent; exp, the compensated sum
+                # and the division add a few units of 2^-53 relative
+                tol = (abs(xj - m) * 1.2e-16 + 8e-16) * ex
+                assert abs(mpmath.mpf(float(got)) - ex) <= tol + 1e-300
+
+
+def test_softmax_online_recurrence_gives_the_same_normaliser():
+    # The running (max, sum) recurrence of lecture 6, section 7.2, applied
+    # block by block, must reach the same max and normaliser as the two-pass
+    # definition; it is a different algorithm for the same quantity.
+    x = RNG.standard_normal(5000) * 7
+    x[::11] = -np.inf
+    m_prev, l_prev = -math.inf, 0.0
+    for blk in np.array_split(x, 37):
+        m_cur = max(m_prev, float(np.max(blk)))
+        corr = math.exp(m_prev - m_cur) if m_prev != -math.inf else 0.0
+        l_prev = corr * l_prev + float(np.sum(np.exp(blk - m_cur)))
+        m_prev = m_cur
+    y_online = np.exp(x - m_prev) / l_prev
+    y = oracle.softmax_rows_f64(x.reshape(1, -1))[0]
+    assert np.max(np.abs(y - y_online)) <= 1e-16 * 50
+
+
+def test_softmax_f32_and_bf16_wrappers_round_once():
+    x = (RNG.standard_normal((33, 1001)) * 4).astype(np.float32)
+    x[:, ::7] = -np.inf
+    ref = oracle.round_to_f32(oracle.softmax_rows_f64(x.astype(np.float64)))
+    assert np.array_equal(oracle.softmax_rows_f32(x).view(np.uint32), ref.view(np.uint32))
+    xb = oracle.round_to_bf16((RNG.standard_normal((17, 2048)) * 8))
+    xb[:, 1000:] = 0xFF80  # -inf
+    refb = oracle.round_to_bf16(oracle.softmax_rows_f64(oracle.bf16_to_f64(xb)))
+    assert np.array_equal(oracle.softmax_rows_bf16(xb), refb)
+
+
+def test_softmax_thread_count_invariance():
+    x = RNG.standard_normal((101, 333)) * 3
+    assert np.array_equal(oracle.softmax_rows_f64(x, nthreads=1), oracle.softmax_rows_f64(x, nthreads=5))
+
+
+# ================================================================= rounding
+
+def _all_finite_bf16():
+    bits = np.arange(0, 0x7F80, dtype=np.uint32)          # +0 .. max finite
+    vals = (bits << 16).view(np.float32).astype(np.float64)
+    return bits.astype(np.uint16), vals
+
+
+def _nearest_even_bf16(v: float, bits, vals) -> int:
+    """Brute force: nearest finite bf16 magnitude, ties to the even pattern,
+    overflow to infinity past the halfway point above the largest finite."""
+    a = abs(v)
+    sign = 0x8000 if math.copysign(1.0, v) < 0 else 0
+    top = vals[-1]
+    ulp_top = vals[-1] - vals[-2]
+    if a >= top + ulp_top / 2:
+        return sign | 0x7F80
+    i = int(np.searchsorted(vals, a))
+    cands = [j for j in (i - 1, i) if 0 <= j < len(vals)]
+    best = min(cands, key=lambda j: (abs(vals[j] - a), int(bits[j]) & 1))
+    return sign | int(bits[best])
+
+
+def test_bf16_rounding_brute_force():
+    bits, vals = _all_finite_bf16()
+    samples = list(RNG.standard_normal(3000) * 10.0 ** RNG.integers(-40, 39, 3000))
+    samples += list(RNG.standard_normal(500) * 1e-39)        # subnormal range
+    # exact ties between neighbours, both parities
+    for k in RNG.integers(1, 0x7F7F, 500):
+        samples.append((vals[k] + vals[k + 1]) / 2)
+        samples.append(-(vals[k] + vals[k + 1]) / 2)
+    samples += [2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135, 2.0 ** -126, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8]
+    got = oracle.round_to_bf16(np.array(samples))
+    for v, g in zip(samples, got):
+        assert int(g) == _nearest_even_bf16(float(v), bits, vals), v
+
+
+def test_bf16_rounding_special_values():
+    top = float((np.uint32(0x7F7F) << 16).view(np.float32))
+    half_ulp = 2.0 ** (127 - 8)
+    r = oracle.round_to_bf16(np.array([np.inf, -np.inf, 0.0, -0.0, top, top + half_ulp,
+                                       top + half_ulp * 0.999]))
+    assert list(r) == [0x7F80, 0xFF80, 0x0000, 0x8000, 0x7F7F, 0x7F80, 0x7F7F]
+    n = oracle.round_to_bf16(np.array([np.nan]))[0]
+    assert (n & 0x7F80) == 0x7F80 and (n & 0x007F) != 0
+
+
+def test_bf16_widening_is_exact_for_every_pattern():
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    got = oracle.bf16_to_f64(b)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert np.all(same)
+
+
+def test_f32_rounding_matches_numpy_cast():
+    v = np.concatenate([RNG.standard_normal(100000) * 10.0 ** RNG.integers(-45, 39, 100000),
+                        [np.inf, -np.inf, 0.0, -0.0, 3.4028235677973366e38]])
+    assert np.array_equal(oracle.round_to_f32(v).view(np.uint32), v.astype(np.float32).view(np.uint32))
