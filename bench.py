@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Throughput of the fused memory-bound operators on B200, as achieved HBM GB/s.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+tanh-GELU over 8,388,608 fp32 values (32 MiB), then row softmax over
+8192 x 4096 fp32, 1,048,576 x 2048 bf16 (32 x 16 heads of 2048 x 2048 causal
+attention scores) and 512 x 131072 fp32 -- every workload of 32 MB and more.
+The bytes counted are the algorithmic ones: one read of every input element
+plus one write of every output element (the fused-kernel traffic of
+"Lecture 6: GPU Kernels and Triton", cs336.sjfarmltd.com, section 1.1).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Timing: W untimed steps, then K steps
+between a barrier + device synchronisation on both sides, CUDA events on
+the launching stream, the maximum over ranks.  Every step reads 4.7 GB, far
+more than the 126 MB L2, so no step finds its inputs in L2.  For N > 1
+(torchrun, one process per GPU) every rank runs the same full workload on
+its own GPU (independent replicas, weak scaling, no collective on the data
+path) and `value` counts the bytes of all ranks.
+
+`--impl reference` times the double-precision CPU oracle (the test checker,
+not a GPU code path) on a bounded sample of the same workload on the host
+cores; it is a deliberately slow baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "achieved HBM GB/s (and % of ~8 TB/s) for row softmax and GELU at 1 B200"
+UNIT = "GB/s"
+SUITE = ["cfg2_gelu", "cfg3_softmax", "cfg4_softmax", "cfg5_softmax"]
+SPEC_HBM_GBS = 8000.0          # nominal B200 HBM3e bandwidth
+FALLBACK_HBM_GBS = 6650.0      # earlier copy measurement on this B200 pool
+KERNEL_NAMES = {               # kernel that each workload's auto plan launches
+    "cfg1_gelu": "gelu_tanh_kernel", "cfg2_gelu": "gelu_tanh_kernel",
+    "cfg1_softmax": "softmax_warp_kernel<float,8>",
+    "cfg3_softmax": "softmax_block_kernel<float,128>",
+    "cfg4_softmax": "softmax_warp_kernel<bf16,8>",
+    "cfg5_softmax": "softmax_block_kernel<float,512,cluster 8>",
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------- host logic
+
+def hbm_traffic_bytes(tensor_bytes: int, n_elementwise_ops: int, fused: bool) -> int:
+    """HBM bytes of n elementwise ops over one tensor: each unfused op reads
+    and writes the whole tensor; the fused kernel reads it once and writes
+    once."""
+    return 2 * tensor_bytes if fused else 2 * n_elementwise_ops * tensor_bytes
+
+
+def workload_list(name: str) -> list[str]:
+    return SUITE if name == "suite" else [name]
+
+
+def describe(names: list[str]) -> str:
+    from memory_bound_fk_b200 import synth
+    return " + ".join(f"{n}: {synth.WORKLOADS[n].recipe}" for n in names)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(values: list[float], world: int, device=None) -> list[float]:
+    """Element-wise maximum of `values` over all ranks (identity for 1 rank)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def aggregate_value(bytes_per_step_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: bytes moved by all ranks / slowest rank's time."""
+    return bytes_per_step_per_rank * steps * world / (max_ms * 1e-3) / 1e9
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("hbm_gbs"):
+            return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "memory_bound_fk_b200", "csrc", "*"))) + \
+        [os.path.join(ROOT, "include", "fk.h")]
+    for p in files:
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, if the
+    kernel sources have not changed since (else None)."""
+    digest = csrc_digest()
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(p).read()
+        for m in re.finditer(r"traffic:\s*workload=(\w+)\s+bytes_per_launch=(\d+)\s+csrc=(\w+)", text):
+            if m.group(1) == workload and m.group(3) == digest:
+                return int(m.group(2)), os.path.relpath(p, ROOT)
+    return None, None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str, period_ms: int = 100):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", str(period_ms)],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, reasons = [], [], set()
+        for line in self.out.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[2:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.out.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def oracle_sample_plan(names, inputs, budget_s: float, threads: int):
+    """Pick the leading fraction f of every workload whose oracle run takes
+    about budget_s on `threads` host threads (calibrated on 1/256)."""
+    import numpy as np  # noqa: F401
+    cal = oracle_run(names, inputs, 1.0 / 256, threads)
+    f = min(1.0, max(1.0 / 4096, budget_s / max(cal["seconds"] * 256, 1e-9)))
+    return f
+
+
+def _slice(name, arr, frac):
+    if arr.ndim == 1:
+        n = max(1, int(arr.shape[0] * frac))
+        return arr[:n]
+    r = max(1, int(round(arr.shape[0] * frac)))
+    return arr[:r]
+
+
+def oracle_run(names, inputs, frac, threads):
+    import oracle
+    from memory_bound_fk_b200 import synth
+    total_bytes, elems = 0, 0
+    t0 = time.perf_counter()
+    for n in names:
+        w = synth.WORKLOADS[n]
+        x = _slice(n, inputs[n], frac)
+        if w.op == "gelu":
+            oracle.gelu_tanh_f32(x, nthreads=threads)
+        elif w.dtype == "f32":
+            oracle.softmax_rows_f32(x, nthreads=threads)
+        else:
+            oracle.softmax_rows_bf16(x, nthreads=threads)
+        total_bytes += 2 * x.size * w.itemsize
+        elems += x.size
+    dt = time.perf_counter() - t0
+    return {"seconds": dt, "bytes": total_bytes, "elements": elems}
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def make_inputs(names):
+    from memory_bound_fk_b200 import synth
+    out = {}
+    for n in names:
+        t = time.perf_counter()
+        out[n] = synth.make(n)
+        log(f"[bench] generated {n} {out[n].shape} in {time.perf_counter() - t:.1f}s")
+    return out
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args) -> dict | None:
+    import numpy as np
+    import torch
+
+    import memory_bound_fk_b200 as fk
+    from memory_bound_fk_b200 import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    fk.lib()  # fail loudly if libfk.so is missing
+    names = workload_list(args.workload)
+    host = make_inputs(names)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+
+    # device buffers, inputs resident in HBM before the timed region
+    dev_in, dev_out, calls = {}, {}, []
+    for n in names:
+        w = synth.WORKLOADS[n]
+        if w.dtype == "bf16":
+            t = torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(host[n])
+        dev_in[n] = t.to(device)
+        dev_out[n] = torch.empty_like(dev_in[n])
+        xp, yp = dev_in[n].data_ptr(), dev_out[n].data_ptr()
+        if w.op == "gelu":
+            calls.append((n, lambda xp=xp, yp=yp, k=w.numel: fk.fk_gelu_tanh(xp, yp, k, sh)))
+        else:
+            r, c = w.shape
+            code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+            calls.append((n, lambda xp=xp, yp=yp, r=r, c=c, code=code:
+                          fk.fk_softmax_rows(xp, yp, r, c, code, sh)))
+    bytes_step = sum(synth.WORKLOADS[n].algorithmic_bytes for n in names)
+    elems_step = sum(synth.WORKLOADS[n].numel for n in names)
+
+    def step(evs=None):
+        for i, (n, call) in enumerate(calls):
+            if evs is not None:
+                evs[i].record(stream)
+            st = call()
+            if st != fk.FK_OK:
+                raise fk.FkError(st, n)
+        if evs is not None:
+            evs[len(calls)].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        step()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+              for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    barrier()
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)  # let the sampler take its first reading
+    barrier()
+    start.record(stream)
+    for k in range(args.steps):
+        step(events[k])
+    stop.record(stream)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = start.elapsed_time(stop)
+    per_kernel_ms = [0.0] * len(calls)
+    for evs in events:
+        for i in range(len(calls)):
+            per_kernel_ms[i] += evs[i].elapsed_time(evs[i + 1])
+    reduced = max_over_ranks([total_ms] + per_kernel_ms, world, device)
+    max_ms, kernel_ms = reduced[0], reduced[1:]
+
+    # end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, names, host, dev_in, dev_out, calls, stream, device, world, bytes_step)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = host_threads()
+        f = oracle_sample_plan(names, host, args.cpu_budget, threads)
+        res = oracle_run(names, host, f, threads)
+        cpu = {"value": res["bytes"] / res["seconds"] / 1e9, "unit": UNIT, "cores": threads,
+               "kind": "oracle",
+               "sample": f"leading {100 * f:.3f}% of every workload ({res['elements']} elements, "
+                         f"{res['bytes'] / 1e9:.3f} GB algorithmic, {res['seconds']:.1f} s)"}
+
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    kernels = []
+    for i, n in enumerate(names):
+        w = synth.WORKLOADS[n]
+        ms = kernel_ms[i] / args.steps
+        gbs = w.algorithmic_bytes / (ms * 1e-3) / 1e9
+        plan = (fk.fk_softmax_rows_plan(w.shape[0], w.shape[1],
+                                        fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32).as_dict()
+                if w.op == "softmax" else {"path": "gelu"})
+        kernels.append({"workload": n, "kernel": KERNEL_NAMES.get(n), "plan": plan,
+                        "ms": round(ms, 5), "GB_s": round(gbs, 1),
+                        "elements_per_s": round(w.numel / (ms * 1e-3), 1),
+                        "pct_of_8TBs": round(100 * gbs / SPEC_HBM_GBS, 2),
+                        "frac_of_measured_copy": round(gbs / peaks["hbm_gbs"], 4),
+                        "bytes_per_launch": w.algorithmic_bytes})
+    dom = max(range(len(names)), key=lambda i: kernel_ms[i])
+    dk = kernels[dom]
+    traffic, traffic_src = profiled_traffic(names[dom])
+    value = aggregate_value(bytes_step, args.steps, world, max_ms)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "detail": describe(names),
+                   "io_dtypes": sorted({synth.WORKLOADS[n].dtype for n in names}),
+                   "bytes_per_step_per_gpu": bytes_step, "elements_per_step_per_gpu": elems_step,
+                   "l2": f"inputs larger than L2: {bytes_step // 2 / 1e9:.2f} GB read per step",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "pct_of_8TBs": round(100 * value / world / SPEC_HBM_GBS, 2),
+        "elements_per_s": round(elems_step * args.steps * world / (max_ms * 1e-3), 1),
+        "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": dk["kernel"], "workload": names[dom],
+                     "achieved": dk["GB_s"], "peak": peaks["hbm_gbs"], "unit": UNIT,
+                     "frac": round(dk["GB_s"] / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"],
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_bytes_per_launch": dk["bytes_per_launch"]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": len(calls) * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+def run_e2e(args, names, host, dev_in, dev_out, calls, stream, device, world, bytes_step):
+    import numpy as np
+    import torch
+    pin_in, pin_out = {}, {}
+    for n in names:
+        a = host[n]
+        src = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        pin_in[n] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+        pin_in[n].copy_(src)
+        pin_out[n] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+    h2d = sum(pin_in[n].numel() * pin_in[n].element_size() for n in names)
+    d2h = sum(pin_out[n].numel() * pin_out[n].element_size() for n in names)
+    import memory_bound_fk_b200 as fk
+
+    def step():
+        for n, call in calls:
+            dst = dev_in[n].view(torch.int16) if dev_in[n].dtype == torch.bfloat16 else dev_in[n]
+            dst.copy_(pin_in[n], non_blocking=True)
+            st = call()
+            if st != fk.FK_OK:
+                raise fk.FkError(st, n)
+            src = dev_out[n].view(torch.int16) if dev_out[n].dtype == torch.bfloat16 else dev_out[n]
+            pin_out[n].copy_(src, non_blocking=True)
+
+    steps = max(3, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks([a.elapsed_time(b)], world, device)[0]
+    return {"value": round(aggregate_value(bytes_step, steps, world, ms), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args) -> dict | None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    names = workload_list(args.workload)
+    host = make_inputs(names)
+    threads = host_threads()
+    per_step = args.reference_budget / max(1, args.steps + args.warmup)
+    f = oracle_sample_plan(names, host, per_step, threads)
+    for _ in range(args.warmup):
+        oracle_run(names, host, f, threads)
+    secs, nbytes, elems = 0.0, 0, 0
+    for _ in range(args.steps):
+        r = oracle_run(names, host, f, threads)
+        secs += r["seconds"]
+        nbytes += r["bytes"]
+        elems += r["elements"]
+    value = nbytes / secs / 1e9
+    sample = (f"leading {100 * f:.4f}% of every workload per step "
+              f"({elems // max(1, args.steps)} elements per step)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "detail": describe(names),
+                   "parallelism": "host cores (oracle)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="suite",
+                   help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
+                        "cfg3_softmax, cfg4_softmax, cfg5_softmax")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    p.add_argument("--reference-budget", type=float, default=120.0,
+                   help="seconds for the whole --impl reference run")
+    a = p.parse_args(argv)
+    if a.warmup < 3 and a.impl == "ours" and a.steps > 10:
+        p.error("--warmup must be at least 3 for a reported measurement")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if args.impl == "ours" and dist_env()[1] > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

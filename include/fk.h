@@ -1,0 +1,165 @@
+/*
+ * fk.h -- C ABI of libfk: fused memory-bound operators for NVIDIA B200 (sm_100a).
+ *
+ * Two operators, each one kernel that reads every input element once from
+ * HBM and writes every output element once (the fusion argument of
+ * "Lecture 6: GPU Kernels and Triton", cs336.sjfarmltd.com, section 1.1:
+ * one read plus one write instead of a read and a write per separate op):
+ *
+ *   fk_gelu_tanh     y = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+ *                    -- CS336 lecture-6 notes (kyc001.github.io), section 4.2.
+ *   fk_softmax_rows  y[r, j] = exp(x[r, j] - m_r) / sum_k exp(x[r, k] - m_r),
+ *                    m_r = max_k x[r, k], over the last axis of a row-major
+ *                    [rows, cols] matrix -- lecture 6, section 7.2 (two-pass
+ *                    form; the running max/sum merge of the same section is
+ *                    used where one row is split across thread blocks), and
+ *                    the lecture-6 notes, section 5.2 (row max, exponentials
+ *                    and sum, normalise).
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ * Memory:    every pointer is caller-owned memory that the current CUDA
+ *            device can access (cudaMalloc / torch tensors, managed or
+ *            mapped pinned host memory).  libfk allocates nothing, holds no
+ *            handles and keeps no state besides a per-device properties
+ *            cache.  Pageable host memory is rejected (FK_ERR_INVALID_ARG).
+ * Layout:    contiguous; softmax rows are row-major with row stride = cols.
+ * Streams:   `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *            default stream).  Calls are asynchronous: the kernel is enqueued
+ *            and the call returns without synchronising.
+ * Aliasing:  x == y (in place) is allowed; any other overlap of the input and
+ *            output ranges is rejected.
+ * Errors:    all argument checks run on the host before anything is
+ *            enqueued; a failing check returns its code and launches nothing.
+ *            A zero-sized problem returns FK_OK and launches nothing (NULL
+ *            pointers are then allowed).  A launch failure returns
+ *            FK_ERR_CUDA (the CUDA error code is kept per host thread, see
+ *            fk_last_cuda_error).  Errors of the asynchronous execution
+ *            surface at the caller's next synchronisation.  Device code never
+ *            traps, asserts or prints.
+ * Device:    kernels are built for sm_100a only; any other device returns
+ *            FK_ERR_UNSUPPORTED_DEVICE.
+ * Threads:   every entry point may be called concurrently from several host
+ *            threads.
+ */
+#ifndef FK_H
+#define FK_H
+
+#include <stddef.h>
+
+/* Exported entry points keep default visibility even when the library is
+ * built with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define FK_API __attribute__((visibility("default")))
+#else
+#define FK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fk_status {
+    FK_OK = 0,
+    FK_ERR_INVALID_ARG = 1,        /* NULL pointer, bad size/overflow, misalignment, overlap, bad plan */
+    FK_ERR_UNSUPPORTED_DTYPE = 2,  /* dtype is not one of fk_dtype */
+    FK_ERR_UNSUPPORTED_DEVICE = 3, /* no CUDA device, or not compute capability 10.0 (sm_100a) */
+    FK_ERR_CUDA = 4                /* a CUDA runtime call or the launch failed */
+} fk_status;
+
+typedef enum fk_dtype {
+    FK_F32 = 0,  /* IEEE binary32 */
+    FK_BF16 = 1  /* bfloat16 (8-bit exponent, 7-bit fraction); math in fp32, output rounded to nearest even */
+} fk_dtype;
+
+/*
+ * fk_gelu_tanh -- elementwise GELU, tanh form (lecture-6 notes, section 4.2).
+ *   x  [in]  n fp32 values, device-accessible, 4-byte aligned.
+ *   y  [out] n fp32 values, same constraints; y == x allowed.
+ *   n        element count (0 = no-op).
+ *   stream   cudaStream_t as void*.
+ * Arithmetic in fp32: y is within 2e-6 of the exact (double) value for every
+ * finite x; GELU(+inf) = +inf, GELU(-inf) = -0, GELU(NaN) = NaN.
+ * 16-byte aligned x and y (same offset mod 16) take the 128-bit vector path;
+ * any other alignment is still correct.
+ */
+FK_API fk_status fk_gelu_tanh(const float *x, float *y, size_t n, void *stream);
+
+/*
+ * fk_softmax_rows -- softmax over each row of a row-major [rows, cols]
+ * matrix (lecture 6, section 7.2; lecture-6 notes, section 5.2).
+ *   x      [in]  rows*cols elements of `dtype`, device-accessible, aligned to
+ *                the element size.
+ *   y      [out] rows*cols elements of the same dtype; y == x allowed.
+ *   rows, cols   matrix shape (either 0 = no-op).
+ *   dtype  an fk_dtype; input and output share it.
+ *   stream cudaStream_t as void*.
+ * Arithmetic: fp32 for both dtypes (bf16 is widened exactly, accumulated in
+ * fp32, rounded to nearest even on store).  Each input element is read from
+ * HBM once and each output written once, except on the two-phase path for
+ * rows longer than a thread-block cluster holds on chip (FK_PATH_TWOPHASE,
+ * over 524288 columns of either dtype), which reads the row twice.
+ * -inf inputs give exactly 0; a row that is all -inf, or holds a NaN or a
+ * +inf, gives NaN throughout.
+ */
+FK_API fk_status fk_softmax_rows(const void *x, void *y, size_t rows, size_t cols, int dtype, void *stream);
+
+/* Kernel paths of fk_softmax_rows. */
+typedef enum fk_softmax_path {
+    FK_PATH_AUTO = 0,     /* let fk_softmax_rows_plan choose */
+    FK_PATH_WARP = 1,     /* one warp per row, row held in registers */
+    FK_PATH_CTA = 2,      /* one thread block per row, row held in registers */
+    FK_PATH_CLUSTER = 3,  /* one thread-block cluster per row, slices in registers,
+                             (max, sum) partials merged over distributed shared memory */
+    FK_PATH_TWOPHASE = 4  /* one cluster per row, streamed twice: running (max, sum)
+                             pass, then normalise pass -- any row length */
+} fk_softmax_path;
+
+/* A resolved launch plan.  `threads` = threads per block; `vpt` = 16-byte
+ * vectors per thread per chunk; `cluster` = blocks per row (1 for WARP/CTA). */
+typedef struct fk_softmax_plan {
+    int path;
+    int threads;
+    int vpt;
+    int cluster;
+} fk_softmax_plan;
+
+/*
+ * fk_softmax_rows_plan -- the plan fk_softmax_rows would use (host only,
+ * launches nothing, needs no device).
+ *   rows, cols, dtype  as for fk_softmax_rows (cols > 0).
+ *   path     FK_PATH_AUTO, or a path to force; its threads/vpt/cluster are
+ *            then chosen for that path.
+ *   out      [out] the plan.
+ * Returns FK_ERR_INVALID_ARG when the forced path cannot hold `cols`
+ * (WARP/CTA/CLUSTER have fixed on-chip capacities).
+ */
+FK_API fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan *out);
+
+/*
+ * fk_softmax_rows_ex -- fk_softmax_rows with an explicit plan (tests and
+ * tuning).  plan == NULL or plan->path == FK_PATH_AUTO behaves like
+ * fk_softmax_rows.  Otherwise every field is validated against the compiled
+ * kernel set (threads in {128,256,512,1024} for block paths; cluster in
+ * 1..16; vpt fixed per dtype and path) and FK_ERR_INVALID_ARG is returned
+ * for a plan that is not built or cannot hold `cols`.  Zero fields take the
+ * path's defaults.
+ */
+FK_API fk_status fk_softmax_rows_ex(const void *x, void *y, size_t rows, size_t cols, int dtype,
+                             const fk_softmax_plan *plan, void *stream);
+
+/* Static description of a status code (never NULL). */
+FK_API const char *fk_status_string(int status);
+
+/* The cudaError_t of the last FK_ERR_CUDA returned on this host thread
+ * (0 if none). */
+FK_API int fk_last_cuda_error(void);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+FK_API int fk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FK_H */

@@ -1,1 +1,212 @@
-"""memory_bound_fk_b200: fused memory-bound operators (tanh-GELU, row softmax) for B200."""
+"""memory_bound_fk_b200 -- fused memory-bound operators for NVIDIA B200 (sm_100a).
+
+Python binding of ``libfk.so`` (declared in ``include/fk.h``).  This module
+only marshals arguments: every step of the computation runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams.
+
+Raw C-ABI mirrors (same names, pointers as integers, stream as a
+``cudaStream_t`` integer):
+    fk_gelu_tanh(x, y, n, stream) -> status
+    fk_softmax_rows(x, y, rows, cols, dtype, stream) -> status
+    fk_softmax_rows_ex(x, y, rows, cols, dtype, plan, stream) -> status
+    fk_softmax_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
+    fk_status_string(status) -> str
+
+Tensor conveniences (contiguous CUDA tensors; the current torch stream):
+    gelu_tanh(x, out=None)
+    softmax_rows(x, out=None, plan=None)    # softmax over the last dimension
+
+There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfk.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "fk.h")
+
+# fk_status
+FK_OK = 0
+FK_ERR_INVALID_ARG = 1
+FK_ERR_UNSUPPORTED_DTYPE = 2
+FK_ERR_UNSUPPORTED_DEVICE = 3
+FK_ERR_CUDA = 4
+# fk_dtype
+FK_F32 = 0
+FK_BF16 = 1
+# fk_softmax_path
+FK_PATH_AUTO = 0
+FK_PATH_WARP = 1
+FK_PATH_CTA = 2
+FK_PATH_CLUSTER = 3
+FK_PATH_TWOPHASE = 4
+PATH_NAMES = {FK_PATH_WARP: "warp", FK_PATH_CTA: "cta", FK_PATH_CLUSTER: "cluster",
+              FK_PATH_TWOPHASE: "twophase"}
+
+
+class FkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {fk_status_string(status)}"
+                         + (f" (cudaError {fk_last_cuda_error()})" if status == FK_ERR_CUDA else ""))
+
+
+class SoftmaxPlan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("threads", ctypes.c_int),
+                ("vpt", ctypes.c_int), ("cluster", ctypes.c_int)]
+
+    def as_dict(self) -> dict:
+        return {"path": PATH_NAMES.get(self.path, self.path), "threads": self.threads,
+                "vpt": self.vpt, "cluster": self.cluster}
+
+    def __repr__(self) -> str:
+        return f"SoftmaxPlan({self.as_dict()})"
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfk.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libfk.so not found at {LIB_PATH}; build it with "
+                              "`python -m memory_bound_fk_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        L.fk_gelu_tanh.argtypes = [vp, vp, sz, vp]
+        L.fk_gelu_tanh.restype = ci
+        L.fk_softmax_rows.argtypes = [vp, vp, sz, sz, ci, vp]
+        L.fk_softmax_rows.restype = ci
+        L.fk_softmax_rows_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.POINTER(SoftmaxPlan), vp]
+        L.fk_softmax_rows_ex.restype = ci
+        L.fk_softmax_rows_plan.argtypes = [sz, sz, ci, ci, ctypes.POINTER(SoftmaxPlan)]
+        L.fk_softmax_rows_plan.restype = ci
+        L.fk_status_string.argtypes = [ci]
+        L.fk_status_string.restype = ctypes.c_char_p
+        L.fk_last_cuda_error.argtypes = []
+        L.fk_last_cuda_error.restype = ci
+        L.fk_version.argtypes = []
+        L.fk_version.restype = ci
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the entry points declared in include/fk.h."""
+    text = open(HEADER_PATH).read()
+    return re.findall(r"FK_API\s+[\w\s\*]+?\b(fk_\w+)\s*\(", text)
+
+
+# ---------------------------------------------------------------- raw mirrors
+
+def fk_gelu_tanh(x: int, y: int, n: int, stream: int = 0) -> int:
+    return lib().fk_gelu_tanh(x, y, n, stream)
+
+
+def fk_softmax_rows(x: int, y: int, rows: int, cols: int, dtype: int, stream: int = 0) -> int:
+    return lib().fk_softmax_rows(x, y, rows, cols, dtype, stream)
+
+
+def fk_softmax_rows_ex(x: int, y: int, rows: int, cols: int, dtype: int,
+                       plan: SoftmaxPlan | None, stream: int = 0) -> int:
+    return lib().fk_softmax_rows_ex(x, y, rows, cols, dtype,
+                                    ctypes.byref(plan) if plan is not None else None, stream)
+
+
+def fk_softmax_rows_plan(rows: int, cols: int, dtype: int, path: int = FK_PATH_AUTO) -> SoftmaxPlan:
+    p = SoftmaxPlan()
+    st = lib().fk_softmax_rows_plan(rows, cols, dtype, path, ctypes.byref(p))
+    if st != FK_OK:
+        raise FkError(st, "fk_softmax_rows_plan")
+    return p
+
+
+def fk_status_string(status: int) -> str:
+    return lib().fk_status_string(status).decode()
+
+
+def fk_last_cuda_error() -> int:
+    return lib().fk_last_cuda_error()
+
+
+def fk_version() -> int:
+    return lib().fk_version()
+
+
+def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0) -> SoftmaxPlan:
+    return SoftmaxPlan(path, threads, vpt, cluster)
+
+
+# ---------------------------------------------------------------- tensors
+
+def _stream_handle(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _check_tensor(t, name: str):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gelu_tanh(x, out=None):
+    """tanh-GELU of a contiguous fp32 CUDA tensor (``out`` may be ``x``)."""
+    import torch
+    _check_tensor(x, "x")
+    if x.dtype != torch.float32:
+        raise TypeError("gelu_tanh takes float32")
+    if out is None:
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.dtype != x.dtype or out.numel() != x.numel() or out.device != x.device:
+        raise ValueError("out must match x in dtype, size and device")
+    st = fk_gelu_tanh(x.data_ptr(), out.data_ptr(), x.numel(), _stream_handle(x))
+    if st != FK_OK:
+        raise FkError(st, "fk_gelu_tanh")
+    return out
+
+
+def _dtype_code(dt) -> int:
+    import torch
+    if dt == torch.float32:
+        return FK_F32
+    if dt == torch.bfloat16:
+        return FK_BF16
+    raise TypeError("softmax_rows takes float32 or bfloat16")
+
+
+def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None):
+    """Softmax over the last dimension of a contiguous fp32/bf16 CUDA tensor."""
+    import torch
+    _check_tensor(x, "x")
+    code = _dtype_code(x.dtype)
+    if out is None:
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.dtype != x.dtype or out.shape != x.shape or out.device != x.device:
+        raise ValueError("out must match x in dtype, shape and device")
+    cols = x.shape[-1] if x.dim() > 0 else 1
+    rows = x.numel() // cols if cols else 0
+    st = fk_softmax_rows_ex(x.data_ptr(), out.data_ptr(), rows, cols, code, plan, _stream_handle(x))
+    if st != FK_OK:
+        raise FkError(st, "fk_softmax_rows")
+    return out
+
+
+__all__ = [
+    "FK_OK", "FK_ERR_INVALID_ARG", "FK_ERR_UNSUPPORTED_DTYPE", "FK_ERR_UNSUPPORTED_DEVICE",
+    "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
+    "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FkError", "SoftmaxPlan", "lib", "header_functions",
+    "fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
+    "fk_status_string", "fk_last_cuda_error", "fk_version", "make_plan", "gelu_tanh",
+    "softmax_rows",
+]

@@ -1,0 +1,208 @@
+// fk_api.cu -- the C ABI of libfk (declared in include/fk.h): argument
+// validation, the per-device properties cache, and dispatch to the kernels.
+//
+// Every check runs on the host before anything is enqueued, so a rejected
+// call launches nothing.  Pointer checks use the CUDA runtime's pointer
+// attributes (pageable host memory is not device-accessible) and the
+// driver's address-range query (the whole [ptr, ptr + bytes) span must lie
+// inside one allocation), which turns a wrong size into an error code
+// instead of a device fault.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "fk.h"
+#include "fk_internal.h"
+
+namespace fk {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kVersion = 10000;  // 1.0.0
+
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_info_once[kMaxDevices];
+thread_local int t_last_cuda_error = 0;
+
+fk_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FK_ERR_CUDA;
+}
+
+void query_device(int dev) {
+  DeviceInfo& d = g_info[dev];
+  d.ok = 0;
+  cudaDeviceProp p;
+  if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return;
+  d.major = p.major;
+  d.minor = p.minor;
+  d.sm_count = p.multiProcessorCount;
+  d.max_threads_sm = p.maxThreadsPerMultiProcessor;
+  d.l2_bytes = static_cast<size_t>(p.l2CacheSize);
+  d.ok = 1;
+}
+
+// cuMemGetAddressRange, resolved once through the runtime so that libfk
+// needs no link-time dependency on the driver library.
+typedef CUresult (*PFN_addr_range)(CUdeviceptr*, size_t*, CUdeviceptr);
+std::atomic<PFN_addr_range> g_addr_range{nullptr};
+std::once_flag g_addr_range_once;
+
+PFN_addr_range addr_range_fn() {
+  std::call_once(g_addr_range_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_addr_range.store(reinterpret_cast<PFN_addr_range>(fn));
+  });
+  return g_addr_range.load();
+}
+
+// Is [p, p + bytes) memory the current device `dev` may access?
+fk_status check_pointer(const void* p, size_t bytes, int dev) {
+  cudaPointerAttributes a;
+  const cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // clear the non-sticky error
+    return FK_ERR_INVALID_ARG;
+  }
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+      if (a.device != dev) return FK_ERR_INVALID_ARG;
+      break;
+    case cudaMemoryTypeManaged:
+      break;
+    case cudaMemoryTypeHost:
+      if (a.devicePointer == nullptr) return FK_ERR_INVALID_ARG;
+      break;
+    default:  // unregistered (pageable) host memory
+      return FK_ERR_INVALID_ARG;
+  }
+  if (a.type == cudaMemoryTypeDevice) {
+    if (PFN_addr_range f = addr_range_fn()) {
+      CUdeviceptr base = 0;
+      size_t size = 0;
+      // device memory whose extent cannot be established is not accepted
+      if (f(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return FK_ERR_INVALID_ARG;
+      const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+      if (lo < base || lo - base > size || bytes > size - (lo - base)) return FK_ERR_INVALID_ARG;
+    }
+  }
+  return FK_OK;
+}
+
+bool overlaps_partially(const void* x, const void* y, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(x), b = reinterpret_cast<uintptr_t>(y);
+  if (a == b) return false;  // exact aliasing: in place, allowed
+  return a < b + bytes && b < a + bytes;
+}
+
+// Common checks for one (x, y, element count, element size) call.
+fk_status check_call(const void* x, const void* y, size_t count, size_t esize,
+                     const DeviceInfo** dev_out) {
+  if (x == nullptr || y == nullptr) return FK_ERR_INVALID_ARG;
+  if (count > SIZE_MAX / esize) return FK_ERR_INVALID_ARG;
+  const size_t bytes = count * esize;
+  if ((reinterpret_cast<uintptr_t>(x) % esize) != 0 || (reinterpret_cast<uintptr_t>(y) % esize) != 0)
+    return FK_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) > UINTPTR_MAX - bytes ||
+      reinterpret_cast<uintptr_t>(y) > UINTPTR_MAX - bytes)
+    return FK_ERR_INVALID_ARG;
+  if (overlaps_partially(x, y, bytes)) return FK_ERR_INVALID_ARG;
+  int dev = -1;
+  const DeviceInfo* info = current_device_info(&dev);
+  if (info == nullptr || !info->ok) return FK_ERR_UNSUPPORTED_DEVICE;
+  if (info->major != 10 || info->minor != 0) return FK_ERR_UNSUPPORTED_DEVICE;
+  fk_status st = check_pointer(x, bytes, dev);
+  if (st != FK_OK) return st;
+  if (y != x) {
+    st = check_pointer(y, bytes, dev);
+    if (st != FK_OK) return st;
+  }
+  *dev_out = info;
+  return FK_OK;
+}
+
+}  // namespace
+
+const DeviceInfo* current_device_info(int* device_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_info_once[dev], query_device, dev);
+  if (device_out) *device_out = dev;
+  return &g_info[dev];
+}
+
+}  // namespace fk
+
+extern "C" {
+
+fk_status fk_gelu_tanh(const float* x, float* y, size_t n, void* stream) {
+  if (n == 0) return FK_OK;
+  const fk::DeviceInfo* dev = nullptr;
+  const fk_status st = fk::check_call(x, y, n, sizeof(float), &dev);
+  if (st != FK_OK) return st;
+  const cudaError_t e =
+      fk::launch_gelu_tanh(x, y, n, *dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out) {
+  return fk::plan_softmax(rows, cols, dtype, path, out);
+}
+
+fk_status fk_softmax_rows_ex(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                             const fk_softmax_plan* plan, void* stream) {
+  if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
+  if (rows == 0 || cols == 0) return FK_OK;
+  if (rows > SIZE_MAX / cols) return FK_ERR_INVALID_ARG;
+  fk_softmax_plan p;
+  fk_status st;
+  if (plan == nullptr || plan->path == FK_PATH_AUTO)
+    st = fk::plan_softmax(rows, cols, dtype, FK_PATH_AUTO, &p);
+  else
+    st = fk::check_plan(cols, dtype, *plan, &p);
+  if (st != FK_OK) return st;
+  const size_t esize = dtype == FK_F32 ? 4 : 2;
+  const fk::DeviceInfo* dev = nullptr;
+  st = fk::check_call(x, y, rows * cols, esize, &dev);
+  if (st != FK_OK) return st;
+  // 16-byte vector access needs both bases on a 16-byte boundary and a row
+  // pitch that is a multiple of 16 bytes.
+  const bool aligned = (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(y) % 16 == 0) && ((cols * esize) % 16 == 0);
+  const cudaError_t e =
+      fk::launch_softmax(x, y, rows, cols, dtype, p, aligned, *dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_softmax_rows(const void* x, void* y, size_t rows, size_t cols, int dtype, void* stream) {
+  return fk_softmax_rows_ex(x, y, rows, cols, dtype, nullptr, stream);
+}
+
+const char* fk_status_string(int status) {
+  switch (status) {
+    case FK_OK: return "FK_OK: success";
+    case FK_ERR_INVALID_ARG: return "FK_ERR_INVALID_ARG: invalid argument (pointer, size, alignment, overlap or plan)";
+    case FK_ERR_UNSUPPORTED_DTYPE: return "FK_ERR_UNSUPPORTED_DTYPE: dtype must be FK_F32 or FK_BF16";
+    case FK_ERR_UNSUPPORTED_DEVICE: return "FK_ERR_UNSUPPORTED_DEVICE: no CUDA device, or not sm_100 (B200)";
+    case FK_ERR_CUDA: return "FK_ERR_CUDA: a CUDA call or kernel launch failed (see fk_last_cuda_error)";
+    default: return "unknown fk_status";
+  }
+}
+
+int fk_last_cuda_error(void) { return fk::t_last_cuda_error; }
+
+int fk_version(void) { return fk::kVersion; }
+
+}  // extern "C"

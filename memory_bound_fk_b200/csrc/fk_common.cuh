@@ -1,0 +1,118 @@
+// fk_common.cuh -- device helpers shared by the libfk kernels (sm_100a).
+//
+// Element traits for 16-byte vector I/O (fp32: 4 per vector, bf16: 8 per
+// vector), streaming loads/stores, the base-2 exponential and the warp
+// reductions.  Nothing here is used by, or uses, the CPU oracle.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace fk {
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e), rounded to fp32
+
+// ---------------------------------------------------------------- math
+
+// 2^v with the MUFU.EX2 unit; subnormal results kept (no flush to zero).
+__device__ __forceinline__ float ex2(float v) {
+  float r;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// 2^v, subnormal results flushed to zero (where they cannot matter).
+__device__ __forceinline__ float ex2_ftz(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- I/O
+
+// Read-only, do-not-keep-in-L1 128-bit load.  The memory clobber keeps the
+// compiler from moving it across the stores of the same thread (in-place
+// operation reads an element before it overwrites it).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// 128-bit store with the streaming (evict-first) cache hint.
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+template <typename T>
+struct Elem;
+
+// fp32: 4 values per 16-byte vector.
+template <>
+struct Elem<float> {
+  static constexpr int VEC = 4;
+  __device__ __forceinline__ static void unpack(uint4 v, float* o) {
+    o[0] = __uint_as_float(v.x);
+    o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z);
+    o[3] = __uint_as_float(v.w);
+  }
+  __device__ __forceinline__ static uint4 pack(const float* i) {
+    return make_uint4(__float_as_uint(i[0]), __float_as_uint(i[1]), __float_as_uint(i[2]),
+                      __float_as_uint(i[3]));
+  }
+  __device__ __forceinline__ static float load1(const float* p) { return __ldg(p); }
+  __device__ __forceinline__ static void store1(float* p, float v) { *p = v; }
+};
+
+// bf16 (stored as raw 16-bit patterns): 8 values per 16-byte vector.
+// Widening is exact (the pattern is the top half of an fp32); narrowing
+// rounds to nearest even.
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int VEC = 8;
+  __device__ __forceinline__ static void unpack2(uint32_t w, float* o) {
+    o[0] = __uint_as_float(w << 16);
+    o[1] = __uint_as_float(w & 0xffff0000u);
+  }
+  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x -> low half
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ __forceinline__ static void unpack(uint4 v, float* o) {
+    unpack2(v.x, o + 0);
+    unpack2(v.y, o + 2);
+    unpack2(v.z, o + 4);
+    unpack2(v.w, o + 6);
+  }
+  __device__ __forceinline__ static uint4 pack(const float* i) {
+    return make_uint4(pack2(i[0], i[1]), pack2(i[2], i[3]), pack2(i[4], i[5]), pack2(i[6], i[7]));
+  }
+  __device__ __forceinline__ static float load1(const __nv_bfloat16* p) {
+    const unsigned short b = __ldg(reinterpret_cast<const unsigned short*>(p));
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+  }
+  __device__ __forceinline__ static void store1(__nv_bfloat16* p, float v) {
+    *p = __float2bfloat16_rn(v);
+  }
+};
+
+}  // namespace fk

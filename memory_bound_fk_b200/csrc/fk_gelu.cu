@@ -1,0 +1,101 @@
+// fk_gelu.cu -- elementwise tanh-GELU (CS336 lecture-6 notes, kyc001.github.io,
+// section 4.2), fused into one pass over HBM: one 16-byte load and one
+// 16-byte store per four elements, all arithmetic in registers (the fusion
+// motivation of section 4.1 of the same notes).
+//
+// Arithmetic.  With u = sqrt(2/pi) (x + 0.044715 x^3),
+//     0.5 x (1 + tanh u) = x / (1 + exp(-2u))
+// (multiply numerator and denominator of 1 + tanh u = 2 e^u / (e^u + e^-u)
+// by e^-u).  The kernel evaluates the right-hand side: one MUFU.EX2 for
+// exp(-2u) = 2^(-2 u log2 e) and one correctly rounded fp32 division.  For
+// large positive x, exp(-2u) underflows to 0 and y == x exactly; for large
+// negative x it overflows to +inf and y == -0; the only input where the
+// quotient itself is undefined is x = -inf, which is mapped to the limit -0.
+// The fp32 error stays below ~3 ulp of y (well inside 2e-6 absolute for
+// |y| <= 20), since exp(-2u) only influences y where |x| < ~6.
+#include "fk_common.cuh"
+#include "fk_internal.h"
+
+namespace fk {
+namespace {
+
+constexpr int kGeluThreads = 256;
+constexpr int kGeluUnroll = 4;       // 16-byte vectors in flight per thread
+constexpr int kGeluBlocksPerSm = 8;  // 2048 resident threads per SM
+
+// -2 sqrt(2/pi) log2(e) and that times 0.044715, rounded once to fp32.
+constexpr float kA = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736);
+constexpr float kB = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736 * 0.044715);
+
+__device__ __forceinline__ float gelu_tanh_f32(float x) {
+  const float v = x * fmaf(kB, x * x, kA);  // -2u log2(e)
+  const float t = ex2_ftz(v);                // exp(-2u); a subnormal t cannot change y
+  const float y = __fdiv_rn(x, 1.0f + t);
+  return (x == -INFINITY) ? -0.0f : y;
+}
+
+__device__ __forceinline__ uint4 gelu4(uint4 v) {
+  float f[4];
+  Elem<float>::unpack(v, f);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f[k] = gelu_tanh_f32(f[k]);
+  return Elem<float>::pack(f);
+}
+
+// x, y: the arrays.  Elements [0, head) and [tail_begin, n) are done with
+// scalar accesses; [head, tail_begin) is nvec 16-byte vectors starting at a
+// 16-byte boundary of both x and y.
+__global__ void __launch_bounds__(kGeluThreads)
+    gelu_tanh_kernel(const float* x, float* y, size_t head, size_t nvec, size_t tail_begin,
+                     size_t n) {
+  const size_t tid = static_cast<size_t>(blockIdx.x) * kGeluThreads + threadIdx.x;
+  const size_t nthr = static_cast<size_t>(gridDim.x) * kGeluThreads;
+
+  for (size_t i = tid; i < head; i += nthr) y[i] = gelu_tanh_f32(Elem<float>::load1(x + i));
+  for (size_t i = tail_begin + tid; i < n; i += nthr) y[i] = gelu_tanh_f32(Elem<float>::load1(x + i));
+
+  const char* xv = reinterpret_cast<const char*>(x + head);
+  char* yv = reinterpret_cast<char*>(y + head);
+  // Batches of kGeluUnroll vectors per thread, all loads issued before any
+  // use; the last batch is predicated rather than done one vector at a time.
+  for (size_t base = tid; base < nvec; base += kGeluUnroll * nthr) {
+    uint4 v[kGeluUnroll];
+#pragma unroll
+    for (int u = 0; u < kGeluUnroll; ++u) {
+      const size_t i = base + u * nthr;
+      if (i < nvec) v[u] = ld_stream_v4(xv + i * 16);
+    }
+#pragma unroll
+    for (int u = 0; u < kGeluUnroll; ++u) {
+      const size_t i = base + u * nthr;
+      if (i < nvec) st_stream_v4(yv + i * 16, gelu4(v[u]));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gelu_tanh(const float* x, float* y, size_t n, const DeviceInfo& dev,
+                             cudaStream_t stream) {
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+  size_t head = n, nvec = 0;
+  if ((xa & 15) == (ya & 15)) {  // a common 16-byte phase: peel up to 3 elements
+    head = ((16 - (xa & 15)) & 15) / 4;
+    if (head > n) head = n;
+    nvec = (n - head) / 4;
+  }
+  const size_t tail_begin = head + nvec * 4;
+  const size_t per_block = static_cast<size_t>(kGeluThreads) * kGeluUnroll;
+  size_t blocks = (nvec + per_block - 1) / per_block;
+  const size_t scalar = head > (n - tail_begin) ? head : (n - tail_begin);
+  const size_t scalar_blocks = (scalar + kGeluThreads - 1) / kGeluThreads;
+  if (blocks < scalar_blocks) blocks = scalar_blocks;
+  const size_t cap = static_cast<size_t>(dev.sm_count) * kGeluBlocksPerSm;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  gelu_tanh_kernel<<<static_cast<unsigned>(blocks), kGeluThreads, 0, stream>>>(x, y, head, nvec,
+                                                                               tail_begin, n);
+  return cudaGetLastError();
+}
+
+}  // namespace fk

@@ -1,0 +1,51 @@
+// fk_internal.h -- host-side interfaces between the C ABI (fk_api.cu) and the
+// kernel launchers (fk_gelu.cu, fk_softmax.cu).  Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "fk.h"
+
+namespace fk {
+
+// Cached properties of one device (filled once per device id).
+struct DeviceInfo {
+  int ok;               // 1 if the query succeeded
+  int major, minor;     // compute capability
+  int sm_count;         // multiprocessors
+  int max_threads_sm;   // resident threads per multiprocessor
+  size_t l2_bytes;      // L2 cache size
+};
+
+// Properties of the current device; nullptr if there is none.
+const DeviceInfo* current_device_info(int* device_out);
+
+// ---- GELU --------------------------------------------------------------
+// y[i] = GELU_tanh(x[i]) for i < n.  Arguments already validated.
+cudaError_t launch_gelu_tanh(const float* x, float* y, size_t n, const DeviceInfo& dev,
+                             cudaStream_t stream);
+
+// ---- softmax -----------------------------------------------------------
+constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
+constexpr int kWarpThreads = 32 * kWarpRowsPerBlock;
+constexpr int kBlockElemsPerThread = 32;    // register-resident elements per thread (CTA/cluster)
+constexpr int kTwoPhaseThreads = 512;
+constexpr int kTwoPhaseElemsPerThread = 16; // elements per thread per streamed chunk
+constexpr int kMaxCluster = 16;
+
+// Vectors (16 bytes) per thread implied by a dtype and an element budget.
+int vec_elems(int dtype);  // 4 for fp32, 8 for bf16
+
+// Host-only plan (see fk_softmax_rows_plan in fk.h).
+fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out);
+// Validate a caller-provided plan and fill defaults.
+fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out);
+
+// Launch a validated plan.  `aligned` = rows and both pointers allow 16-byte
+// vector access.
+cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                           const fk_softmax_plan& plan, bool aligned, const DeviceInfo& dev,
+                           cudaStream_t stream);
+
+}  // namespace fk

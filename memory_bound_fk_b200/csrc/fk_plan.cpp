@@ -1,0 +1,148 @@
+// fk_plan.cpp -- host-only choice of the softmax kernel for a row length.
+//
+// The capacities follow from the kernels' register budgets:
+//   warp     : 32 lanes x VPT 16-byte vectors, VPT in {1, 2, 4, 8}
+//              -> up to 1024 fp32 / 2048 bf16 columns
+//   block    : 32 elements per thread, threads in {128, 256, 512, 1024}
+//              -> up to 32768 columns
+//   cluster  : 2..16 blocks of the block kernel -> up to 524288 columns
+//   twophase : any length (row streamed twice)
+// The automatic choice takes the smallest shape that holds the row on chip,
+// so a row is read from HBM once whenever it fits in a cluster.
+#include <stddef.h>
+
+#include "fk_internal.h"
+
+namespace fk {
+
+int vec_elems(int dtype) { return dtype == FK_BF16 ? 8 : 4; }
+
+namespace {
+
+bool valid_dtype(int dtype) { return dtype == FK_F32 || dtype == FK_BF16; }
+
+size_t ceil_div(size_t a, size_t b) { return (a + b - 1) / b; }
+
+bool block_threads_ok(int t) { return t == 128 || t == 256 || t == 512 || t == 1024; }
+
+size_t warp_cap(int dtype, int vpt) { return static_cast<size_t>(32) * vpt * vec_elems(dtype); }
+
+size_t block_cap(int threads) { return static_cast<size_t>(threads) * kBlockElemsPerThread; }
+
+}  // namespace
+
+fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out) {
+  (void)rows;
+  if (!valid_dtype(dtype)) return FK_ERR_UNSUPPORTED_DTYPE;
+  if (out == nullptr || cols == 0) return FK_ERR_INVALID_ARG;
+  if (path == FK_PATH_AUTO) {
+    if (cols <= warp_cap(dtype, 8))
+      path = FK_PATH_WARP;
+    else if (cols <= block_cap(1024))
+      path = FK_PATH_CTA;
+    else if (cols <= static_cast<size_t>(kMaxCluster) * block_cap(1024))
+      path = FK_PATH_CLUSTER;
+    else
+      path = FK_PATH_TWOPHASE;
+  }
+  fk_softmax_plan p = {path, 0, 0, 1};
+  switch (path) {
+    case FK_PATH_WARP: {
+      int vpt = 1;
+      while (vpt < 8 && warp_cap(dtype, vpt) < cols) vpt *= 2;
+      if (warp_cap(dtype, vpt) < cols) return FK_ERR_INVALID_ARG;
+      p.threads = kWarpThreads;
+      p.vpt = vpt;
+      break;
+    }
+    case FK_PATH_CTA: {
+      int t = 128;
+      while (t < 1024 && block_cap(t) < cols) t *= 2;
+      if (block_cap(t) < cols) return FK_ERR_INVALID_ARG;
+      p.threads = t;
+      p.vpt = kBlockElemsPerThread / vec_elems(dtype);
+      break;
+    }
+    case FK_PATH_CLUSTER: {
+      // 512-thread blocks up to 8 per cluster (portable size), then
+      // 1024-thread blocks up to 16 per cluster.
+      size_t k = ceil_div(cols, block_cap(512));
+      int t = 512;
+      if (k > 8) {
+        t = 1024;
+        k = ceil_div(cols, block_cap(1024));
+      }
+      if (k < 2) k = 2;
+      if (k > static_cast<size_t>(kMaxCluster)) return FK_ERR_INVALID_ARG;
+      p.threads = t;
+      p.vpt = kBlockElemsPerThread / vec_elems(dtype);
+      p.cluster = static_cast<int>(k);
+      break;
+    }
+    case FK_PATH_TWOPHASE: {
+      // enough blocks that each streams at most ~64 chunks, capped at 16
+      const size_t chunk = static_cast<size_t>(kTwoPhaseThreads) * kTwoPhaseElemsPerThread;
+      size_t k = ceil_div(cols, chunk * 4);
+      if (k < 1) k = 1;
+      if (k > static_cast<size_t>(kMaxCluster)) k = kMaxCluster;
+      p.threads = kTwoPhaseThreads;
+      p.vpt = kTwoPhaseElemsPerThread / vec_elems(dtype);
+      p.cluster = static_cast<int>(k);
+      break;
+    }
+    default:
+      return FK_ERR_INVALID_ARG;
+  }
+  *out = p;
+  return FK_OK;
+}
+
+fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out) {
+  if (!valid_dtype(dtype)) return FK_ERR_UNSUPPORTED_DTYPE;
+  fk_softmax_plan d;
+  const fk_status st = plan_softmax(1, cols, dtype, in.path, &d);
+  if (st != FK_OK) {
+    // the default for this path may not hold cols, but an explicit plan could
+    if (in.path != FK_PATH_CTA && in.path != FK_PATH_CLUSTER) return st;
+    d.path = in.path;
+    d.threads = 1024;
+    d.vpt = kBlockElemsPerThread / vec_elems(dtype);
+    d.cluster = in.path == FK_PATH_CLUSTER ? kMaxCluster : 1;
+  }
+  fk_softmax_plan p = d;
+  if (in.threads != 0) p.threads = in.threads;
+  if (in.vpt != 0) p.vpt = in.vpt;
+  if (in.cluster != 0) p.cluster = in.cluster;
+  const int vec = vec_elems(dtype);
+  switch (p.path) {
+    case FK_PATH_WARP:
+      if (p.threads != kWarpThreads || p.cluster != 1) return FK_ERR_INVALID_ARG;
+      if (p.vpt != 1 && p.vpt != 2 && p.vpt != 4 && p.vpt != 8) return FK_ERR_INVALID_ARG;
+      if (warp_cap(dtype, p.vpt) < cols) return FK_ERR_INVALID_ARG;
+      break;
+    case FK_PATH_CTA:
+      if (!block_threads_ok(p.threads) || p.cluster != 1) return FK_ERR_INVALID_ARG;
+      if (p.vpt != kBlockElemsPerThread / vec) return FK_ERR_INVALID_ARG;
+      if (block_cap(p.threads) < cols) return FK_ERR_INVALID_ARG;
+      break;
+    case FK_PATH_CLUSTER:
+      if (!block_threads_ok(p.threads) || p.cluster < 2 || p.cluster > kMaxCluster)
+        return FK_ERR_INVALID_ARG;
+      if (p.vpt != kBlockElemsPerThread / vec) return FK_ERR_INVALID_ARG;
+      // each block's slice, ceil(vectors / cluster), must fit its registers
+      if (ceil_div(ceil_div(cols, vec), p.cluster) * vec > block_cap(p.threads))
+        return FK_ERR_INVALID_ARG;
+      break;
+    case FK_PATH_TWOPHASE:
+      if (p.threads != kTwoPhaseThreads || p.vpt != kTwoPhaseElemsPerThread / vec)
+        return FK_ERR_INVALID_ARG;
+      if (p.cluster < 1 || p.cluster > kMaxCluster) return FK_ERR_INVALID_ARG;
+      break;
+    default:
+      return FK_ERR_INVALID_ARG;
+  }
+  *out = p;
+  return FK_OK;
+}
+
+}  // namespace fk

@@ -1,0 +1,483 @@
+// fk_softmax.cu -- row softmax kernels for sm_100a.
+//
+// What is computed (lecture 6, "GPU Kernels and Triton", cs336.sjfarmltd.com,
+// section 7.2; CS336 lecture-6 notes, kyc001.github.io, section 5.2): for each
+// row of a row-major [rows, cols] matrix, m = max_j x_j, l = sum_j exp(x_j - m),
+// y_j = exp(x_j - m) / l.  exp(v) is evaluated as 2^(v log2 e) on MUFU.EX2 and
+// the division as a multiplication by the correctly rounded 1/l.
+//
+// Four kernel shapes, chosen by row length (see fk_plan.cpp):
+//   warp     -- one warp per row; the row sits in registers (up to 32 vectors
+//               per lane-row, i.e. 1024 fp32 / 2048 bf16 columns);
+//               max and sum by warp shuffles.
+//   block    -- one thread block per row, 32 register-resident elements per
+//               thread (up to 32768 columns); warp shuffles, then one shared
+//               memory exchange between warps.
+//   cluster  -- the same block kernel launched as a thread-block cluster of
+//               2..16 blocks per row; each block reduces its slice to a
+//               partial (m_c, l_c) and the partials are merged over
+//               distributed shared memory with the running-max rule of
+//               section 7.2:  M = max_c m_c,  L = sum_c l_c exp(m_c - M).
+//               Every element is still read once and written once.
+//   twophase -- for rows longer than a cluster can hold: each block streams
+//               its slice, keeping a per-thread running (m, l) (the online
+//               recurrence of section 7.2), merges as above, then streams the
+//               slice again to write exp(x - M) / L.  Three HBM transfers per
+//               element instead of two.
+//
+// Placement within a row: a team of TEAM threads (a warp or a block) covers
+// the row (or its slice) in chunks of TEAM 16-byte vectors.  On the vector
+// path, thread t owns vector (chunk * TEAM + t), so a warp's loads are 512
+// contiguous bytes.  When rows or pointers are not 16-byte aligned, the
+// scalar path keeps the same chunks but gives thread t the elements
+// chunk*TEAM*VEC + k*TEAM + t (k < VEC), which is again contiguous per warp.
+//
+// Special values: padding lanes hold -inf (exp gives 0, never stored);
+// -inf inputs give exactly 0; a row that is all -inf gives 0/0 = NaN; a NaN
+// is skipped by fmaxf but poisons the sum; a +inf gives inf - inf = NaN.
+// Partial results of slices that are all -inf are merged without forming
+// (-inf) - (-inf): see rescale().
+#include <cuda_bf16.h>
+
+#include "fk_common.cuh"
+#include "fk_internal.h"
+
+namespace fk {
+namespace {
+
+template <typename I>
+__device__ __forceinline__ I imin(I a, I b) {
+  return a < b ? a : b;
+}
+
+// ---------------------------------------------------------------- cluster PTX
+
+__device__ __forceinline__ unsigned cluster_ctarank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ unsigned cluster_nctarank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Full cluster barrier: release this block's shared-memory writes, acquire
+// the other blocks'.  Every thread of every block of the cluster calls it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release;\n\t"
+      "barrier.cluster.wait.acquire;" ::
+          : "memory");
+}
+
+// Load a float2 from the shared memory of block `rank` of this cluster, at
+// the offset of `local` in this block's shared memory.
+__device__ __forceinline__ float2 ld_dsmem_f2(const float2* local, unsigned rank) {
+  const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(local));
+  unsigned ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(ra) : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------- merge rule
+
+// exp(m_from - m_to) for m_from <= m_to: the factor that moves a partial sum
+// taken relative to max m_from onto max m_to.  Equal maxima give exactly 1,
+// which also covers (-inf, -inf) (an all -inf partial, whose sum is 0) and
+// (+inf, +inf) (whose sum is already NaN).
+__device__ __forceinline__ float rescale(float m_from, float m_to) {
+  return (m_from == m_to) ? 1.0f : ex2((m_from - m_to) * kLog2e);
+}
+
+// Reference point for exponentials of a partial whose max is m: m itself,
+// or 0 for an all -inf partial (so that exp(-inf - ref) = 0, not NaN).
+__device__ __forceinline__ float exp_ref(float m) { return (m == -INFINITY) ? 0.0f : m; }
+
+// ---------------------------------------------------------------- row I/O
+
+// Load VPT chunks of a team slice into registers (VPT * VEC floats).
+// Vectors [vb, ve) of the row are the slice; anything outside is -inf.
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+__device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, int t,
+                                            float* v) {
+  constexpr int VEC = Elem<T>::VEC;
+#pragma unroll
+  for (int c = 0; c < VPT; ++c) {
+    if constexpr (ALIGNED) {
+      const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
+      if (vi < ve) {
+        Elem<T>::unpack(ld_stream_v4(row + static_cast<size_t>(vi) * VEC), v + c * VEC);
+      } else {
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) v[c * VEC + k] = -INFINITY;
+      }
+    } else {
+      const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
+      const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) {
+        const Idx e = e0 + static_cast<Idx>(k) * TEAM;
+        v[c * VEC + k] = (e < eend) ? Elem<T>::load1(row + e) : -INFINITY;
+      }
+    }
+  }
+}
+
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+__device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx cols, int t,
+                                             const float* v) {
+  constexpr int VEC = Elem<T>::VEC;
+#pragma unroll
+  for (int c = 0; c < VPT; ++c) {
+    if constexpr (ALIGNED) {
+      const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
+      if (vi < ve) st_stream_v4(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(v + c * VEC));
+    } else {
+      const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
+      const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) {
+        const Idx e = e0 + static_cast<Idx>(k) * TEAM;
+        if (e < eend) Elem<T>::store1(row + e, v[c * VEC + k]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- warp path
+
+template <typename T, int VPT, bool ALIGNED>
+__global__ void __launch_bounds__(kWarpThreads)
+    softmax_warp_kernel(const T* x, T* y, size_t rows, int cols) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int E = VPT * VEC;
+  const int lane = threadIdx.x & 31;
+  const int nvec = (cols + VEC - 1) / VEC;
+  const size_t stride = static_cast<size_t>(gridDim.x) * kWarpRowsPerBlock;
+  for (size_t row = static_cast<size_t>(blockIdx.x) * kWarpRowsPerBlock + (threadIdx.x >> 5);
+       row < rows; row += stride) {
+    const T* xr = x + row * static_cast<size_t>(cols);
+    T* yr = y + row * static_cast<size_t>(cols);
+    float v[E];
+    load_chunks<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, v);
+
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; ++e) m = fmaxf(m, v[e]);
+    m = warp_max(m);
+
+    // One reference m for the whole row: the rounding of m*log2(e) is a
+    // common factor of every exponential and of their sum, so it cancels.
+    const float mL = m * kLog2e;
+    float s = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      v[e] = ex2(fmaf(v[e], kLog2e, -mL));
+      s += v[e];
+    }
+    s = warp_sum(s);
+    const float r = __frcp_rn(s);
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] *= r;
+    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v);
+  }
+}
+
+// ---------------------------------------------------------------- block / cluster path
+
+// CLUSTER = false: one block per row.  CLUSTER = true: launched as clusters
+// of 2..16 blocks; block `rank` of a cluster holds vectors
+// [rank*per, (rank+1)*per) of the row, per = ceil(nvec / cluster size).
+template <typename T, int THREADS, bool ALIGNED, bool CLUSTER>
+__global__ void __launch_bounds__(THREADS)
+    softmax_block_kernel(const T* x, T* y, size_t rows, int cols) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int VPT = kBlockElemsPerThread / VEC;
+  constexpr int E = VPT * VEC;
+  constexpr int NW = THREADS / 32;
+  __shared__ float red_max[NW];
+  __shared__ float red_sum[NW];
+  __shared__ float2 part[2];  // this block's (max, sum), double-buffered by row parity
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int csize = CLUSTER ? static_cast<int>(cluster_nctarank()) : 1;
+  const int crank = CLUSTER ? static_cast<int>(cluster_ctarank()) : 0;
+  const int nvec = (cols + VEC - 1) / VEC;
+  const int per = (nvec + csize - 1) / csize;
+  const int vb = imin(nvec, crank * per);
+  const int ve = imin(nvec, vb + per);
+
+  const size_t stride = gridDim.x / csize;
+  int parity = 0;
+  for (size_t row = blockIdx.x / csize; row < rows; row += stride, parity ^= 1) {
+    const T* xr = x + row * static_cast<size_t>(cols);
+    T* yr = y + row * static_cast<size_t>(cols);
+    float v[E];
+    load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, v);
+
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; ++e) m = fmaxf(m, v[e]);
+    m = warp_max(m);
+    if (lane == 0) red_max[warp] = m;
+    __syncthreads();
+    m = red_max[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
+
+    float s = 0.0f;
+    if constexpr (CLUSTER) {
+      // Blocks use different references, so take the exponent difference
+      // exactly-ish ((x - ref) rounds relative to |x - ref|, which is 0 for
+      // the largest terms) instead of folding ref*log2(e) into an FMA.
+      const float ref = exp_ref(m);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        v[e] = ex2((v[e] - ref) * kLog2e);
+        s += v[e];
+      }
+    } else {
+      const float mL = m * kLog2e;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        v[e] = ex2(fmaf(v[e], kLog2e, -mL));
+        s += v[e];
+      }
+    }
+    s = warp_sum(s);
+    if (lane == 0) red_sum[warp] = s;
+    __syncthreads();
+    s = red_sum[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) s += red_sum[w];
+
+    float scale;
+    if constexpr (CLUSTER) {
+      if (t == 0) part[parity] = make_float2(m, s);
+      cluster_sync_all();
+      // every warp merges the cluster's partials itself: lane i reads block i
+      float mi = -INFINITY, li = 0.0f;
+      if (lane < csize) {
+        const float2 p = ld_dsmem_f2(&part[parity], static_cast<unsigned>(lane));
+        mi = p.x;
+        li = p.y;
+      }
+      const float M = warp_max(mi);
+      const float L = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
+      scale = rescale(m, M) * __frcp_rn(L);
+    } else {
+      scale = __frcp_rn(s);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] *= scale;
+    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v);
+    __syncthreads();  // red_max / red_sum are rewritten by the next row
+  }
+  if constexpr (CLUSTER) cluster_sync_all();  // keep `part` alive until all readers are done
+}
+
+// ---------------------------------------------------------------- two-phase path
+
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+  const float M = fmaxf(m, m2);
+  l = l * rescale(m, M) + l2 * rescale(m2, M);
+  m = M;
+}
+
+template <typename T, bool ALIGNED>
+__global__ void __launch_bounds__(kTwoPhaseThreads)
+    softmax_twophase_kernel(const T* x, T* y, size_t rows, size_t cols) {
+  constexpr int THREADS = kTwoPhaseThreads;
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
+  constexpr int E = VPT * VEC;
+  constexpr int NW = THREADS / 32;
+  constexpr size_t CHUNK = static_cast<size_t>(THREADS) * VPT;  // vectors per chunk
+  __shared__ float2 red[NW];
+  __shared__ float2 part[2];
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int csize = static_cast<int>(cluster_nctarank());  // 1 without a cluster launch
+  const int crank = static_cast<int>(cluster_ctarank());
+  const size_t nvec = (cols + VEC - 1) / VEC;
+  const size_t per = (nvec + csize - 1) / csize;
+  const size_t vb = imin(nvec, static_cast<size_t>(crank) * per);
+  const size_t ve = imin(nvec, vb + per);
+
+  const size_t stride = gridDim.x / csize;
+  int parity = 0;
+  for (size_t row = blockIdx.x / csize; row < rows; row += stride, parity ^= 1) {
+    const T* xr = x + row * cols;
+    T* yr = y + row * cols;
+
+    // pass 1: running (m, l) per thread over the streamed chunks
+    float m = -INFINITY, l = 0.0f;
+    for (size_t c = vb; c < ve; c += CHUNK) {
+      float v[E];
+      load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
+      float cm = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < E; ++e) cm = fmaxf(cm, v[e]);
+      const float mn = fmaxf(m, cm);
+      const float ref = exp_ref(mn);
+      float acc = 0.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc += ex2((v[e] - ref) * kLog2e);
+      l = l * rescale(m, mn) + acc;
+      m = mn;
+    }
+
+    // merge the threads' partials: warp, then block
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      merge_ml(m, l, m2, l2);
+    }
+    if (lane == 0) red[warp] = make_float2(m, l);
+    __syncthreads();
+    m = red[0].x;
+    l = red[0].y;
+#pragma unroll
+    for (int w = 1; w < NW; ++w) merge_ml(m, l, red[w].x, red[w].y);
+
+    // merge the blocks' partials across the cluster
+    if (csize > 1) {
+      if (t == 0) part[parity] = make_float2(m, l);
+      cluster_sync_all();
+      float mi = -INFINITY, li = 0.0f;
+      if (lane < csize) {
+        const float2 p = ld_dsmem_f2(&part[parity], static_cast<unsigned>(lane));
+        mi = p.x;
+        li = p.y;
+      }
+      const float M = warp_max(mi);
+      l = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
+      m = M;
+    }
+
+    // pass 2: y = exp(x - M) / L
+    const float r = __frcp_rn(l);
+    const float ref = exp_ref(m);
+    for (size_t c = vb; c < ve; c += CHUNK) {
+      float v[E];
+      load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = ex2((v[e] - ref) * kLog2e) * r;
+      store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v);
+    }
+    __syncthreads();  // red is rewritten by the next row
+  }
+  if (csize > 1) cluster_sync_all();
+}
+
+// ---------------------------------------------------------------- launch helpers
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), size_t blocks, int threads, int cluster,
+                   cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;
+  if (cluster > 1) {
+    if (cluster > 8) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+constexpr size_t kMaxGrid = 0x7fffffffu;
+
+template <typename T, bool ALIGNED>
+cudaError_t launch_warp(const void* x, void* y, size_t rows, size_t cols, int vpt,
+                        cudaStream_t s) {
+  size_t blocks = (rows + kWarpRowsPerBlock - 1) / kWarpRowsPerBlock;
+  if (blocks > kMaxGrid) blocks = kMaxGrid;
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
+  const int c = static_cast<int>(cols);
+  switch (vpt) {
+    case 1: return launch(softmax_warp_kernel<T, 1, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
+    case 2: return launch(softmax_warp_kernel<T, 2, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
+    case 4: return launch(softmax_warp_kernel<T, 4, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
+    case 8: return launch(softmax_warp_kernel<T, 8, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T, bool ALIGNED, bool CLUSTER>
+cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int threads,
+                         int cluster, cudaStream_t s) {
+  const size_t cl = CLUSTER ? static_cast<size_t>(cluster) : 1;
+  size_t groups = rows;
+  if (groups > kMaxGrid / cl) groups = kMaxGrid / cl;
+  const size_t blocks = groups * cl;
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
+  const int c = static_cast<int>(cols);
+  const int k = static_cast<int>(cl);
+  switch (threads) {
+    case 128: return launch(softmax_block_kernel<T, 128, ALIGNED, CLUSTER>, blocks, 128, k, s, xp, yp, rows, c);
+    case 256: return launch(softmax_block_kernel<T, 256, ALIGNED, CLUSTER>, blocks, 256, k, s, xp, yp, rows, c);
+    case 512: return launch(softmax_block_kernel<T, 512, ALIGNED, CLUSTER>, blocks, 512, k, s, xp, yp, rows, c);
+    case 1024: return launch(softmax_block_kernel<T, 1024, ALIGNED, CLUSTER>, blocks, 1024, k, s, xp, yp, rows, c);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T, bool ALIGNED>
+cudaError_t launch_twophase(const void* x, void* y, size_t rows, size_t cols, int cluster,
+                            cudaStream_t s) {
+  const size_t cl = static_cast<size_t>(cluster);
+  size_t groups = rows;
+  if (groups > kMaxGrid / cl) groups = kMaxGrid / cl;
+  return launch(softmax_twophase_kernel<T, ALIGNED>, groups * cl, kTwoPhaseThreads, cluster, s,
+                static_cast<const T*>(x), static_cast<T*>(y), rows, cols);
+}
+
+template <typename T, bool ALIGNED>
+cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
+                         const fk_softmax_plan& p, cudaStream_t s) {
+  switch (p.path) {
+    case FK_PATH_WARP: return launch_warp<T, ALIGNED>(x, y, rows, cols, p.vpt, s);
+    case FK_PATH_CTA: return launch_block<T, ALIGNED, false>(x, y, rows, cols, p.threads, 1, s);
+    case FK_PATH_CLUSTER:
+      return launch_block<T, ALIGNED, true>(x, y, rows, cols, p.threads, p.cluster, s);
+    case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED>(x, y, rows, cols, p.cluster, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                           const fk_softmax_plan& plan, bool aligned, const DeviceInfo& dev,
+                           cudaStream_t stream) {
+  (void)dev;
+  if (dtype == FK_F32) {
+    return aligned ? launch_typed<float, true>(x, y, rows, cols, plan, stream)
+                   : launch_typed<float, false>(x, y, rows, cols, plan, stream);
+  }
+  return aligned ? launch_typed<__nv_bfloat16, true>(x, y, rows, cols, plan, stream)
+                 : launch_typed<__nv_bfloat16, false>(x, y, rows, cols, plan, stream);
+}
+
+}  // namespace fk

@@ -266,3 +266,21 @@ def causal_scores(heads: int, t: int, sigma: float, seed: int) -> np.ndarray:
             b[i, i + 1:] = NEG_INF_BF16
         x[h * t:(h + 1) * t] = b
     return x
+
+
+def softmax_input(rows: int, cols: int, dtype: str = "f32", sigma: float = 4.0,
+                  neg_inf_frac: float = 0.0, seed: int = 0, shift: float = 0.0) -> np.ndarray:
+    """Generic row-softmax test input: N(shift, sigma^2) entries, and in each
+    row round(neg_inf_frac * cols) positions (without replacement) set to
+    -inf.  fp32 array, or bf16 bits."""
+    g = np.random.default_rng(seed)
+    x = (g.standard_normal((rows, cols)) * sigma + shift).astype(np.float32)
+    k = int(round(neg_inf_frac * cols))
+    if k:
+        for r in range(rows):
+            x[r, g.choice(cols, size=k, replace=False)] = -np.inf
+    if dtype == "f32":
+        return x
+    b = f32_to_bf16_bits(np.where(np.isneginf(x), 0.0, x))
+    b[np.isneginf(x)] = NEG_INF_BF16
+    return b

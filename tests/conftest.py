@@ -19,3 +19,13 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("test marked gpu but no CUDA device is visible")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def fk():
+    """The binding, with libfk.so built in-tree first (a no-op when current)."""
+    from memory_bound_fk_b200 import build
+    build.build()
+    import memory_bound_fk_b200 as m
+    m.lib()
+    return m

@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: exports, status strings, planning, and the
+argument checks that must reject a call before anything is launched."""
+import ctypes
+
+import pytest
+
+
+def test_library_exports_every_declared_entry_point(fk):
+    names = fk.header_functions()
+    assert set(names) >= {"fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex",
+                          "fk_softmax_rows_plan", "fk_status_string", "fk_last_cuda_error",
+                          "fk_version"}
+    lib = ctypes.CDLL(fk.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(fk):
+    assert fk.fk_version() == 10000
+    for code, word in [(0, "FK_OK"), (1, "INVALID_ARG"), (2, "DTYPE"), (3, "DEVICE"), (4, "CUDA")]:
+        assert word in fk.fk_status_string(code)
+    assert "unknown" in fk.fk_status_string(99)
+
+
+@pytest.mark.parametrize("rows,cols,dtype,expect", [
+    (256, 1000, 0, ("warp", 256, 8, 1)),        # 256x1000 fp32
+    (8192, 4096, 0, ("cta", 128, 8, 1)),        # 8192x4096 fp32
+    (1 << 20, 2048, 1, ("warp", 256, 8, 1)),    # bf16 attention rows
+    (512, 131072, 0, ("cluster", 512, 8, 8)),   # vocab-sized rows
+    (4, 1, 0, ("warp", 256, 1, 1)),
+    (4, 128, 0, ("warp", 256, 1, 1)),
+    (4, 129, 0, ("warp", 256, 2, 1)),
+    (4, 1024, 0, ("warp", 256, 8, 1)),
+    (4, 1025, 0, ("cta", 128, 8, 1)),
+    (4, 2049, 1, ("cta", 128, 4, 1)),
+    (4, 32768, 0, ("cta", 1024, 8, 1)),
+    (4, 32769, 0, ("cluster", 512, 8, 3)),
+    (4, 131073, 0, ("cluster", 1024, 8, 5)),
+    (4, 524288, 0, ("cluster", 1024, 8, 16)),
+    (4, 524289, 0, ("twophase", 512, 4, 16)),
+    (4, 524289, 1, ("twophase", 512, 2, 16)),
+    (4, 524288, 1, ("cluster", 1024, 4, 16)),
+])
+def test_auto_plans(fk, rows, cols, dtype, expect):
+    p = fk.fk_softmax_rows_plan(rows, cols, dtype).as_dict()
+    assert (p["path"], p["threads"], p["vpt"], p["cluster"]) == expect
+
+
+def test_forced_plans_and_capacity_errors(fk):
+    P = fk
+    assert P.fk_softmax_rows_plan(2, 100, 0, P.FK_PATH_TWOPHASE).as_dict()["cluster"] == 1
+    assert P.fk_softmax_rows_plan(2, 100, 0, P.FK_PATH_CLUSTER).as_dict()["cluster"] == 2
+    assert P.fk_softmax_rows_plan(2, 100, 0, P.FK_PATH_CTA).as_dict()["threads"] == 128
+    with pytest.raises(P.FkError):
+        P.fk_softmax_rows_plan(2, 1025, 0, P.FK_PATH_WARP)
+    with pytest.raises(P.FkError):
+        P.fk_softmax_rows_plan(2, 32769, 0, P.FK_PATH_CTA)
+    with pytest.raises(P.FkError):
+        P.fk_softmax_rows_plan(2, 16 * 32768 + 1, 0, P.FK_PATH_CLUSTER)
+    with pytest.raises(P.FkError) as e:
+        P.fk_softmax_rows_plan(2, 10, 7)
+    assert e.value.status == P.FK_ERR_UNSUPPORTED_DTYPE
+    with pytest.raises(P.FkError):
+        P.fk_softmax_rows_plan(2, 0, 0)
+
+
+# Fake addresses: never dereferenced.  Without a GPU the checks end at
+# "no device"; on a GPU machine the pointer-attribute query rejects them.
+A, B = 0x10000000, 0x20000000
+REJECT_NO_LAUNCH = {1, 3}
+
+
+def test_zero_sizes_are_noops_even_with_null(fk):
+    assert fk.fk_gelu_tanh(0, 0, 0, 0) == fk.FK_OK
+    assert fk.fk_softmax_rows(0, 0, 0, 10, 0, 0) == fk.FK_OK
+    assert fk.fk_softmax_rows(0, 0, 10, 0, 1, 0) == fk.FK_OK
+
+
+def test_null_pointers_with_nonzero_size(fk):
+    assert fk.fk_gelu_tanh(0, B, 10, 0) == fk.FK_ERR_INVALID_ARG
+    assert fk.fk_gelu_tanh(A, 0, 10, 0) == fk.FK_ERR_INVALID_ARG
+    assert fk.fk_softmax_rows(0, B, 4, 4, 0, 0) == fk.FK_ERR_INVALID_ARG
+
+
+def test_bad_dtype_is_reported_first(fk):
+    assert fk.fk_softmax_rows(A, B, 4, 4, 2, 0) == fk.FK_ERR_UNSUPPORTED_DTYPE
+    assert fk.fk_softmax_rows(A, B, 0, 4, -1, 0) == fk.FK_ERR_UNSUPPORTED_DTYPE
+
+
+def test_misaligned_and_overflowing_and_overlapping_arguments(fk):
+    assert fk.fk_gelu_tanh(A + 1, B, 10, 0) == fk.FK_ERR_INVALID_ARG          # not 4-byte aligned
+    assert fk.fk_softmax_rows(A, B + 1, 4, 4, 1, 0) == fk.FK_ERR_INVALID_ARG  # bf16, odd address
+    assert fk.fk_softmax_rows(A, B, 1 << 62, 1 << 3, 0, 0) == fk.FK_ERR_INVALID_ARG  # bytes overflow
+    assert fk.fk_gelu_tanh(A, A + 4, 16, 0) == fk.FK_ERR_INVALID_ARG         # partial overlap
+    assert fk.fk_softmax_rows(A, A + 64, 4, 32, 0, 0) == fk.FK_ERR_INVALID_ARG
+
+
+def test_valid_looking_arguments_without_a_usable_device_are_rejected(fk):
+    assert fk.fk_gelu_tanh(A, B, 10, 0) in REJECT_NO_LAUNCH
+    assert fk.fk_gelu_tanh(A, A, 10, 0) in REJECT_NO_LAUNCH                   # in place
+    assert fk.fk_softmax_rows(A, B, 4, 4, 0, 0) in REJECT_NO_LAUNCH
+
+
+def test_explicit_plan_validation(fk):
+    bad = [fk.make_plan(fk.FK_PATH_WARP, threads=128),
+           fk.make_plan(fk.FK_PATH_WARP, vpt=3),
+           fk.make_plan(fk.FK_PATH_CTA, threads=96),
+           fk.make_plan(fk.FK_PATH_CLUSTER, cluster=17),
+           fk.make_plan(fk.FK_PATH_CLUSTER, cluster=1),
+           fk.make_plan(fk.FK_PATH_TWOPHASE, threads=256),
+           fk.make_plan(9)]
+    for p in bad:
+        assert fk.fk_softmax_rows_ex(A, B, 4, 64, 0, p, 0) == fk.FK_ERR_INVALID_ARG, p
+    # a plan that cannot hold the row
+    assert fk.fk_softmax_rows_ex(A, B, 4, 5000, 0, fk.make_plan(fk.FK_PATH_CTA, threads=128), 0) \
+        == fk.FK_ERR_INVALID_ARG
