@@ -37,6 +37,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -46,13 +48,6 @@ UNIT = "GB/s"
 SUITE = ["cfg2_gelu", "cfg3_softmax", "cfg4_softmax", "cfg5_softmax"]
 SPEC_HBM_GBS = 8000.0          # nominal B200 HBM3e bandwidth
 FALLBACK_HBM_GBS = 6650.0      # earlier copy measurement on this B200 pool
-KERNEL_NAMES = {               # kernel that each workload's auto plan launches
-    "cfg1_gelu": "gelu_tanh_kernel", "cfg2_gelu": "gelu_tanh_kernel",
-    "cfg1_softmax": "softmax_warp_kernel<float,8>",
-    "cfg3_softmax": "softmax_block_kernel<float,128>",
-    "cfg4_softmax": "softmax_warp_kernel<bf16,8>",
-    "cfg5_softmax": "softmax_block_kernel<float,512,cluster 8>",
-}
 
 
 def log(*a):
@@ -60,6 +55,21 @@ def log(*a):
 
 
 # ---------------------------------------------------------------- host logic
+
+def kernel_name(w, plan: dict) -> str:
+    """The libfk kernel a workload's plan launches."""
+    if w.op == "gelu":
+        return "gelu_tanh_kernel"
+    t = "bf16" if w.dtype == "bf16" else "float"
+    vec = 8 if w.dtype == "bf16" else 4
+    p = plan["path"]
+    if p == "warp":
+        return f"softmax_warp_kernel<{t},vpt={plan['vpt']}>"
+    if p in ("cta", "cluster"):
+        extra = f",cluster={plan['cluster']}" if p == "cluster" else ""
+        return f"softmax_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{extra}>"
+    return f"softmax_twophase_kernel<{t},cluster={plan['cluster']}>"
+
 
 def hbm_traffic_bytes(tensor_bytes: int, n_elementwise_ops: int, fused: bool) -> int:
     """HBM bytes of n elementwise ops over one tensor: each unfused op reads
@@ -227,12 +237,12 @@ def host_threads() -> int:
         return os.cpu_count() or 1
 
 
-def make_inputs(names):
+def make_inputs(names, rows=None):
     from memory_bound_fk_b200 import synth
     out = {}
     for n in names:
         t = time.perf_counter()
-        out[n] = synth.make(n)
+        out[n] = np.ascontiguousarray(synth.make(n, rows=rows))
         log(f"[bench] generated {n} {out[n].shape} in {time.perf_counter() - t:.1f}s")
     return out
 
@@ -257,7 +267,8 @@ def run_ours(args) -> dict | None:
                                 device_id=device)
     fk.lib()  # fail loudly if libfk.so is missing
     names = workload_list(args.workload)
-    host = make_inputs(names)
+    host = make_inputs(names, args.rows)
+    shapes = {n: host[n].shape for n in names}
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
 
@@ -273,14 +284,14 @@ def run_ours(args) -> dict | None:
         dev_out[n] = torch.empty_like(dev_in[n])
         xp, yp = dev_in[n].data_ptr(), dev_out[n].data_ptr()
         if w.op == "gelu":
-            calls.append((n, lambda xp=xp, yp=yp, k=w.numel: fk.fk_gelu_tanh(xp, yp, k, sh)))
+            calls.append((n, lambda xp=xp, yp=yp, k=host[n].size: fk.fk_gelu_tanh(xp, yp, k, sh)))
         else:
-            r, c = w.shape
+            r, c = shapes[n]
             code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
             calls.append((n, lambda xp=xp, yp=yp, r=r, c=c, code=code:
                           fk.fk_softmax_rows(xp, yp, r, c, code, sh)))
-    bytes_step = sum(synth.WORKLOADS[n].algorithmic_bytes for n in names)
-    elems_step = sum(synth.WORKLOADS[n].numel for n in names)
+    bytes_step = sum(2 * host[n].nbytes for n in names)
+    elems_step = sum(host[n].size for n in names)
 
     def step(evs=None):
         for i, (n, call) in enumerate(calls):
@@ -344,16 +355,17 @@ def run_ours(args) -> dict | None:
     for i, n in enumerate(names):
         w = synth.WORKLOADS[n]
         ms = kernel_ms[i] / args.steps
-        gbs = w.algorithmic_bytes / (ms * 1e-3) / 1e9
-        plan = (fk.fk_softmax_rows_plan(w.shape[0], w.shape[1],
+        nbytes = 2 * host[n].nbytes
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        plan = (fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1],
                                         fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32).as_dict()
                 if w.op == "softmax" else {"path": "gelu"})
-        kernels.append({"workload": n, "kernel": KERNEL_NAMES.get(n), "plan": plan,
-                        "ms": round(ms, 5), "GB_s": round(gbs, 1),
-                        "elements_per_s": round(w.numel / (ms * 1e-3), 1),
+        kernels.append({"workload": n, "kernel": kernel_name(w, plan), "plan": plan,
+                        "shape": list(shapes[n]), "ms": round(ms, 5), "GB_s": round(gbs, 1),
+                        "elements_per_s": round(host[n].size / (ms * 1e-3), 1),
                         "pct_of_8TBs": round(100 * gbs / SPEC_HBM_GBS, 2),
                         "frac_of_measured_copy": round(gbs / peaks["hbm_gbs"], 4),
-                        "bytes_per_launch": w.algorithmic_bytes})
+                        "bytes_per_launch": nbytes})
     dom = max(range(len(names)), key=lambda i: kernel_ms[i])
     dk = kernels[dom]
     traffic, traffic_src = profiled_traffic(names[dom])
@@ -363,7 +375,8 @@ def run_ours(args) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "detail": describe(names),
+        "config": {"workload": args.workload if args.rows is None else f"{args.workload} (leading {args.rows} rows)",
+                   "detail": describe(names),
                    "io_dtypes": sorted({synth.WORKLOADS[n].dtype for n in names}),
                    "bytes_per_step_per_gpu": bytes_step, "elements_per_step_per_gpu": elems_step,
                    "l2": f"inputs larger than L2: {bytes_step // 2 / 1e9:.2f} GB read per step",
@@ -434,7 +447,7 @@ def run_reference(args) -> dict | None:
     if rank != 0:
         return None
     names = workload_list(args.workload)
-    host = make_inputs(names)
+    host = make_inputs(names, args.rows)
     threads = host_threads()
     per_step = args.reference_budget / max(1, args.steps + args.warmup)
     f = oracle_sample_plan(names, host, per_step, threads)
@@ -454,7 +467,8 @@ def run_reference(args) -> dict | None:
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "detail": describe(names),
+        "config": {"workload": args.workload if args.rows is None else f"{args.workload} (leading {args.rows} rows)",
+                   "detail": describe(names),
                    "parallelism": "host cores (oracle)"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -474,6 +488,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
                         "cfg3_softmax, cfg4_softmax, cfg5_softmax")
+    p.add_argument("--rows", type=int, default=None,
+                   help="profiling only: leading rows (elements for GELU) of each workload")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-cpu-baseline", action="store_true")

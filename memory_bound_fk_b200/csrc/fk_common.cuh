@@ -62,6 +62,41 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
                : "memory");
 }
 
+// Predicated forms: the access happens only when `pred` holds (the address
+// is not touched otherwise).  Keeping the predicate inside one asm statement,
+// instead of branching around the access, lets the compiler interleave the
+// stores with the arithmetic that produces them; with branches it hoists all
+// of that arithmetic first and the register count of the row kernels nearly
+// doubles.  A load that does not happen returns `fill` in every word.
+__device__ __forceinline__ uint4 ld_stream_v4_if(const void* p, bool pred, uint32_t fill) {
+  uint4 v = make_uint4(fill, fill, fill, fill);
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t"
+      "@q ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "l"(p), "r"(static_cast<unsigned>(pred))
+      : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_stream_v4_if(void* p, uint4 v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t"
+      "@q st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};\n\t}" ::"l"(p),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(static_cast<unsigned>(pred))
+      : "memory");
+}
+
+// Max / sum of E register values with four independent accumulators, so the
+// dependency chain is E/4 long instead of E.
+template <int E>
+__device__ __forceinline__ float max_of(const float* v) {
+  float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int e = 0; e < E; ++e) a[e & 3] = fmaxf(a[e & 3], v[e]);
+  return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+}
+
 template <typename T>
 struct Elem;
 
@@ -69,6 +104,7 @@ struct Elem;
 template <>
 struct Elem<float> {
   static constexpr int VEC = 4;
+  static constexpr uint32_t kNegInfWord = 0xff800000u;  // one -inf
   __device__ __forceinline__ static void unpack(uint4 v, float* o) {
     o[0] = __uint_as_float(v.x);
     o[1] = __uint_as_float(v.y);
@@ -89,6 +125,7 @@ struct Elem<float> {
 template <>
 struct Elem<__nv_bfloat16> {
   static constexpr int VEC = 8;
+  static constexpr uint32_t kNegInfWord = 0xff80ff80u;  // two -inf
   __device__ __forceinline__ static void unpack2(uint32_t w, float* o) {
     o[0] = __uint_as_float(w << 16);
     o[1] = __uint_as_float(w & 0xffff0000u);

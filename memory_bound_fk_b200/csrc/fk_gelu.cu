@@ -19,9 +19,14 @@
 namespace fk {
 namespace {
 
+// One block covers kGeluThreads * kGeluUnroll consecutive 16-byte vectors and
+// each thread loads its kGeluUnroll vectors before using any.  Measured on
+// B200 for 32 MiB (L2 cleaned between runs), this one-batch-per-thread grid
+// matches cudaMemcpy's time for the same bytes, while grid-stride loops over
+// a resident grid were 20% slower.
 constexpr int kGeluThreads = 256;
-constexpr int kGeluUnroll = 4;       // 16-byte vectors in flight per thread
-constexpr int kGeluBlocksPerSm = 8;  // 2048 resident threads per SM
+constexpr int kGeluUnroll = 2;
+constexpr size_t kGeluMaxGrid = 0x7fffffffu;
 
 // -2 sqrt(2/pi) log2(e) and that times 0.044715, rounded once to fp32.
 constexpr float kA = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736);
@@ -56,19 +61,19 @@ __global__ void __launch_bounds__(kGeluThreads)
 
   const char* xv = reinterpret_cast<const char*>(x + head);
   char* yv = reinterpret_cast<char*>(y + head);
-  // Batches of kGeluUnroll vectors per thread, all loads issued before any
-  // use; the last batch is predicated rather than done one vector at a time.
-  for (size_t base = tid; base < nvec; base += kGeluUnroll * nthr) {
+  constexpr size_t kPerBlock = static_cast<size_t>(kGeluThreads) * kGeluUnroll;
+  for (size_t b = blockIdx.x; b * kPerBlock < nvec; b += gridDim.x) {
+    const size_t base = b * kPerBlock + threadIdx.x;
     uint4 v[kGeluUnroll];
 #pragma unroll
     for (int u = 0; u < kGeluUnroll; ++u) {
-      const size_t i = base + u * nthr;
-      if (i < nvec) v[u] = ld_stream_v4(xv + i * 16);
+      const size_t i = base + static_cast<size_t>(u) * kGeluThreads;
+      v[u] = ld_stream_v4_if(xv + i * 16, i < nvec, 0u);
     }
 #pragma unroll
     for (int u = 0; u < kGeluUnroll; ++u) {
-      const size_t i = base + u * nthr;
-      if (i < nvec) st_stream_v4(yv + i * 16, gelu4(v[u]));
+      const size_t i = base + static_cast<size_t>(u) * kGeluThreads;
+      st_stream_v4_if(yv + i * 16, gelu4(v[u]), i < nvec);
     }
   }
 }
@@ -90,9 +95,9 @@ cudaError_t launch_gelu_tanh(const float* x, float* y, size_t n, const DeviceInf
   const size_t scalar = head > (n - tail_begin) ? head : (n - tail_begin);
   const size_t scalar_blocks = (scalar + kGeluThreads - 1) / kGeluThreads;
   if (blocks < scalar_blocks) blocks = scalar_blocks;
-  const size_t cap = static_cast<size_t>(dev.sm_count) * kGeluBlocksPerSm;
-  if (blocks > cap) blocks = cap;
+  if (blocks > kGeluMaxGrid) blocks = kGeluMaxGrid;
   if (blocks < 1) blocks = 1;
+  (void)dev;
   gelu_tanh_kernel<<<static_cast<unsigned>(blocks), kGeluThreads, 0, stream>>>(x, y, head, nvec,
                                                                                tail_begin, n);
   return cudaGetLastError();

@@ -29,7 +29,8 @@ cudaError_t launch_gelu_tanh(const float* x, float* y, size_t n, const DeviceInf
 // ---- softmax -----------------------------------------------------------
 constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
 constexpr int kWarpThreads = 32 * kWarpRowsPerBlock;
-constexpr int kBlockElemsPerThread = 32;    // register-resident elements per thread (CTA/cluster)
+constexpr int kBlockEptSmall = 16;          // register-resident elements per thread (CTA/cluster)
+constexpr int kBlockEptLarge = 32;
 constexpr int kTwoPhaseThreads = 512;
 constexpr int kTwoPhaseElemsPerThread = 16; // elements per thread per streamed chunk
 constexpr int kMaxCluster = 16;

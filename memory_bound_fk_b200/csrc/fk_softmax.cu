@@ -101,7 +101,7 @@ __device__ __forceinline__ float exp_ref(float m) { return (m == -INFINITY) ? 0.
 // ---------------------------------------------------------------- row I/O
 
 // Load VPT chunks of a team slice into registers (VPT * VEC floats).
-// Vectors [vb, ve) of the row are the slice; anything outside is -inf.
+// Vectors [vfirst, ve) of the row are the slice; anything outside is -inf.
 template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
 __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, int t,
                                             float* v) {
@@ -110,12 +110,8 @@ __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Id
   for (int c = 0; c < VPT; ++c) {
     if constexpr (ALIGNED) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      if (vi < ve) {
-        Elem<T>::unpack(ld_stream_v4(row + static_cast<size_t>(vi) * VEC), v + c * VEC);
-      } else {
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) v[c * VEC + k] = -INFINITY;
-      }
+      Elem<T>::unpack(ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, vi < ve, Elem<T>::kNegInfWord),
+                      v + c * VEC);
     } else {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
       const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
@@ -128,25 +124,46 @@ __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Id
   }
 }
 
+// Store v * scale for the same placement as load_chunks.
 template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
 __device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx cols, int t,
-                                             const float* v) {
+                                             const float* v, float scale) {
   constexpr int VEC = Elem<T>::VEC;
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
+    float o[VEC];
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) o[k] = v[c * VEC + k] * scale;
     if constexpr (ALIGNED) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      if (vi < ve) st_stream_v4(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(v + c * VEC));
+      st_stream_v4_if(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(o), vi < ve);
     } else {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
       const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
 #pragma unroll
       for (int k = 0; k < VEC; ++k) {
         const Idx e = e0 + static_cast<Idx>(k) * TEAM;
-        if (e < eend) Elem<T>::store1(row + e, v[c * VEC + k]);
+        if (e < eend) Elem<T>::store1(row + e, o[k]);
       }
     }
   }
+}
+
+// Exponentials of v relative to ref, in place; returns their sum (four
+// accumulators).  FOLD: ref*log2(e) folded into one FMA per element (used
+// when every exponential of the row shares the reference, so the rounding of
+// ref*log2(e) is a common factor that cancels in the normalisation).
+// Otherwise (x - ref) is formed first, exact for the largest terms.
+template <int E, bool FOLD>
+__device__ __forceinline__ float exp_sum(float* v, float ref) {
+  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const float refL = ref * kLog2e;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    v[e] = FOLD ? ex2(fmaf(v[e], kLog2e, -refL)) : ex2((v[e] - ref) * kLog2e);
+    s[e & 3] += v[e];
+  }
+  return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
 // ---------------------------------------------------------------- warp path
@@ -165,26 +182,9 @@ __global__ void __launch_bounds__(kWarpThreads)
     T* yr = y + row * static_cast<size_t>(cols);
     float v[E];
     load_chunks<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, v);
-
-    float m = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < E; ++e) m = fmaxf(m, v[e]);
-    m = warp_max(m);
-
-    // One reference m for the whole row: the rounding of m*log2(e) is a
-    // common factor of every exponential and of their sum, so it cancels.
-    const float mL = m * kLog2e;
-    float s = 0.0f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      v[e] = ex2(fmaf(v[e], kLog2e, -mL));
-      s += v[e];
-    }
-    s = warp_sum(s);
-    const float r = __frcp_rn(s);
-#pragma unroll
-    for (int e = 0; e < E; ++e) v[e] *= r;
-    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v);
+    const float m = warp_max(max_of<E>(v));
+    const float s = warp_sum(exp_sum<E, true>(v, m));
+    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, __frcp_rn(s));
   }
 }
 
@@ -193,13 +193,15 @@ __global__ void __launch_bounds__(kWarpThreads)
 // CLUSTER = false: one block per row.  CLUSTER = true: launched as clusters
 // of 2..16 blocks; block `rank` of a cluster holds vectors
 // [rank*per, (rank+1)*per) of the row, per = ceil(nvec / cluster size).
-template <typename T, int THREADS, bool ALIGNED, bool CLUSTER>
+// EPT = register-resident elements per thread.
+template <typename T, int THREADS, int EPT, bool ALIGNED, bool CLUSTER>
 __global__ void __launch_bounds__(THREADS)
     softmax_block_kernel(const T* x, T* y, size_t rows, int cols) {
   constexpr int VEC = Elem<T>::VEC;
-  constexpr int VPT = kBlockElemsPerThread / VEC;
+  constexpr int VPT = EPT / VEC;
   constexpr int E = VPT * VEC;
   constexpr int NW = THREADS / 32;
+  static_assert(VPT * VEC == EPT, "EPT must be a multiple of the vector width");
   __shared__ float red_max[NW];
   __shared__ float red_sum[NW];
   __shared__ float2 part[2];  // this block's (max, sum), double-buffered by row parity
@@ -220,36 +222,16 @@ __global__ void __launch_bounds__(THREADS)
     float v[E];
     load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, v);
 
-    float m = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < E; ++e) m = fmaxf(m, v[e]);
-    m = warp_max(m);
+    float m = warp_max(max_of<E>(v));
     if (lane == 0) red_max[warp] = m;
     __syncthreads();
     m = red_max[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
 
-    float s = 0.0f;
-    if constexpr (CLUSTER) {
-      // Blocks use different references, so take the exponent difference
-      // exactly-ish ((x - ref) rounds relative to |x - ref|, which is 0 for
-      // the largest terms) instead of folding ref*log2(e) into an FMA.
-      const float ref = exp_ref(m);
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        v[e] = ex2((v[e] - ref) * kLog2e);
-        s += v[e];
-      }
-    } else {
-      const float mL = m * kLog2e;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        v[e] = ex2(fmaf(v[e], kLog2e, -mL));
-        s += v[e];
-      }
-    }
-    s = warp_sum(s);
+    // Blocks of a cluster use different references, so there the exponent
+    // difference is formed exactly-ish instead of folded into an FMA.
+    float s = warp_sum(CLUSTER ? exp_sum<E, false>(v, exp_ref(m)) : exp_sum<E, true>(v, m));
     if (lane == 0) red_sum[warp] = s;
     __syncthreads();
     s = red_sum[0];
@@ -273,9 +255,7 @@ __global__ void __launch_bounds__(THREADS)
     } else {
       scale = __frcp_rn(s);
     }
-#pragma unroll
-    for (int e = 0; e < E; ++e) v[e] *= scale;
-    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v);
+    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, scale);
     __syncthreads();  // red_max / red_sum are rewritten by the next row
   }
   if constexpr (CLUSTER) cluster_sync_all();  // keep `part` alive until all readers are done
@@ -320,14 +300,8 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
     for (size_t c = vb; c < ve; c += CHUNK) {
       float v[E];
       load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
-      float cm = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < E; ++e) cm = fmaxf(cm, v[e]);
-      const float mn = fmaxf(m, cm);
-      const float ref = exp_ref(mn);
-      float acc = 0.0f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc += ex2((v[e] - ref) * kLog2e);
+      const float mn = fmaxf(m, max_of<E>(v));
+      const float acc = exp_sum<E, false>(v, exp_ref(mn));
       l = l * rescale(m, mn) + acc;
       m = mn;
     }
@@ -368,8 +342,8 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
       float v[E];
       load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = ex2((v[e] - ref) * kLog2e) * r;
-      store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v);
+      for (int e = 0; e < E; ++e) v[e] = ex2((v[e] - ref) * kLog2e);
+      store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
     }
     __syncthreads();  // red is rewritten by the next row
   }
@@ -423,8 +397,20 @@ cudaError_t launch_warp(const void* x, void* y, size_t rows, size_t cols, int vp
   }
 }
 
+template <typename T, int EPT, bool ALIGNED, bool CLUSTER>
+cudaError_t launch_block_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads,
+                             int k, cudaStream_t s) {
+  switch (threads) {
+    case 128: return launch(softmax_block_kernel<T, 128, EPT, ALIGNED, CLUSTER>, blocks, 128, k, s, xp, yp, rows, c);
+    case 256: return launch(softmax_block_kernel<T, 256, EPT, ALIGNED, CLUSTER>, blocks, 256, k, s, xp, yp, rows, c);
+    case 512: return launch(softmax_block_kernel<T, 512, EPT, ALIGNED, CLUSTER>, blocks, 512, k, s, xp, yp, rows, c);
+    case 1024: return launch(softmax_block_kernel<T, 1024, EPT, ALIGNED, CLUSTER>, blocks, 1024, k, s, xp, yp, rows, c);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <typename T, bool ALIGNED, bool CLUSTER>
-cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int threads,
+cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int threads, int vpt,
                          int cluster, cudaStream_t s) {
   const size_t cl = CLUSTER ? static_cast<size_t>(cluster) : 1;
   size_t groups = rows;
@@ -434,11 +420,9 @@ cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int t
   T* yp = static_cast<T*>(y);
   const int c = static_cast<int>(cols);
   const int k = static_cast<int>(cl);
-  switch (threads) {
-    case 128: return launch(softmax_block_kernel<T, 128, ALIGNED, CLUSTER>, blocks, 128, k, s, xp, yp, rows, c);
-    case 256: return launch(softmax_block_kernel<T, 256, ALIGNED, CLUSTER>, blocks, 256, k, s, xp, yp, rows, c);
-    case 512: return launch(softmax_block_kernel<T, 512, ALIGNED, CLUSTER>, blocks, 512, k, s, xp, yp, rows, c);
-    case 1024: return launch(softmax_block_kernel<T, 1024, ALIGNED, CLUSTER>, blocks, 1024, k, s, xp, yp, rows, c);
+  switch (vpt * Elem<T>::VEC) {
+    case 16: return launch_block_ept<T, 16, ALIGNED, CLUSTER>(xp, yp, rows, c, blocks, threads, k, s);
+    case 32: return launch_block_ept<T, 32, ALIGNED, CLUSTER>(xp, yp, rows, c, blocks, threads, k, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -458,9 +442,9 @@ cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
                          const fk_softmax_plan& p, cudaStream_t s) {
   switch (p.path) {
     case FK_PATH_WARP: return launch_warp<T, ALIGNED>(x, y, rows, cols, p.vpt, s);
-    case FK_PATH_CTA: return launch_block<T, ALIGNED, false>(x, y, rows, cols, p.threads, 1, s);
+    case FK_PATH_CTA: return launch_block<T, ALIGNED, false>(x, y, rows, cols, p.threads, p.vpt, 1, s);
     case FK_PATH_CLUSTER:
-      return launch_block<T, ALIGNED, true>(x, y, rows, cols, p.threads, p.cluster, s);
+      return launch_block<T, ALIGNED, true>(x, y, rows, cols, p.threads, p.vpt, p.cluster, s);
     case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED>(x, y, rows, cols, p.cluster, s);
     default: return cudaErrorInvalidValue;
   }

@@ -231,20 +231,27 @@ def _cfg5(rows: int = 512, cols: int = 131072, seed: int = 4, threads=None) -> n
 
 # ------------------------------------------------------------------ public
 
-def make(name: str, threads: int | None = None) -> np.ndarray:
-    """Full input of a named workload (fp32 array, or uint16 bf16 bits)."""
+def make(name: str, threads: int | None = None, rows: int | None = None) -> np.ndarray:
+    """Input of a named workload (fp32 array, or uint16 bf16 bits).
+
+    `rows` (softmax) or element count (GELU) shrinks the workload to its
+    leading part with the same recipe -- for small profiling cases; None is
+    the full size."""
     if name == "cfg1_softmax":
-        return _cfg1_values().reshape(256, 1000)
+        return _cfg1_values().reshape(256, 1000)[:rows]
     if name == "cfg1_gelu":
-        return _cfg1_values()
+        return _cfg1_values()[:rows]
     if name == "cfg2_gelu":
-        return _cfg2()
+        return _cfg2()[:rows]
     if name == "cfg3_softmax":
-        return _cfg3(threads=threads)
+        r = rows or 8192
+        return _cfg3(rows=-(-r // CFG3_ROWS_PER_CHUNK) * CFG3_ROWS_PER_CHUNK, threads=threads)[:r]
     if name == "cfg4_softmax":
-        return _cfg4(threads=threads)
+        r = rows or CFG4_HEADS * CFG4_T
+        return _cfg4(heads=-(-r // CFG4_T), threads=threads)[:r]
     if name == "cfg5_softmax":
-        return _cfg5(threads=threads)
+        r = rows or 512
+        return _cfg5(rows=-(-r // CFG5_ROWS_PER_CHUNK) * CFG5_ROWS_PER_CHUNK, threads=threads)[:r]
     raise KeyError(name)
 
 

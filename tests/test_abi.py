@@ -25,14 +25,16 @@ def test_version_and_status_strings(fk):
 @pytest.mark.parametrize("rows,cols,dtype,expect", [
     (256, 1000, 0, ("warp", 256, 8, 1)),        # 256x1000 fp32
     (8192, 4096, 0, ("cta", 128, 8, 1)),        # 8192x4096 fp32
-    (1 << 20, 2048, 1, ("warp", 256, 8, 1)),    # bf16 attention rows
+    (1 << 20, 2048, 1, ("cta", 128, 2, 1)),     # bf16 attention rows
     (512, 131072, 0, ("cluster", 512, 8, 8)),   # vocab-sized rows
     (4, 1, 0, ("warp", 256, 1, 1)),
     (4, 128, 0, ("warp", 256, 1, 1)),
     (4, 129, 0, ("warp", 256, 2, 1)),
     (4, 1024, 0, ("warp", 256, 8, 1)),
     (4, 1025, 0, ("cta", 128, 8, 1)),
-    (4, 2049, 1, ("cta", 128, 4, 1)),
+    (4, 2049, 1, ("cta", 256, 2, 1)),
+    (4, 1024, 1, ("warp", 256, 4, 1)),
+    (4, 16385, 1, ("cta", 1024, 4, 1)),
     (4, 32768, 0, ("cta", 1024, 8, 1)),
     (4, 32769, 0, ("cluster", 512, 8, 3)),
     (4, 131073, 0, ("cluster", 1024, 8, 5)),

@@ -75,13 +75,14 @@ def test_auto_plan_bf16(fk, torch_mod, rows, cols):
 
 def _forced_plans(fk, cols, dtype):
     plans = []
-    for t in (128, 256, 512, 1024):
-        if t * 32 >= cols:
-            plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t))
-    for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (1024, 16)):
-        vec = 4 if dtype == "f32" else 8
-        if -(-(-(-cols // vec)) // k) * vec <= t * 32:
-            plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k))
+    vec = 4 if dtype == "f32" else 8
+    for ept in (16, 32):
+        for t in (128, 256, 512, 1024):
+            if t * ept >= cols:
+                plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t, vpt=ept // vec))
+        for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (1024, 16)):
+            if -(-(-(-cols // vec)) // k) * vec <= t * ept:
+                plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k, vpt=ept // vec))
     for k in (1, 2, 3, 16):
         plans.append(fk.make_plan(fk.FK_PATH_TWOPHASE, cluster=k))
     if cols <= (1024 if dtype == "f32" else 2048):
