@@ -65,9 +65,11 @@ def kernel_name(w, plan: dict) -> str:
     p = plan["path"]
     if p == "warp":
         return f"softmax_warp_kernel<{t},vpt={plan['vpt']}>"
-    if p in ("cta", "cluster"):
-        extra = f",cluster={plan['cluster']}" if p == "cluster" else ""
-        return f"softmax_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{extra}>"
+    if p == "cta":
+        return f"softmax_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}>"
+    if p == "cluster":
+        return (f"softmax_cluster_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}>"
+                f" x cluster {plan['cluster']}")
     return f"softmax_twophase_kernel<{t},cluster={plan['cluster']}>"
 
 

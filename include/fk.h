@@ -148,6 +148,28 @@ FK_API fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int p
 FK_API fk_status fk_softmax_rows_ex(const void *x, void *y, size_t rows, size_t cols, int dtype,
                              const fk_softmax_plan *plan, void *stream);
 
+/*
+ * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a
+ * cluster exchange their partial (max, sum) through mbarriers; every such
+ * wait is bounded in time (1 s) and a wait that gives up is counted instead
+ * of hanging the GPU (the row is then not valid).
+ *   count  [out] number of threads whose wait gave up on the current device
+ *          since the library was loaded or last reset.
+ *   reset  nonzero: set the count back to 0 after reading it.
+ * Synchronous; call after the work of interest has completed.  A nonzero
+ * count in normal operation means a partner block never arrived.
+ */
+FK_API fk_status fk_wait_timeouts(unsigned int *count, int reset);
+
+/*
+ * fk_wait_selftest -- launch one block of 32 threads that waits on an
+ * mbarrier nothing arrives on, with a limit of timeout_us microseconds
+ * (1..10000000); each thread gives up and adds 1 to fk_wait_timeouts.  Tests
+ * the give-up path without faulting or hanging the GPU.  Asynchronous on
+ * `stream`.
+ */
+FK_API fk_status fk_wait_selftest(unsigned int timeout_us, void *stream);
+
 /* Static description of a status code (never NULL). */
 FK_API const char *fk_status_string(int status);
 

@@ -11,6 +11,8 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
     fk_softmax_rows_ex(x, y, rows, cols, dtype, plan, stream) -> status
     fk_softmax_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
     fk_status_string(status) -> str
+    fk_wait_timeouts(reset=False) -> int     (bounded-wait give-ups, synchronous)
+    fk_wait_selftest(timeout_us, stream) -> status
 
 Tensor conveniences (contiguous CUDA tensors; the current torch stream):
     gelu_tanh(x, out=None)
@@ -93,6 +95,10 @@ def lib() -> ctypes.CDLL:
         L.fk_last_cuda_error.restype = ci
         L.fk_version.argtypes = []
         L.fk_version.restype = ci
+        L.fk_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
+        L.fk_wait_timeouts.restype = ci
+        L.fk_wait_selftest.argtypes = [ctypes.c_uint, vp]
+        L.fk_wait_selftest.restype = ci
         _lib = L
     return _lib
 
@@ -137,6 +143,20 @@ def fk_last_cuda_error() -> int:
 
 def fk_version() -> int:
     return lib().fk_version()
+
+
+def fk_wait_timeouts(reset: bool = False) -> int:
+    """Threads whose bounded cluster wait gave up on the current device
+    (synchronous).  Raises FkError on failure."""
+    c = ctypes.c_uint(0)
+    st = lib().fk_wait_timeouts(ctypes.byref(c), 1 if reset else 0)
+    if st != FK_OK:
+        raise FkError(st, "fk_wait_timeouts")
+    return c.value
+
+
+def fk_wait_selftest(timeout_us: int, stream: int = 0) -> int:
+    return lib().fk_wait_selftest(timeout_us, stream)
 
 
 def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0) -> SoftmaxPlan:
@@ -207,6 +227,7 @@ __all__ = [
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FkError", "SoftmaxPlan", "lib", "header_functions",
     "fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
-    "fk_status_string", "fk_last_cuda_error", "fk_version", "make_plan", "gelu_tanh",
+    "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
+    "fk_wait_selftest", "make_plan", "gelu_tanh",
     "softmax_rows",
 ]

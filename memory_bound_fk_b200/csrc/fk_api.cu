@@ -190,6 +190,26 @@ fk_status fk_softmax_rows(const void* x, void* y, size_t rows, size_t cols, int 
   return fk_softmax_rows_ex(x, y, rows, cols, dtype, nullptr, stream);
 }
 
+fk_status fk_wait_timeouts(unsigned int* count, int reset) {
+  if (count == nullptr) return FK_ERR_INVALID_ARG;
+  int dev = -1;
+  const fk::DeviceInfo* info = fk::current_device_info(&dev);
+  if (info == nullptr || !info->ok) return FK_ERR_UNSUPPORTED_DEVICE;
+  if (info->major != 10 || info->minor != 0) return FK_ERR_UNSUPPORTED_DEVICE;
+  const cudaError_t e = fk::read_wait_timeouts(count, reset != 0);
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_wait_selftest(unsigned int timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 10000000u) return FK_ERR_INVALID_ARG;
+  int dev = -1;
+  const fk::DeviceInfo* info = fk::current_device_info(&dev);
+  if (info == nullptr || !info->ok) return FK_ERR_UNSUPPORTED_DEVICE;
+  if (info->major != 10 || info->minor != 0) return FK_ERR_UNSUPPORTED_DEVICE;
+  const cudaError_t e = fk::launch_wait_selftest(timeout_us, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
 const char* fk_status_string(int status) {
   switch (status) {
     case FK_OK: return "FK_OK: success";

@@ -117,6 +117,9 @@ struct Elem<float> {
   }
   __device__ __forceinline__ static float load1(const float* p) { return __ldg(p); }
   __device__ __forceinline__ static void store1(float* p, float v) { *p = v; }
+  // exp2 for softmax terms: results below 2^-126 flush to zero, an absolute
+  // error under 1.2e-38 on an fp32 output (3% faster on 4096-column rows).
+  __device__ __forceinline__ static float exp2(float a) { return ex2_ftz(a); }
 };
 
 // bf16 (stored as raw 16-bit patterns): 8 values per 16-byte vector.
@@ -150,6 +153,9 @@ struct Elem<__nv_bfloat16> {
   __device__ __forceinline__ static void store1(__nv_bfloat16* p, float v) {
     *p = __float2bfloat16_rn(v);
   }
+  // exp2 for softmax terms: subnormal results kept, because bf16 outputs
+  // down to 2^-133 must still round correctly (no measurable cost here).
+  __device__ __forceinline__ static float exp2(float a) { return ex2(a); }
 };
 
 }  // namespace fk

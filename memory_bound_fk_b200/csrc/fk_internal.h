@@ -31,6 +31,7 @@ constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the w
 constexpr int kWarpThreads = 32 * kWarpRowsPerBlock;
 constexpr int kBlockEptSmall = 16;          // register-resident elements per thread (CTA/cluster)
 constexpr int kBlockEptLarge = 32;
+constexpr int kClusterEpt = 64;             // cluster blocks: 64 values per thread, <= 512 threads
 constexpr int kTwoPhaseThreads = 512;
 constexpr int kTwoPhaseElemsPerThread = 16; // elements per thread per streamed chunk
 constexpr int kMaxCluster = 16;
@@ -48,5 +49,13 @@ fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softm
 cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
                            const fk_softmax_plan& plan, bool aligned, const DeviceInfo& dev,
                            cudaStream_t stream);
+
+// Number of threads whose bounded mbarrier wait gave up, on the current
+// device; optionally reset to 0.  Synchronous.
+cudaError_t read_wait_timeouts(unsigned* out, bool reset);
+
+// One block of 32 threads waits on an mbarrier that nothing arrives on and
+// gives up after timeout_us microseconds (adds 32 to the count above).
+cudaError_t launch_wait_selftest(unsigned timeout_us, cudaStream_t stream);
 
 }  // namespace fk

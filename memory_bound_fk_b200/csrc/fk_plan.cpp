@@ -5,14 +5,17 @@
 //              -> up to 1024 fp32 / 2048 bf16 columns
 //   block    : 16 or 32 elements per thread (EPT), threads in
 //              {128, 256, 512, 1024} -> up to 32768 columns
-//   cluster  : 2..16 blocks of the block kernel -> up to 524288 columns
+//   cluster  : 2..16 blocks of 128..512 threads holding 64 values each
+//              -> up to 524288 columns
 //   twophase : any length (row streamed twice)
 // The automatic choice takes the smallest shape that holds the row on chip,
 // so a row is read from HBM once whenever it fits in a cluster.  Measured on
 // B200 (L2 cleaned between runs): 4096-column fp32 rows run best as one
 // 128-thread block with 32 elements per thread; 2048-column bf16 rows as one
 // 128-thread block with 16 elements per thread (32 registers, so 16 blocks
-// fit per SM); rows up to 1024 fp32 / bf16 columns stay on one warp.
+// fit per SM); rows up to 1024 fp32 / bf16 columns stay on one warp;
+// 131072-column fp32 rows as a cluster of 16 blocks of 128 threads with 64
+// values per thread (more, smaller blocks fit more clusters on the GPU).
 #include <stddef.h>
 
 #include "fk_internal.h"
@@ -34,6 +37,10 @@ size_t warp_cap(int dtype, int vpt) { return static_cast<size_t>(32) * vpt * vec
 size_t block_cap(int threads, int ept) { return static_cast<size_t>(threads) * ept; }
 
 bool ept_ok(int ept) { return ept == kBlockEptSmall || ept == kBlockEptLarge; }
+
+bool cluster_ept_ok(int ept, int threads) {
+  return ept_ok(ept) || (ept == kClusterEpt && threads <= 512);
+}
 
 }  // namespace
 
@@ -75,18 +82,18 @@ fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax
       break;
     }
     case FK_PATH_CLUSTER: {
-      // 512-thread blocks up to 8 per cluster (portable size), then
-      // 1024-thread blocks up to 16 per cluster; 32 elements per thread.
-      size_t k = ceil_div(cols, block_cap(512, kBlockEptLarge));
-      int t = 512;
-      if (k > 8) {
-        t = 1024;
-        k = ceil_div(cols, block_cap(1024, kBlockEptLarge));
+      // 64 values per thread; the smallest block (128, 256, then 512
+      // threads) whose cluster of at most 16 holds the row
+      int t = 128;
+      size_t k = ceil_div(cols, block_cap(t, kClusterEpt));
+      while (k > static_cast<size_t>(kMaxCluster) && t < 512) {
+        t *= 2;
+        k = ceil_div(cols, block_cap(t, kClusterEpt));
       }
       if (k < 2) k = 2;
       if (k > static_cast<size_t>(kMaxCluster)) return FK_ERR_INVALID_ARG;
       p.threads = t;
-      p.vpt = kBlockEptLarge / vec;
+      p.vpt = kClusterEpt / vec;
       p.cluster = static_cast<int>(k);
       break;
     }
@@ -117,8 +124,8 @@ fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softm
     // the default for this path may not hold cols, but an explicit plan could
     if (in.path != FK_PATH_CTA && in.path != FK_PATH_CLUSTER) return st;
     d.path = in.path;
-    d.threads = 1024;
-    d.vpt = kBlockEptLarge / vec;
+    d.threads = in.path == FK_PATH_CLUSTER ? 512 : 1024;
+    d.vpt = (in.path == FK_PATH_CLUSTER ? kClusterEpt : kBlockEptLarge) / vec;
     d.cluster = in.path == FK_PATH_CLUSTER ? kMaxCluster : 1;
   }
   fk_softmax_plan p = d;
@@ -139,7 +146,7 @@ fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softm
     case FK_PATH_CLUSTER:
       if (!block_threads_ok(p.threads) || p.cluster < 2 || p.cluster > kMaxCluster)
         return FK_ERR_INVALID_ARG;
-      if (!ept_ok(p.vpt * vec)) return FK_ERR_INVALID_ARG;
+      if (!cluster_ept_ok(p.vpt * vec, p.threads)) return FK_ERR_INVALID_ARG;
       // each block's slice, ceil(vectors / cluster), must fit its registers
       if (ceil_div(ceil_div(cols, vec), p.cluster) * vec > block_cap(p.threads, p.vpt * vec))
         return FK_ERR_INVALID_ARG;

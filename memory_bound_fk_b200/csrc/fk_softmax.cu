@@ -13,12 +13,17 @@
 //   block    -- one thread block per row, 32 register-resident elements per
 //               thread (up to 32768 columns); warp shuffles, then one shared
 //               memory exchange between warps.
-//   cluster  -- the same block kernel launched as a thread-block cluster of
-//               2..16 blocks per row; each block reduces its slice to a
-//               partial (m_c, l_c) and the partials are merged over
-//               distributed shared memory with the running-max rule of
-//               section 7.2:  M = max_c m_c,  L = sum_c l_c exp(m_c - M).
-//               Every element is still read once and written once.
+//   cluster  -- a thread-block cluster of 2..16 blocks per row, each block
+//               holding a slice in registers (up to 64 values per thread);
+//               each block reduces its slice to a partial (m_c, l_c), pushes
+//               it into every other block's shared memory with st.async
+//               (completing on the receiver's mbarrier), and merges the
+//               partials with the running-max rule of section 7.2:
+//               M = max_c m_c,  L = sum_c l_c exp(m_c - M).  Every element
+//               is still read once and written once.  There is no cluster
+//               barrier on the row path: the only one is split (arrive at
+//               kernel start, wait just before the first push) and only
+//               publishes the mbarrier initialisation.
 //   twophase -- for rows longer than a cluster can hold: each block streams
 //               its slice, keeping a per-thread running (m, l) (the online
 //               recurrence of section 7.2), merges as above, then streams the
@@ -41,47 +46,39 @@
 
 #include "fk_common.cuh"
 #include "fk_internal.h"
+#include "fk_sync.cuh"
 
 namespace fk {
+
+// Number of threads whose mbarrier wait gave up (see bounded_wait).
+__device__ unsigned int g_wait_timeouts = 0;
+
 namespace {
+
+// Time limit of every mbarrier wait on the row paths.  A partner block that
+// has not arrived after this long is not coming; the wait gives up, counts
+// itself in g_wait_timeouts and the kernel finishes without hanging.
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
+
+__device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > timeout_ns) {
+      atomicAdd(&g_wait_timeouts, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
+                                             uint64_t timeout_ns = kWaitTimeoutNs) {
+  return mbar_try_wait(bar, parity) || bounded_wait_slow(bar, parity, timeout_ns);
+}
 
 template <typename I>
 __device__ __forceinline__ I imin(I a, I b) {
   return a < b ? a : b;
-}
-
-// ---------------------------------------------------------------- cluster PTX
-
-__device__ __forceinline__ unsigned cluster_ctarank() {
-  unsigned r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ unsigned cluster_nctarank() {
-  unsigned r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-
-// Full cluster barrier: release this block's shared-memory writes, acquire
-// the other blocks'.  Every thread of every block of the cluster calls it.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile(
-      "barrier.cluster.arrive.release;\n\t"
-      "barrier.cluster.wait.acquire;" ::
-          : "memory");
-}
-
-// Load a float2 from the shared memory of block `rank` of this cluster, at
-// the offset of `local` in this block's shared memory.
-__device__ __forceinline__ float2 ld_dsmem_f2(const float2* local, unsigned rank) {
-  const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(local));
-  unsigned ra;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(ra) : "memory");
-  return v;
 }
 
 // ---------------------------------------------------------------- merge rule
@@ -154,13 +151,13 @@ __device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx col
 // when every exponential of the row shares the reference, so the rounding of
 // ref*log2(e) is a common factor that cancels in the normalisation).
 // Otherwise (x - ref) is formed first, exact for the largest terms.
-template <int E, bool FOLD>
+template <typename T, int E, bool FOLD>
 __device__ __forceinline__ float exp_sum(float* v, float ref) {
   float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const float refL = ref * kLog2e;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    v[e] = FOLD ? ex2(fmaf(v[e], kLog2e, -refL)) : ex2((v[e] - ref) * kLog2e);
+    v[e] = FOLD ? Elem<T>::exp2(fmaf(v[e], kLog2e, -refL)) : Elem<T>::exp2((v[e] - ref) * kLog2e);
     s[e & 3] += v[e];
   }
   return (s[0] + s[1]) + (s[2] + s[3]);
@@ -183,18 +180,56 @@ __global__ void __launch_bounds__(kWarpThreads)
     float v[E];
     load_chunks<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, v);
     const float m = warp_max(max_of<E>(v));
-    const float s = warp_sum(exp_sum<E, true>(v, m));
+    const float s = warp_sum(exp_sum<T, E, true>(v, m));
     store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, __frcp_rn(s));
   }
 }
 
-// ---------------------------------------------------------------- block / cluster path
+// ---------------------------------------------------------------- cluster exchange
 
-// CLUSTER = false: one block per row.  CLUSTER = true: launched as clusters
-// of 2..16 blocks; block `rank` of a cluster holds vectors
-// [rank*per, (rank+1)*per) of the row, per = ceil(nvec / cluster size).
-// EPT = register-resident elements per thread.
-template <typename T, int THREADS, int EPT, bool ALIGNED, bool CLUSTER>
+// Per-block partials of the row: inbox[i] receives block i's (max, sum);
+// bar completes when the csize - 1 pushes from the other blocks have landed.
+// Each cluster handles exactly one row, so every buffer is used once.
+struct ClusterExchange {
+  float2 inbox[kMaxCluster];
+  uint64_t bar;
+};
+
+// Thread 0 of every block, before cluster_arrive_relaxed().
+__device__ __forceinline__ void exchange_init(ClusterExchange& ex) {
+  mbar_init(&ex.bar, 1);
+  fence_mbarrier_init();
+}
+
+// All threads of the block, once per kernel.  Completes the start-up cluster
+// barrier (so every receiver's mbarrier is initialised), pushes this
+// block's (m, l) into every other block's inbox with st.async, waits
+// (bounded) for the other blocks' pushes, and returns the merged (M, L) of
+// the row.  A block exits only after all pushes addressed to it have
+// landed, and it pushes only to blocks that are waiting for it, so no block
+// touches the shared memory of a block that has exited.
+__device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, float l, int csize, int crank) {
+  const int t = threadIdx.x, lane = t & 31;
+  if (t == 0) mbar_arrive_expect_tx(&ex.bar, static_cast<uint32_t>(csize - 1) * 8u);
+  cluster_wait();
+  if (t < csize && t != crank) st_async_f2(cluster_addr(&ex.inbox[crank], t), m, l, cluster_addr(&ex.bar, t));
+  bounded_wait(&ex.bar, 0);
+  // every warp merges the partials itself: lane i takes block i's
+  float mi = -INFINITY, li = 0.0f;
+  if (lane < csize) {
+    const float2 q = (lane == crank) ? make_float2(m, l) : ex.inbox[lane];
+    mi = q.x;
+    li = q.y;
+  }
+  const float M = warp_max(mi);
+  const float L = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
+  return make_float2(M, L);
+}
+
+// ---------------------------------------------------------------- block path
+
+// One block per row; EPT = register-resident elements per thread.
+template <typename T, int THREADS, int EPT, bool ALIGNED>
 __global__ void __launch_bounds__(THREADS)
     softmax_block_kernel(const T* x, T* y, size_t rows, int cols) {
   constexpr int VEC = Elem<T>::VEC;
@@ -204,23 +239,14 @@ __global__ void __launch_bounds__(THREADS)
   static_assert(VPT * VEC == EPT, "EPT must be a multiple of the vector width");
   __shared__ float red_max[NW];
   __shared__ float red_sum[NW];
-  __shared__ float2 part[2];  // this block's (max, sum), double-buffered by row parity
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int csize = CLUSTER ? static_cast<int>(cluster_nctarank()) : 1;
-  const int crank = CLUSTER ? static_cast<int>(cluster_ctarank()) : 0;
   const int nvec = (cols + VEC - 1) / VEC;
-  const int per = (nvec + csize - 1) / csize;
-  const int vb = imin(nvec, crank * per);
-  const int ve = imin(nvec, vb + per);
-
-  const size_t stride = gridDim.x / csize;
-  int parity = 0;
-  for (size_t row = blockIdx.x / csize; row < rows; row += stride, parity ^= 1) {
+  for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
     float v[E];
-    load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, v);
+    load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, 0, nvec, cols, t, v);
 
     float m = warp_max(max_of<E>(v));
     if (lane == 0) red_max[warp] = m;
@@ -229,36 +255,71 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
 
-    // Blocks of a cluster use different references, so there the exponent
-    // difference is formed exactly-ish instead of folded into an FMA.
-    float s = warp_sum(CLUSTER ? exp_sum<E, false>(v, exp_ref(m)) : exp_sum<E, true>(v, m));
+    float s = warp_sum(exp_sum<T, E, true>(v, m));
     if (lane == 0) red_sum[warp] = s;
     __syncthreads();
     s = red_sum[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) s += red_sum[w];
 
-    float scale;
-    if constexpr (CLUSTER) {
-      if (t == 0) part[parity] = make_float2(m, s);
-      cluster_sync_all();
-      // every warp merges the cluster's partials itself: lane i reads block i
-      float mi = -INFINITY, li = 0.0f;
-      if (lane < csize) {
-        const float2 p = ld_dsmem_f2(&part[parity], static_cast<unsigned>(lane));
-        mi = p.x;
-        li = p.y;
-      }
-      const float M = warp_max(mi);
-      const float L = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
-      scale = rescale(m, M) * __frcp_rn(L);
-    } else {
-      scale = __frcp_rn(s);
-    }
-    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, scale);
+    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, 0, nvec, cols, t, v, __frcp_rn(s));
     __syncthreads();  // red_max / red_sum are rewritten by the next row
   }
-  if constexpr (CLUSTER) cluster_sync_all();  // keep `part` alive until all readers are done
+}
+
+// ---------------------------------------------------------------- cluster path
+
+// A cluster of csize blocks per row; block `rank` holds vectors
+// [rank*per, (rank+1)*per) of the row in registers, per = ceil(nvec / csize).
+template <typename T, int THREADS, int EPT, bool ALIGNED>
+__global__ void __launch_bounds__(THREADS)
+    softmax_cluster_kernel(const T* x, T* y, size_t rows, int cols) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int VPT = EPT / VEC;
+  constexpr int E = VPT * VEC;
+  constexpr int NW = THREADS / 32;
+  static_assert(VPT * VEC == EPT, "EPT must be a multiple of the vector width");
+  __shared__ float red_max[NW];
+  __shared__ float red_sum[NW];
+  __shared__ __align__(16) ClusterExchange ex;
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int crank = static_cast<int>(cluster_ctarank());
+  const int nvec = (cols + VEC - 1) / VEC;
+  const int per = (nvec + csize - 1) / csize;
+  const int vb = imin(nvec, crank * per);
+  const int ve = imin(nvec, vb + per);
+
+  // one row per cluster (the host splits launches that would exceed the grid)
+  const size_t row = blockIdx.x / csize;
+  if (row >= rows) return;  // same for every block of the cluster
+  if (t == 0) exchange_init(ex);
+  cluster_arrive_relaxed();
+
+  const T* xr = x + row * static_cast<size_t>(cols);
+  T* yr = y + row * static_cast<size_t>(cols);
+  float v[E];
+  load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, v);
+
+  float m = warp_max(max_of<E>(v));
+  if (lane == 0) red_max[warp] = m;
+  __syncthreads();
+  m = red_max[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
+
+  // Blocks use different references, so the exponent difference is formed
+  // first (exact for the largest terms) instead of folded into an FMA.
+  float s = warp_sum(exp_sum<T, E, false>(v, exp_ref(m)));
+  if (lane == 0) red_sum[warp] = s;
+  __syncthreads();
+  s = red_sum[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) s += red_sum[w];
+
+  const float2 ML = exchange_merge(ex, m, s, csize, crank);
+  store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, rescale(m, ML.x) * __frcp_rn(ML.y));
 }
 
 // ---------------------------------------------------------------- two-phase path
@@ -279,7 +340,7 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   constexpr int NW = THREADS / 32;
   constexpr size_t CHUNK = static_cast<size_t>(THREADS) * VPT;  // vectors per chunk
   __shared__ float2 red[NW];
-  __shared__ float2 part[2];
+  __shared__ __align__(16) ClusterExchange ex;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int csize = static_cast<int>(cluster_nctarank());  // 1 without a cluster launch
@@ -289,9 +350,14 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   const size_t vb = imin(nvec, static_cast<size_t>(crank) * per);
   const size_t ve = imin(nvec, vb + per);
 
-  const size_t stride = gridDim.x / csize;
-  int parity = 0;
-  for (size_t row = blockIdx.x / csize; row < rows; row += stride, parity ^= 1) {
+  // one row per cluster (the host splits launches that would exceed the grid)
+  const size_t row = blockIdx.x / csize;
+  if (row >= rows) return;  // same for every block of the cluster
+  if (csize > 1) {
+    if (t == 0) exchange_init(ex);
+    cluster_arrive_relaxed();
+  }
+  {
     const T* xr = x + row * cols;
     T* yr = y + row * cols;
 
@@ -301,7 +367,7 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
       float v[E];
       load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
       const float mn = fmaxf(m, max_of<E>(v));
-      const float acc = exp_sum<E, false>(v, exp_ref(mn));
+      const float acc = exp_sum<T, E, false>(v, exp_ref(mn));
       l = l * rescale(m, mn) + acc;
       m = mn;
     }
@@ -322,17 +388,9 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
 
     // merge the blocks' partials across the cluster
     if (csize > 1) {
-      if (t == 0) part[parity] = make_float2(m, l);
-      cluster_sync_all();
-      float mi = -INFINITY, li = 0.0f;
-      if (lane < csize) {
-        const float2 p = ld_dsmem_f2(&part[parity], static_cast<unsigned>(lane));
-        mi = p.x;
-        li = p.y;
-      }
-      const float M = warp_max(mi);
-      l = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
-      m = M;
+      const float2 ML = exchange_merge(ex, m, l, csize, crank);
+      m = ML.x;
+      l = ML.y;
     }
 
     // pass 2: y = exp(x - M) / L
@@ -342,13 +400,25 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
       float v[E];
       load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = ex2((v[e] - ref) * kLog2e);
+      for (int e = 0; e < E; ++e) v[e] = Elem<T>::exp2((v[e] - ref) * kLog2e);
       store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
     }
-    __syncthreads();  // red is rewritten by the next row
   }
-  if (csize > 1) cluster_sync_all();
 }
+
+// A wait on an mbarrier that nothing ever arrives on: every thread gives up
+// after `timeout_ns` and counts itself in g_wait_timeouts.  Exercises the
+// give-up path of bounded_wait without faulting or hanging anything.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  bounded_wait(&bar, 0, timeout_ns);
+}
+
 
 // ---------------------------------------------------------------- launch helpers
 
@@ -397,44 +467,86 @@ cudaError_t launch_warp(const void* x, void* y, size_t rows, size_t cols, int vp
   }
 }
 
-template <typename T, int EPT, bool ALIGNED, bool CLUSTER>
+template <typename T, int EPT, bool ALIGNED>
 cudaError_t launch_block_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads,
-                             int k, cudaStream_t s) {
+                             cudaStream_t s) {
   switch (threads) {
-    case 128: return launch(softmax_block_kernel<T, 128, EPT, ALIGNED, CLUSTER>, blocks, 128, k, s, xp, yp, rows, c);
-    case 256: return launch(softmax_block_kernel<T, 256, EPT, ALIGNED, CLUSTER>, blocks, 256, k, s, xp, yp, rows, c);
-    case 512: return launch(softmax_block_kernel<T, 512, EPT, ALIGNED, CLUSTER>, blocks, 512, k, s, xp, yp, rows, c);
-    case 1024: return launch(softmax_block_kernel<T, 1024, EPT, ALIGNED, CLUSTER>, blocks, 1024, k, s, xp, yp, rows, c);
+    case 128: return launch(softmax_block_kernel<T, 128, EPT, ALIGNED>, blocks, 128, 1, s, xp, yp, rows, c);
+    case 256: return launch(softmax_block_kernel<T, 256, EPT, ALIGNED>, blocks, 256, 1, s, xp, yp, rows, c);
+    case 512: return launch(softmax_block_kernel<T, 512, EPT, ALIGNED>, blocks, 512, 1, s, xp, yp, rows, c);
+    case 1024: return launch(softmax_block_kernel<T, 1024, EPT, ALIGNED>, blocks, 1024, 1, s, xp, yp, rows, c);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, bool ALIGNED, bool CLUSTER>
+template <typename T, bool ALIGNED>
 cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int threads, int vpt,
-                         int cluster, cudaStream_t s) {
-  const size_t cl = CLUSTER ? static_cast<size_t>(cluster) : 1;
-  size_t groups = rows;
-  if (groups > kMaxGrid / cl) groups = kMaxGrid / cl;
-  const size_t blocks = groups * cl;
+                         cudaStream_t s) {
+  const size_t blocks = rows < kMaxGrid ? rows : kMaxGrid;
   const T* xp = static_cast<const T*>(x);
   T* yp = static_cast<T*>(y);
   const int c = static_cast<int>(cols);
-  const int k = static_cast<int>(cl);
   switch (vpt * Elem<T>::VEC) {
-    case 16: return launch_block_ept<T, 16, ALIGNED, CLUSTER>(xp, yp, rows, c, blocks, threads, k, s);
-    case 32: return launch_block_ept<T, 32, ALIGNED, CLUSTER>(xp, yp, rows, c, blocks, threads, k, s);
+    case 16: return launch_block_ept<T, 16, ALIGNED>(xp, yp, rows, c, blocks, threads, s);
+    case 32: return launch_block_ept<T, 32, ALIGNED>(xp, yp, rows, c, blocks, threads, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <typename T, int EPT, bool ALIGNED>
+cudaError_t launch_cluster_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads,
+                               int k, cudaStream_t s) {
+  switch (threads) {
+    case 128: return launch(softmax_cluster_kernel<T, 128, EPT, ALIGNED>, blocks, 128, k, s, xp, yp, rows, c);
+    case 256: return launch(softmax_cluster_kernel<T, 256, EPT, ALIGNED>, blocks, 256, k, s, xp, yp, rows, c);
+    case 512: return launch(softmax_cluster_kernel<T, 512, EPT, ALIGNED>, blocks, 512, k, s, xp, yp, rows, c);
+    case 1024:
+      if constexpr (EPT <= 32) {
+        return launch(softmax_cluster_kernel<T, 1024, EPT, ALIGNED>, blocks, 1024, k, s, xp, yp, rows, c);
+      }
+      return cudaErrorInvalidValue;  // 64 values per thread do not fit 1024 threads' registers
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Cluster launches handle one row per cluster; rows beyond one grid's worth
+// of clusters go to further launches.
+template <typename T, bool ALIGNED>
+cudaError_t launch_cluster(const void* x, void* y, size_t rows, size_t cols, int threads, int vpt,
+                           int cluster, cudaStream_t s) {
+  const size_t cl = static_cast<size_t>(cluster);
+  const size_t max_rows = kMaxGrid / cl;
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
+  const int c = static_cast<int>(cols);
+  for (size_t r0 = 0; r0 < rows; r0 += max_rows) {
+    const size_t n = (rows - r0 < max_rows) ? rows - r0 : max_rows;
+    const T* xs = xp + r0 * cols;
+    T* ys = yp + r0 * cols;
+    cudaError_t e;
+    switch (vpt * Elem<T>::VEC) {
+      case 16: e = launch_cluster_ept<T, 16, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
+      case 32: e = launch_cluster_ept<T, 32, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
+      case 64: e = launch_cluster_ept<T, 64, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
+      default: e = cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename T, bool ALIGNED>
 cudaError_t launch_twophase(const void* x, void* y, size_t rows, size_t cols, int cluster,
                             cudaStream_t s) {
   const size_t cl = static_cast<size_t>(cluster);
-  size_t groups = rows;
-  if (groups > kMaxGrid / cl) groups = kMaxGrid / cl;
-  return launch(softmax_twophase_kernel<T, ALIGNED>, groups * cl, kTwoPhaseThreads, cluster, s,
-                static_cast<const T*>(x), static_cast<T*>(y), rows, cols);
+  const size_t max_rows = kMaxGrid / cl;
+  for (size_t r0 = 0; r0 < rows; r0 += max_rows) {
+    const size_t n = (rows - r0 < max_rows) ? rows - r0 : max_rows;
+    const cudaError_t e = launch(softmax_twophase_kernel<T, ALIGNED>, n * cl, kTwoPhaseThreads, cluster, s,
+                                 static_cast<const T*>(x) + r0 * cols, static_cast<T*>(y) + r0 * cols, n, cols);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename T, bool ALIGNED>
@@ -442,9 +554,9 @@ cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
                          const fk_softmax_plan& p, cudaStream_t s) {
   switch (p.path) {
     case FK_PATH_WARP: return launch_warp<T, ALIGNED>(x, y, rows, cols, p.vpt, s);
-    case FK_PATH_CTA: return launch_block<T, ALIGNED, false>(x, y, rows, cols, p.threads, p.vpt, 1, s);
+    case FK_PATH_CTA: return launch_block<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, s);
     case FK_PATH_CLUSTER:
-      return launch_block<T, ALIGNED, true>(x, y, rows, cols, p.threads, p.vpt, p.cluster, s);
+      return launch_cluster<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, p.cluster, s);
     case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED>(x, y, rows, cols, p.cluster, s);
     default: return cudaErrorInvalidValue;
   }
@@ -462,6 +574,20 @@ cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int
   }
   return aligned ? launch_typed<__nv_bfloat16, true>(x, y, rows, cols, plan, stream)
                  : launch_typed<__nv_bfloat16, false>(x, y, rows, cols, plan, stream);
+}
+
+cudaError_t read_wait_timeouts(unsigned* out, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_wait_timeouts, sizeof(unsigned));
+  if (e == cudaSuccess && reset) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned));
+  }
+  return e;
+}
+
+cudaError_t launch_wait_selftest(unsigned timeout_us, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError();
 }
 
 }  // namespace fk

@@ -1,0 +1,91 @@
+// fk_sync.cuh -- thread-block-cluster and mbarrier helpers (sm_90+ PTX, used
+// on sm_100a): cluster rank/size, the split cluster barrier, distributed
+// shared-memory addresses, asynchronous remote stores that complete on the
+// receiver's mbarrier, and a time-bounded mbarrier wait.
+//
+// No wait in libfk is unbounded: bounded_wait() gives up after a time limit,
+// counts the give-up in a device word (read by the host through
+// fk_wait_timeouts) and returns false, so a kernel can never hang the GPU on
+// a partner that does not arrive.
+#pragma once
+
+#include <stdint.h>
+
+namespace fk {
+
+__device__ __forceinline__ unsigned cluster_ctarank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ unsigned cluster_nctarank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Split cluster barrier: arrive without ordering (used right after the
+// mbarrier initialisation, which is published by fence_mbarrier_init), and
+// wait with acquire semantics later, once other work has hidden its latency.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Address of the same shared-memory variable in block `rank` of this cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, unsigned rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(local)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisations visible to the other blocks of the cluster
+// (and to the asynchronous proxy).
+__device__ __forceinline__ void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Arrive once on `bar` and expect `bytes` more of asynchronous transactions
+// in the current phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Store (a, b) into another block's shared memory at cluster address `dst`;
+// the 8 bytes complete a transaction on that block's mbarrier `dst_bar`.
+__device__ __forceinline__ void st_async_f2(uint32_t dst, float a, float b, uint32_t dst_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst),
+      "f"(a), "f"(b), "r"(dst_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+}  // namespace fk

@@ -9,7 +9,7 @@ def test_library_exports_every_declared_entry_point(fk):
     names = fk.header_functions()
     assert set(names) >= {"fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex",
                           "fk_softmax_rows_plan", "fk_status_string", "fk_last_cuda_error",
-                          "fk_version"}
+                          "fk_version", "fk_wait_timeouts", "fk_wait_selftest"}
     lib = ctypes.CDLL(fk.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -26,7 +26,7 @@ def test_version_and_status_strings(fk):
     (256, 1000, 0, ("warp", 256, 8, 1)),        # 256x1000 fp32
     (8192, 4096, 0, ("cta", 128, 8, 1)),        # 8192x4096 fp32
     (1 << 20, 2048, 1, ("cta", 128, 2, 1)),     # bf16 attention rows
-    (512, 131072, 0, ("cluster", 512, 8, 8)),   # vocab-sized rows
+    (512, 131072, 0, ("cluster", 128, 16, 16)), # vocab-sized rows
     (4, 1, 0, ("warp", 256, 1, 1)),
     (4, 128, 0, ("warp", 256, 1, 1)),
     (4, 129, 0, ("warp", 256, 2, 1)),
@@ -36,12 +36,12 @@ def test_version_and_status_strings(fk):
     (4, 1024, 1, ("warp", 256, 4, 1)),
     (4, 16385, 1, ("cta", 1024, 4, 1)),
     (4, 32768, 0, ("cta", 1024, 8, 1)),
-    (4, 32769, 0, ("cluster", 512, 8, 3)),
-    (4, 131073, 0, ("cluster", 1024, 8, 5)),
-    (4, 524288, 0, ("cluster", 1024, 8, 16)),
+    (4, 32769, 0, ("cluster", 128, 16, 5)),
+    (4, 131073, 0, ("cluster", 256, 16, 9)),
+    (4, 524288, 0, ("cluster", 512, 16, 16)),
     (4, 524289, 0, ("twophase", 512, 4, 16)),
     (4, 524289, 1, ("twophase", 512, 2, 16)),
-    (4, 524288, 1, ("cluster", 1024, 4, 16)),
+    (4, 524288, 1, ("cluster", 512, 8, 16)),
 ])
 def test_auto_plans(fk, rows, cols, dtype, expect):
     p = fk.fk_softmax_rows_plan(rows, cols, dtype).as_dict()
@@ -116,3 +116,18 @@ def test_explicit_plan_validation(fk):
     # a plan that cannot hold the row
     assert fk.fk_softmax_rows_ex(A, B, 4, 5000, 0, fk.make_plan(fk.FK_PATH_CTA, threads=128), 0) \
         == fk.FK_ERR_INVALID_ARG
+
+
+def test_wait_entry_points_check_arguments_first(fk):
+    assert fk.lib().fk_wait_selftest(0, None) == fk.FK_ERR_INVALID_ARG
+    assert fk.lib().fk_wait_selftest(10_000_001, None) == fk.FK_ERR_INVALID_ARG
+    assert fk.lib().fk_wait_timeouts(None, 0) == fk.FK_ERR_INVALID_ARG
+
+
+def test_cluster_plan_validation(fk):
+    P = fk
+    # 64 values per thread fit blocks of at most 512 threads
+    ok = P.make_plan(P.FK_PATH_CLUSTER, threads=512, vpt=16, cluster=16)
+    bad = P.make_plan(P.FK_PATH_CLUSTER, threads=1024, vpt=16, cluster=16)
+    assert P.fk_softmax_rows_ex(A, B, 4, 1000, 0, bad, 0) == P.FK_ERR_INVALID_ARG
+    assert P.fk_softmax_rows_ex(A, B, 4, 1000, 0, ok, 0) in REJECT_NO_LAUNCH

@@ -80,7 +80,10 @@ def _forced_plans(fk, cols, dtype):
         for t in (128, 256, 512, 1024):
             if t * ept >= cols:
                 plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t, vpt=ept // vec))
-        for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (1024, 16)):
+    for ept in (16, 32, 64):
+        for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (512, 16), (1024, 16)):
+            if ept == 64 and t > 512:
+                continue
             if -(-(-(-cols // vec)) // k) * vec <= t * ept:
                 plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k, vpt=ept // vec))
     for k in (1, 2, 3, 16):
@@ -164,3 +167,21 @@ def test_api_rejects_overlap_and_out_of_range(fk, torch_mod):
     y = torch.empty(4096, device="cuda")
     assert fk.fk_softmax_rows(x.data_ptr(), y.data_ptr(), 1 << 30, 4096, fk.FK_F32, 0) \
         == fk.FK_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("cols", [3, 1000, 2048, 4096, 131072, 600000])
+def test_bf16_outputs_in_the_subnormal_range_round_correctly(fk, torch_mod, cols):
+    # One entry at 0, the rest at -88 .. -95: exp() of those lies below
+    # 2^-126, so the correctly rounded bf16 outputs are subnormals down to
+    # 2^-133 (or 0); each must still be within 1 ulp of the oracle's rounding.
+    x = np.zeros((2, cols), np.float32)
+    x[:, 1:] = -88.0 - (np.arange(cols - 1) % 8)
+    x[1] = np.roll(x[1], cols // 2)
+    xb = synth.f32_to_bf16_bits(x)
+    yb = run(fk, torch_mod, xb)
+    check(xb, yb)
+    ref = oracle.softmax_rows_bf16(xb)
+    sub = ((ref & 0x7F80) == 0) & ((ref & 0x7F) != 0)
+    assert sub.any()  # the case really reaches bf16 subnormals
+    # fp32: the same rows stay within the absolute tolerance
+    check(x, run(fk, torch_mod, x))
