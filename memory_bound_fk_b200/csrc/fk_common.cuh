@@ -29,6 +29,14 @@ __device__ __forceinline__ float ex2_ftz(float v) {
   return r;
 }
 
+// 1/v with MUFU.RCP, at most 1 ulp off; v must be a normal number >= 1
+// (true for every softmax normaliser here).
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -120,6 +128,24 @@ struct Elem<float> {
   // exp2 for softmax terms: results below 2^-126 flush to zero, an absolute
   // error under 1.2e-38 on an fp32 output (3% faster on 4096-column rows).
   __device__ __forceinline__ static float exp2(float a) { return ex2_ftz(a); }
+  // Exponent offset of the single-reference (folded) path: none for fp32.
+  static constexpr float kFoldBias = 0.0f;
+  // 1 / (row sum), correctly rounded.  (MUFU.RCP alone made the compiler
+  // schedule the 32-value rows into 76 registers or spills.)
+  __device__ __forceinline__ static float recip(float s) { return __frcp_rn(s); }
+  // Max of N raw vectors (4 independent accumulators).
+  template <int N>
+  __device__ __forceinline__ static float max_raw(const uint4* r) {
+    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      a[0] = fmaxf(a[0], __uint_as_float(r[i].x));
+      a[1] = fmaxf(a[1], __uint_as_float(r[i].y));
+      a[2] = fmaxf(a[2], __uint_as_float(r[i].z));
+      a[3] = fmaxf(a[3], __uint_as_float(r[i].w));
+    }
+    return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+  }
 };
 
 // bf16 (stored as raw 16-bit patterns): 8 values per 16-byte vector.
@@ -154,8 +180,34 @@ struct Elem<__nv_bfloat16> {
     *p = __float2bfloat16_rn(v);
   }
   // exp2 for softmax terms: subnormal results kept, because bf16 outputs
-  // down to 2^-133 must still round correctly (no measurable cost here).
+  // down to 2^-133 must still round correctly.
   __device__ __forceinline__ static float exp2(float a) { return ex2(a); }
+  // Single-reference (folded) path: exponentials are taken as 2^(a + 64)
+  // with the flush-to-zero MUFU.EX2 (one instruction, against several for the
+  // subnormal-preserving form).  The common factor 2^64 cancels against the
+  // sum; terms whose unscaled value is below 2^-190 flush to 0, and their
+  // correctly rounded bf16 output is 0 anyway (the smallest bf16 is 2^-133
+  // and the normaliser is >= 1), while terms down to 2^-190 stay normal and
+  // reach the bf16 subnormal range through the final multiplication.
+  static constexpr float kFoldBias = 64.0f;
+  // 1 / (row sum) with MUFU.RCP: at most 1 ulp off, invisible after rounding
+  // to bf16; the sum is >= 2^64 here, so never subnormal.
+  __device__ __forceinline__ static float recip(float s) { return rcp_approx(s); }
+  // Max of N raw vectors with packed bf16x2 maximum (exact: the max of bf16
+  // values is one of them).
+  template <int N>
+  __device__ __forceinline__ static float max_raw(const uint4* r) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(-INFINITY, -INFINITY), b = a;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162*>(&r[i].x));
+      b = __hmax2(b, *reinterpret_cast<const __nv_bfloat162*>(&r[i].y));
+      a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162*>(&r[i].z));
+      b = __hmax2(b, *reinterpret_cast<const __nv_bfloat162*>(&r[i].w));
+    }
+    a = __hmax2(a, b);
+    return fmaxf(__low2float(a), __high2float(a));
+  }
 };
 
 }  // namespace fk

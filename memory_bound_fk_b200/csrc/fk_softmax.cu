@@ -97,26 +97,28 @@ __device__ __forceinline__ float exp_ref(float m) { return (m == -INFINITY) ? 0.
 
 // ---------------------------------------------------------------- row I/O
 
-// Load VPT chunks of a team slice into registers (VPT * VEC floats).
+// Load VPT chunks of a team slice as raw 16-byte words (VPT * VEC values).
 // Vectors [vfirst, ve) of the row are the slice; anything outside is -inf.
+// The scalar (unaligned) path packs its scalar loads into the same layout.
 template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
 __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, int t,
-                                            float* v) {
+                                            uint4* raw) {
   constexpr int VEC = Elem<T>::VEC;
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
     if constexpr (ALIGNED) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      Elem<T>::unpack(ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, vi < ve, Elem<T>::kNegInfWord),
-                      v + c * VEC);
+      raw[c] = ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, vi < ve, Elem<T>::kNegInfWord);
     } else {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
       const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+      float f[VEC];
 #pragma unroll
       for (int k = 0; k < VEC; ++k) {
         const Idx e = e0 + static_cast<Idx>(k) * TEAM;
-        v[c * VEC + k] = (e < eend) ? Elem<T>::load1(row + e) : -INFINITY;
+        f[k] = (e < eend) ? Elem<T>::load1(row + e) : -INFINITY;
       }
+      raw[c] = Elem<T>::pack(f);  // exact: the values are already of type T
     }
   }
 }
@@ -146,21 +148,61 @@ __device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx col
   }
 }
 
-// Exponentials of v relative to ref, in place; returns their sum (four
-// accumulators).  FOLD: ref*log2(e) folded into one FMA per element (used
-// when every exponential of the row shares the reference, so the rounding of
-// ref*log2(e) is a common factor that cancels in the normalisation).
-// Otherwise (x - ref) is formed first, exact for the largest terms.
-template <typename T, int E, bool FOLD>
-__device__ __forceinline__ float exp_sum(float* v, float ref) {
+// Exponentials relative to ref, into v; returns their sum (four
+// accumulators).  fp32 works in place on v (already unpacked at load); bf16
+// unpacks the raw words as it goes, so the packed row is what stays live
+// while the max is taken.
+// FOLD (every exponential of the row shares the reference): one FMA and one
+// flush-to-zero MUFU.EX2 per element, 2^(x log2 e - ref log2 e + bias); the
+// rounding of ref*log2(e) and the 2^bias scale are common factors that
+// cancel in the normalisation (bias: see Elem<T>::kFoldBias).
+// Otherwise (blocks or chunks with different references are merged later):
+// (x - ref) is formed first, exact for the largest terms, and no bias is
+// applied, so the partial sums of different references compare directly.
+template <typename T, int VPT, bool FOLD>
+__device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref) {
+  constexpr int VEC = Elem<T>::VEC;
   float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  const float refL = ref * kLog2e;
+  const float c = Elem<T>::kFoldBias - ref * kLog2e;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    v[e] = FOLD ? Elem<T>::exp2(fmaf(v[e], kLog2e, -refL)) : Elem<T>::exp2((v[e] - ref) * kLog2e);
-    s[e & 3] += v[e];
+  for (int i = 0; i < VPT; ++i) {
+    float f[VEC];
+    if constexpr (sizeof(T) == 4) {
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) f[k] = v[i * VEC + k];
+    } else {
+      Elem<T>::unpack(raw[i], f);
+    }
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) {
+      const float e = FOLD ? ex2_ftz(fmaf(f[k], kLog2e, c)) : Elem<T>::exp2((f[k] - ref) * kLog2e);
+      v[i * VEC + k] = e;
+      s[k & 3] += e;
+    }
   }
   return (s[0] + s[1]) + (s[2] + s[3]);
+}
+
+// Row loads: raw 16-byte words; fp32 rows are unpacked into v at once (the
+// same bits), bf16 rows stay packed until exp_sum.
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+__device__ __forceinline__ void load_row(const T* row, Idx vfirst, Idx ve, Idx cols, int t, uint4* raw,
+                                         float* v) {
+  load_chunks<T, VPT, TEAM, ALIGNED, Idx>(row, vfirst, ve, cols, t, raw);
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) Elem<T>::unpack(raw[i], v + i * Elem<T>::VEC);
+  }
+}
+
+// Max of the values a thread holds (after load_row).
+template <typename T, int VPT>
+__device__ __forceinline__ float row_max(const uint4* raw, const float* v) {
+  if constexpr (sizeof(T) == 4) {
+    return max_of<VPT * Elem<T>::VEC>(v);
+  } else {
+    return Elem<T>::template max_raw<VPT>(raw);
+  }
 }
 
 // ---------------------------------------------------------------- warp path
@@ -177,11 +219,12 @@ __global__ void __launch_bounds__(kWarpThreads)
        row < rows; row += stride) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
+    uint4 raw[VPT];
     float v[E];
-    load_chunks<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, v);
-    const float m = warp_max(max_of<E>(v));
-    const float s = warp_sum(exp_sum<T, E, true>(v, m));
-    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, __frcp_rn(s));
+    load_row<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, raw, v);
+    const float m = warp_max(row_max<T, VPT>(raw, v));
+    const float s = warp_sum(exp_sum<T, VPT, true>(raw, v, m));
+    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, Elem<T>::recip(s));
   }
 }
 
@@ -245,24 +288,25 @@ __global__ void __launch_bounds__(THREADS)
   for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
+    uint4 raw[VPT];
     float v[E];
-    load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, 0, nvec, cols, t, v);
+    load_row<T, VPT, THREADS, ALIGNED, int>(xr, 0, nvec, cols, t, raw, v);
 
-    float m = warp_max(max_of<E>(v));
+    float m = warp_max(row_max<T, VPT>(raw, v));
     if (lane == 0) red_max[warp] = m;
     __syncthreads();
     m = red_max[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
 
-    float s = warp_sum(exp_sum<T, E, true>(v, m));
+    float s = warp_sum(exp_sum<T, VPT, true>(raw, v, m));
     if (lane == 0) red_sum[warp] = s;
     __syncthreads();
     s = red_sum[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) s += red_sum[w];
 
-    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, 0, nvec, cols, t, v, __frcp_rn(s));
+    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, 0, nvec, cols, t, v, Elem<T>::recip(s));
     __syncthreads();  // red_max / red_sum are rewritten by the next row
   }
 }
@@ -299,10 +343,11 @@ __global__ void __launch_bounds__(THREADS)
 
   const T* xr = x + row * static_cast<size_t>(cols);
   T* yr = y + row * static_cast<size_t>(cols);
+  uint4 raw[VPT];
   float v[E];
-  load_chunks<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, v);
+  load_row<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, raw, v);
 
-  float m = warp_max(max_of<E>(v));
+  float m = warp_max(row_max<T, VPT>(raw, v));
   if (lane == 0) red_max[warp] = m;
   __syncthreads();
   m = red_max[0];
@@ -311,7 +356,7 @@ __global__ void __launch_bounds__(THREADS)
 
   // Blocks use different references, so the exponent difference is formed
   // first (exact for the largest terms) instead of folded into an FMA.
-  float s = warp_sum(exp_sum<T, E, false>(v, exp_ref(m)));
+  float s = warp_sum(exp_sum<T, VPT, false>(raw, v, exp_ref(m)));
   if (lane == 0) red_sum[warp] = s;
   __syncthreads();
   s = red_sum[0];
@@ -364,10 +409,11 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
     // pass 1: running (m, l) per thread over the streamed chunks
     float m = -INFINITY, l = 0.0f;
     for (size_t c = vb; c < ve; c += CHUNK) {
+      uint4 raw[VPT];
       float v[E];
-      load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
-      const float mn = fmaxf(m, max_of<E>(v));
-      const float acc = exp_sum<T, E, false>(v, exp_ref(mn));
+      load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
+      const float mn = fmaxf(m, row_max<T, VPT>(raw, v));
+      const float acc = exp_sum<T, VPT, false>(raw, v, exp_ref(mn));
       l = l * rescale(m, mn) + acc;
       m = mn;
     }
@@ -397,10 +443,10 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
     const float r = __frcp_rn(l);
     const float ref = exp_ref(m);
     for (size_t c = vb; c < ve; c += CHUNK) {
+      uint4 raw[VPT];
       float v[E];
-      load_chunks<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, v);
-#pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = Elem<T>::exp2((v[e] - ref) * kLog2e);
+      load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
+      exp_sum<T, VPT, false>(raw, v, ref);
       store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
     }
   }
