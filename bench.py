@@ -476,6 +476,107 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
             "ms_per_step": round(ms / steps, 3), "chunks_per_step": len(chunks), "streams": 2}
 
 
+# ---------------------------------------------------------------- unfused comparison
+
+GELU_C = 0.7978845608028654  # sqrt(2/pi)
+
+
+def gelu_unfused(x):
+    """tanh-GELU as the printed formula, one PyTorch eager op (one kernel,
+    one full read and write of a tensor) per step."""
+    import torch
+    a = torch.pow(x, 3)
+    a = a * 0.044715
+    a = x + a
+    a = a * GELU_C
+    a = torch.tanh(a)
+    a = 1.0 + a
+    a = x * a
+    return 0.5 * a
+
+
+def softmax_unfused(x):
+    """'Manual' row softmax: max, subtract, exp, sum, divide as separate ops."""
+    import torch
+    m = x.max(dim=-1, keepdim=True).values
+    z = x - m
+    e = torch.exp(z)
+    s = e.sum(dim=-1, keepdim=True)
+    return e / s
+
+
+def unfused_traffic_bytes(op: str, tensor_bytes: int) -> int:
+    """HBM bytes of the unfused sequences above if no tensor stays in cache:
+    every op reads its full-size inputs and writes its full-size output
+    (the per-row max and sum are negligible)."""
+    if op == "gelu":
+        reads, writes = 10, 8   # pow, mul, add(2), mul, tanh, add, mul(2), mul
+    else:
+        reads, writes = 5, 3    # max, sub, exp, sum, div
+    return (reads + writes) * tensor_bytes
+
+
+def run_unfused(args) -> dict | None:
+    """Times the unfused PyTorch sequences against libfk's fused kernels on
+    the same device buffers (one GPU; the lecture's 192 MB vs 64 MB claim)."""
+    import torch
+
+    import memory_bound_fk_b200 as fk
+    from memory_bound_fk_b200 import synth
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    fk.lib()
+    names = workload_list(args.workload)
+    host = make_inputs(names, args.rows)
+    out = []
+    for n in names:
+        w = synth.WORKLOADS[n]
+        a = host[n]
+        x = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
+             else torch.from_numpy(a)).to(device)
+        y = torch.empty_like(x)
+        s = torch.cuda.current_stream(device).cuda_stream
+        if w.op == "gelu":
+            unf = lambda: gelu_unfused(x)  # noqa: E731
+            fused = lambda: fk.fk_gelu_tanh(x.data_ptr(), y.data_ptr(), x.numel(), s)  # noqa: E731
+        else:
+            code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+            unf = lambda: softmax_unfused(x)  # noqa: E731
+            fused = lambda: fk.fk_softmax_rows(x.data_ptr(), y.data_ptr(), x.shape[0], x.shape[1], code, s)  # noqa: E731
+        res = {}
+        for label, fn in (("unfused", unf), ("fused", fused)):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize(device)
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record()
+            for _ in range(args.steps):
+                fn()
+            ev1.record()
+            torch.cuda.synchronize(device)
+            res[label] = ev0.elapsed_time(ev1) / args.steps
+        tb = a.nbytes
+        out.append({"workload": n, "shape": list(a.shape), "dtype": w.dtype,
+                    "unfused_ms": round(res["unfused"], 5), "fused_ms": round(res["fused"], 5),
+                    "speedup": round(res["unfused"] / res["fused"], 2),
+                    "unfused_traffic_model_bytes": unfused_traffic_bytes(w.op, tb),
+                    "fused_traffic_bytes": 2 * tb,
+                    "traffic_ratio_model": round(unfused_traffic_bytes(w.op, tb) / (2 * tb), 2)})
+        del x, y
+        torch.cuda.empty_cache()
+    tot_u = sum(o["unfused_ms"] for o in out)
+    tot_f = sum(o["fused_ms"] for o in out)
+    bytes_step = sum(2 * host[n].nbytes for n in names)
+    return {"impl": "unfused", "metric": METRIC, "value": round(bytes_step / (tot_u * 1e-3) / 1e9, 1),
+            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_u, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "detail": describe(names),
+                       "what": "PyTorch eager, one kernel per formula step, vs libfk's fused kernels"},
+            "fused_value": round(bytes_step / (tot_f * 1e-3) / 1e9, 1),
+            "speedup_fused_over_unfused": round(tot_u / tot_f, 2), "workloads": out}
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args) -> dict | None:
@@ -520,7 +621,9 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--impl", choices=["ours", "reference", "unfused"], default="ours",
+                   help="ours: libfk kernels; reference: the CPU oracle; unfused: PyTorch "
+                        "eager op-by-op sequences timed against libfk (one GPU)")
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
                         "cfg3_softmax, cfg4_softmax, cfg5_softmax")
@@ -535,14 +638,19 @@ def parse_args(argv=None):
     p.add_argument("--reference-budget", type=float, default=120.0,
                    help="seconds for the whole --impl reference run")
     a = p.parse_args(argv)
-    if a.warmup < 3 and a.impl == "ours" and a.steps > 10:
+    if a.warmup < 3 and a.impl != "reference" and a.steps > 10:
         p.error("--warmup must be at least 3 for a reported measurement")
     return a
 
 
 def main(argv=None):
     args = parse_args(argv)
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        line = run_reference(args)
+    elif args.impl == "unfused":
+        line = run_unfused(args)
+    else:
+        line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
     if args.impl == "ours" and dist_env()[1] > 1:

@@ -122,3 +122,9 @@ def test_clock_sampler_parses_nvidia_smi_csv(tmp_path):
     s.out, s.proc = f, type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout: 0})()
     r = s.stop()
     assert r == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_traffic_model_of_the_unfused_sequences():
+    t = 32 << 20
+    assert bench.unfused_traffic_bytes("gelu", t) == 18 * t
+    assert bench.unfused_traffic_bytes("softmax", t) == 8 * t
