@@ -20,9 +20,15 @@
  * ---------------------------------------
  * Memory:    every pointer is caller-owned memory that the current CUDA
  *            device can access (cudaMalloc / torch tensors, managed or
- *            mapped pinned host memory).  libfk allocates nothing, holds no
- *            handles and keeps no state besides a per-device properties
- *            cache.  Pageable host memory is rejected (FK_ERR_INVALID_ARG).
+ *            mapped pinned host memory).  Pageable host memory is rejected
+ *            (FK_ERR_INVALID_ARG).  libfk holds no handles and keeps no state
+ *            besides a per-device properties cache.  The only allocation it
+ *            ever makes is the workspace of the split path (FK_PATH_SPLIT:
+ *            very long rows, few of them), a few KiB to at most 8 MiB taken
+ *            stream-ordered on the caller's stream from a private memory pool
+ *            of the library (which keeps up to 64 MiB reserved between calls)
+ *            and released on the same stream; fk_softmax_rows_ws takes a
+ *            caller-provided workspace instead and allocates nothing.
  * Layout:    contiguous; softmax rows are row-major with row stride = cols.
  * Streams:   `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *            default stream).  Calls are asynchronous: the kernel is enqueued
@@ -96,9 +102,12 @@ FK_API fk_status fk_gelu_tanh(const float *x, float *y, size_t n, void *stream);
  *   stream cudaStream_t as void*.
  * Arithmetic: fp32 for both dtypes (bf16 is widened exactly, accumulated in
  * fp32, rounded to nearest even on store).  Each input element is read from
- * HBM once and each output written once, except on the two-phase path for
- * rows longer than a thread-block cluster holds on chip (FK_PATH_TWOPHASE,
- * over 524288 columns of either dtype), which reads the row twice.
+ * HBM once and each output written once, except for rows longer than a
+ * thread-block cluster holds on chip (over 524288 columns of either dtype),
+ * which are read twice: by FK_PATH_SPLIT (every chunk of a row in its own
+ * block, (max, sum) partials in a workspace, see above) when there are fewer
+ * than 4 rows or the rows have 4194304 columns or more, else by
+ * FK_PATH_TWOPHASE (one cluster per row).
  * -inf inputs give exactly 0; a row that is all -inf, or holds a NaN or a
  * +inf, gives NaN throughout.
  */
@@ -111,17 +120,24 @@ typedef enum fk_softmax_path {
     FK_PATH_CTA = 2,      /* one thread block per row, row held in registers */
     FK_PATH_CLUSTER = 3,  /* one thread-block cluster per row, slices in registers,
                              (max, sum) partials merged over distributed shared memory */
-    FK_PATH_TWOPHASE = 4  /* one cluster per row, streamed twice: running (max, sum)
+    FK_PATH_TWOPHASE = 4, /* one cluster per row, streamed twice: running (max, sum)
                              pass, then normalise pass -- any row length */
+    FK_PATH_SPLIT = 5     /* every chunk of every row in its own block: a stats kernel
+                             writes each chunk's (max, sum) to a workspace, a normalise
+                             kernel merges a row's partials -- any row length, any
+                             number of rows, needs workspace */
 } fk_softmax_path;
 
 /* A resolved launch plan.  `threads` = threads per block; `vpt` = 16-byte
- * vectors per thread per chunk; `cluster` = blocks per row (1 for WARP/CTA). */
+ * vectors per thread per step; `cluster` = blocks per row for the cluster
+ * paths (1 otherwise); `chunks` = blocks per row on the split path (derived
+ * from the shape; 1 otherwise). */
 typedef struct fk_softmax_plan {
     int path;
     int threads;
     int vpt;
     int cluster;
+    int chunks;
 } fk_softmax_plan;
 
 /*
@@ -147,6 +163,30 @@ FK_API fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int p
  */
 FK_API fk_status fk_softmax_rows_ex(const void *x, void *y, size_t rows, size_t cols, int dtype,
                              const fk_softmax_plan *plan, void *stream);
+
+/*
+ * fk_softmax_rows_workspace -- device workspace, in bytes, that a softmax
+ * call of this shape and plan needs (0 for every path but FK_PATH_SPLIT;
+ * at most 8 MiB).  Host only.
+ *   plan   NULL or FK_PATH_AUTO = the automatic plan.
+ *   bytes  [out]
+ */
+FK_API fk_status fk_softmax_rows_workspace(size_t rows, size_t cols, int dtype, const fk_softmax_plan *plan,
+                                           size_t *bytes);
+
+/*
+ * fk_softmax_rows_ws -- fk_softmax_rows_ex with caller-provided workspace;
+ * allocates nothing.
+ *   workspace        device memory of at least fk_softmax_rows_workspace
+ *                    bytes, 8-byte aligned, not overlapping x or y (may be
+ *                    NULL when that size is 0).  Its contents on entry do not
+ *                    matter; it must not be used by other work until the
+ *                    call's kernels have finished on `stream`.
+ *   workspace_bytes  its size; too small -> FK_ERR_INVALID_ARG.
+ */
+FK_API fk_status fk_softmax_rows_ws(const void *x, void *y, size_t rows, size_t cols, int dtype,
+                                    const fk_softmax_plan *plan, void *workspace, size_t workspace_bytes,
+                                    void *stream);
 
 /*
  * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a

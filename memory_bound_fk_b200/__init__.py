@@ -10,6 +10,8 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
     fk_softmax_rows(x, y, rows, cols, dtype, stream) -> status
     fk_softmax_rows_ex(x, y, rows, cols, dtype, plan, stream) -> status
     fk_softmax_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
+    fk_softmax_rows_workspace(rows, cols, dtype, plan=None) -> bytes
+    fk_softmax_rows_ws(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, stream) -> status
     fk_status_string(status) -> str
     fk_wait_timeouts(reset=False) -> int     (bounded-wait give-ups, synchronous)
     fk_wait_selftest(timeout_us, stream) -> status
@@ -46,8 +48,9 @@ FK_PATH_WARP = 1
 FK_PATH_CTA = 2
 FK_PATH_CLUSTER = 3
 FK_PATH_TWOPHASE = 4
+FK_PATH_SPLIT = 5
 PATH_NAMES = {FK_PATH_WARP: "warp", FK_PATH_CTA: "cta", FK_PATH_CLUSTER: "cluster",
-              FK_PATH_TWOPHASE: "twophase"}
+              FK_PATH_TWOPHASE: "twophase", FK_PATH_SPLIT: "split"}
 
 
 class FkError(RuntimeError):
@@ -59,11 +62,11 @@ class FkError(RuntimeError):
 
 class SoftmaxPlan(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("threads", ctypes.c_int),
-                ("vpt", ctypes.c_int), ("cluster", ctypes.c_int)]
+                ("vpt", ctypes.c_int), ("cluster", ctypes.c_int), ("chunks", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {"path": PATH_NAMES.get(self.path, self.path), "threads": self.threads,
-                "vpt": self.vpt, "cluster": self.cluster}
+                "vpt": self.vpt, "cluster": self.cluster, "chunks": self.chunks}
 
     def __repr__(self) -> str:
         return f"SoftmaxPlan({self.as_dict()})"
@@ -95,6 +98,11 @@ def lib() -> ctypes.CDLL:
         L.fk_last_cuda_error.restype = ci
         L.fk_version.argtypes = []
         L.fk_version.restype = ci
+        L.fk_softmax_rows_workspace.argtypes = [sz, sz, ci, ctypes.POINTER(SoftmaxPlan),
+                                                ctypes.POINTER(ctypes.c_size_t)]
+        L.fk_softmax_rows_workspace.restype = ci
+        L.fk_softmax_rows_ws.argtypes = [vp, vp, sz, sz, ci, ctypes.POINTER(SoftmaxPlan), vp, sz, vp]
+        L.fk_softmax_rows_ws.restype = ci
         L.fk_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
         L.fk_wait_timeouts.restype = ci
         L.fk_wait_selftest.argtypes = [ctypes.c_uint, vp]
@@ -133,6 +141,22 @@ def fk_softmax_rows_plan(rows: int, cols: int, dtype: int, path: int = FK_PATH_A
     return p
 
 
+def fk_softmax_rows_workspace(rows: int, cols: int, dtype: int, plan: SoftmaxPlan | None = None) -> int:
+    """Workspace bytes a softmax call of this shape (and plan) needs."""
+    b = ctypes.c_size_t(0)
+    st = lib().fk_softmax_rows_workspace(rows, cols, dtype, ctypes.byref(plan) if plan is not None else None,
+                                         ctypes.byref(b))
+    if st != FK_OK:
+        raise FkError(st, "fk_softmax_rows_workspace")
+    return b.value
+
+
+def fk_softmax_rows_ws(x: int, y: int, rows: int, cols: int, dtype: int, plan: SoftmaxPlan | None,
+                       workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return lib().fk_softmax_rows_ws(x, y, rows, cols, dtype, ctypes.byref(plan) if plan is not None else None,
+                                    workspace, workspace_bytes, stream)
+
+
 def fk_status_string(status: int) -> str:
     return lib().fk_status_string(status).decode()
 
@@ -159,8 +183,8 @@ def fk_wait_selftest(timeout_us: int, stream: int = 0) -> int:
     return lib().fk_wait_selftest(timeout_us, stream)
 
 
-def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0) -> SoftmaxPlan:
-    return SoftmaxPlan(path, threads, vpt, cluster)
+def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0, chunks: int = 0) -> SoftmaxPlan:
+    return SoftmaxPlan(path, threads, vpt, cluster, chunks)
 
 
 # ---------------------------------------------------------------- tensors
@@ -204,8 +228,11 @@ def _dtype_code(dt) -> int:
     raise TypeError("softmax_rows takes float32 or bfloat16")
 
 
-def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None):
-    """Softmax over the last dimension of a contiguous fp32/bf16 CUDA tensor."""
+def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None, workspace=None):
+    """Softmax over the last dimension of a contiguous fp32/bf16 CUDA tensor.
+    `workspace` (a CUDA tensor of at least fk_softmax_rows_workspace bytes)
+    makes the call allocation-free; without it the split path allocates its
+    workspace stream-ordered."""
     import torch
     _check_tensor(x, "x")
     code = _dtype_code(x.dtype)
@@ -216,7 +243,12 @@ def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None):
         raise ValueError("out must match x in dtype, shape and device")
     cols = x.shape[-1] if x.dim() > 0 else 1
     rows = x.numel() // cols if cols else 0
-    st = fk_softmax_rows_ex(x.data_ptr(), out.data_ptr(), rows, cols, code, plan, _stream_handle(x))
+    if workspace is not None:
+        _check_tensor(workspace, "workspace")
+        st = fk_softmax_rows_ws(x.data_ptr(), out.data_ptr(), rows, cols, code, plan, workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream_handle(x))
+    else:
+        st = fk_softmax_rows_ex(x.data_ptr(), out.data_ptr(), rows, cols, code, plan, _stream_handle(x))
     if st != FK_OK:
         raise FkError(st, "fk_softmax_rows")
     return out
@@ -225,8 +257,9 @@ def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None):
 __all__ = [
     "FK_OK", "FK_ERR_INVALID_ARG", "FK_ERR_UNSUPPORTED_DTYPE", "FK_ERR_UNSUPPORTED_DEVICE",
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
-    "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FkError", "SoftmaxPlan", "lib", "header_functions",
+    "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
     "fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
+    "fk_softmax_rows_workspace", "fk_softmax_rows_ws",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
     "fk_wait_selftest", "make_plan", "gelu_tanh",
     "softmax_rows",

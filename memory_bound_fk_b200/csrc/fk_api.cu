@@ -28,6 +28,32 @@ DeviceInfo g_info[kMaxDevices];
 std::once_flag g_info_once[kMaxDevices];
 thread_local int t_last_cuda_error = 0;
 
+// Private stream-ordered memory pool per device for the split path's
+// workspace.  Its release threshold keeps up to 64 MiB reserved across
+// synchronisations, so repeated calls reuse memory instead of going back to
+// the driver (the default pool's threshold of 0 made every call a fresh
+// allocation).  A private pool leaves the process-wide default pool as it is.
+std::once_flag g_pool_once[kMaxDevices];
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+cudaMemPool_t workspace_pool(int dev) {
+  std::call_once(g_pool_once[dev], [dev] {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return;
+    }
+    uint64_t keep = uint64_t{64} << 20;
+    (void)cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = pool;
+  });
+  return g_pool[dev];
+}
+
 fk_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return FK_ERR_CUDA;
@@ -161,29 +187,89 @@ fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int path, fk
   return fk::plan_softmax(rows, cols, dtype, path, out);
 }
 
-fk_status fk_softmax_rows_ex(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                             const fk_softmax_plan* plan, void* stream) {
+namespace {
+
+// Resolve the plan of a softmax call (auto or explicit).
+fk_status resolve_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan, fk_softmax_plan* p) {
+  if (plan == nullptr || plan->path == FK_PATH_AUTO) return fk::plan_softmax(rows, cols, dtype, FK_PATH_AUTO, p);
+  return fk::check_plan(rows, cols, dtype, *plan, p);
+}
+
+// Shared body of the softmax entry points.  ws == nullptr and
+// allow_alloc: a needed workspace is allocated stream-ordered.
+fk_status softmax_call(const void* x, void* y, size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan,
+                       void* ws, size_t ws_bytes, bool allow_alloc, void* stream) {
   if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
   if (rows == 0 || cols == 0) return FK_OK;
   if (rows > SIZE_MAX / cols) return FK_ERR_INVALID_ARG;
   fk_softmax_plan p;
-  fk_status st;
-  if (plan == nullptr || plan->path == FK_PATH_AUTO)
-    st = fk::plan_softmax(rows, cols, dtype, FK_PATH_AUTO, &p);
-  else
-    st = fk::check_plan(cols, dtype, *plan, &p);
+  fk_status st = resolve_plan(rows, cols, dtype, plan, &p);
   if (st != FK_OK) return st;
   const size_t esize = dtype == FK_F32 ? 4 : 2;
   const fk::DeviceInfo* dev = nullptr;
   st = fk::check_call(x, y, rows * cols, esize, &dev);
   if (st != FK_OK) return st;
+  const size_t need = fk::workspace_bytes(rows, cols, dtype, p);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bool owned = false;
+  if (need > 0) {
+    if (ws != nullptr) {
+      if (ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % 8) != 0) return FK_ERR_INVALID_ARG;
+      const size_t data = rows * cols * esize;
+      const uintptr_t w = reinterpret_cast<uintptr_t>(ws);
+      const uintptr_t a = reinterpret_cast<uintptr_t>(x), b = reinterpret_cast<uintptr_t>(y);
+      if ((w < a + data && a < w + need) || (w < b + data && b < w + need)) return FK_ERR_INVALID_ARG;
+      int d = -1;
+      if (cudaGetDevice(&d) != cudaSuccess) return FK_ERR_UNSUPPORTED_DEVICE;
+      st = fk::check_pointer(ws, need, d);
+      if (st != FK_OK) return st;
+    } else {
+      if (!allow_alloc) return FK_ERR_INVALID_ARG;
+      int d = -1;
+      if (cudaGetDevice(&d) != cudaSuccess) return FK_ERR_UNSUPPORTED_DEVICE;
+      const cudaMemPool_t pool = fk::workspace_pool(d);
+      const cudaError_t e = pool ? cudaMallocFromPoolAsync(&ws, need, pool, s) : cudaMallocAsync(&ws, need, s);
+      if (e != cudaSuccess) return fk::cuda_fail(e);
+      owned = true;
+    }
+  }
   // 16-byte vector access needs both bases on a 16-byte boundary and a row
   // pitch that is a multiple of 16 bytes.
   const bool aligned = (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
                        (reinterpret_cast<uintptr_t>(y) % 16 == 0) && ((cols * esize) % 16 == 0);
-  const cudaError_t e =
-      fk::launch_softmax(x, y, rows, cols, dtype, p, aligned, *dev, static_cast<cudaStream_t>(stream));
+  cudaError_t e = fk::launch_softmax(x, y, rows, cols, dtype, p, aligned, ws, *dev, s);
+  if (owned) {
+    const cudaError_t f = cudaFreeAsync(ws, s);
+    if (e == cudaSuccess) e = f;
+  }
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+}  // namespace
+
+fk_status fk_softmax_rows_ex(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                             const fk_softmax_plan* plan, void* stream) {
+  return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, stream);
+}
+
+fk_status fk_softmax_rows_ws(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                             const fk_softmax_plan* plan, void* workspace, size_t workspace_bytes, void* stream) {
+  return softmax_call(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, false, stream);
+}
+
+fk_status fk_softmax_rows_workspace(size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan,
+                                    size_t* bytes) {
+  if (bytes == nullptr) return FK_ERR_INVALID_ARG;
+  if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
+  if (rows == 0 || cols == 0) {
+    *bytes = 0;
+    return FK_OK;
+  }
+  fk_softmax_plan p;
+  const fk_status st = resolve_plan(rows, cols, dtype, plan, &p);
+  if (st != FK_OK) return st;
+  *bytes = fk::workspace_bytes(rows, cols, dtype, p);
+  return FK_OK;
 }
 
 fk_status fk_softmax_rows(const void* x, void* y, size_t rows, size_t cols, int dtype, void* stream) {

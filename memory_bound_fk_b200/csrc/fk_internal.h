@@ -39,16 +39,32 @@ constexpr int kMaxCluster = 16;
 // Vectors (16 bytes) per thread implied by a dtype and an element budget.
 int vec_elems(int dtype);  // 4 for fp32, 8 for bf16
 
+// Geometry of the split path (FK_PATH_SPLIT): each row is cut into nchunks
+// chunks of chunk_vecs 16-byte vectors, one block per chunk; rows go in
+// batches of rows_per_launch, whose partials fit ws_bytes of workspace.
+struct SplitGeometry {
+  size_t chunk_vecs;
+  unsigned nchunks;
+  size_t rows_per_launch;
+  size_t ws_bytes;
+};
+SplitGeometry split_geometry(size_t rows, size_t cols, int dtype);
+
 // Host-only plan (see fk_softmax_rows_plan in fk.h).
 fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out);
 // Validate a caller-provided plan and fill defaults.
-fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out);
+fk_status check_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out);
 
 // Launch a validated plan.  `aligned` = rows and both pointers allow 16-byte
 // vector access.
+// `ws` is device workspace of at least workspace_bytes(plan) bytes (only the
+// split path uses it; may be null otherwise).
 cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                           const fk_softmax_plan& plan, bool aligned, const DeviceInfo& dev,
+                           const fk_softmax_plan& plan, bool aligned, void* ws, const DeviceInfo& dev,
                            cudaStream_t stream);
+
+// Workspace bytes a validated plan needs (0 except on the split path).
+size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan);
 
 // Number of threads whose bounded mbarrier wait gave up, on the current
 // device; optionally reset to 0.  Synchronous.

@@ -7,7 +7,11 @@
 //              {128, 256, 512, 1024} -> up to 32768 columns
 //   cluster  : 2..16 blocks of 128..512 threads holding 64 values each
 //              -> up to 524288 columns
-//   twophase : any length (row streamed twice)
+//   twophase : any length; one cluster per row streams it twice
+//   split    : any length; every chunk of every row gets its own block, and a
+//              small workspace carries the chunks' (max, sum) partials --
+//              the choice for long rows when there are too few rows to give
+//              one cluster each and still fill the GPU
 // The automatic choice takes the smallest shape that holds the row on chip,
 // so a row is read from HBM once whenever it fits in a cluster.  Measured on
 // B200 (L2 cleaned between runs): 4096-column fp32 rows run best as one
@@ -38,11 +42,47 @@ size_t block_cap(int threads, int ept) { return static_cast<size_t>(threads) * e
 
 bool ept_ok(int ept) { return ept == kBlockEptSmall || ept == kBlockEptLarge; }
 
+constexpr size_t kSplitFillBlocks = 148 * 8;     // blocks that fill a B200 several times over
+constexpr size_t kSplitMaxIters = 32;             // streamed steps per block at most
+constexpr size_t kSplitMaxPartials = size_t{1} << 20;  // workspace: 8 MiB of partials at most
+// Long rows (past cluster capacity) use the split path when there are fewer
+// than kSplitBelowRows rows, or when rows have kSplitFromCols columns or more;
+// otherwise one cluster per row streams it twice.  Measured on B200 (fp32,
+// L2 cleaned): at 1M columns the cluster path wins from 4 to 32 rows (e.g.
+// 2.18 vs 1.99 TB/s at 8 rows) and they tie from 64 rows; at 4M and 16M
+// columns the split path wins at every row count (1.43 vs 0.47 TB/s at one
+// row of 4M, 3.05 vs 0.52 at one row of 16M, 4.37 vs 4.18 at 128 rows of 4M).
+constexpr size_t kSplitBelowRows = 4;
+constexpr size_t kSplitFromCols = size_t{1} << 22;
+
 bool cluster_ept_ok(int ept, int threads) {
   return ept_ok(ept) || (ept == kClusterEpt && threads <= 512);
 }
 
 }  // namespace
+
+SplitGeometry split_geometry(size_t rows, size_t cols, int dtype) {
+  const size_t vec = static_cast<size_t>(vec_elems(dtype));
+  const size_t unit = static_cast<size_t>(kTwoPhaseThreads) * (kTwoPhaseElemsPerThread / vec);  // vectors/step
+  const size_t nvec = ceil_div(cols, vec);
+  size_t want = ceil_div(kSplitFillBlocks, rows > 0 ? rows : 1);
+  const size_t by_len = ceil_div(nvec, unit * kSplitMaxIters);
+  if (want < by_len) want = by_len;
+  if (want < 1) want = 1;
+  SplitGeometry g;
+  g.chunk_vecs = ceil_div(ceil_div(nvec, want), unit) * unit;
+  g.nchunks = static_cast<unsigned>(ceil_div(nvec, g.chunk_vecs));
+  size_t rpl = kSplitMaxPartials / g.nchunks;
+  if (rpl < 1) rpl = 1;
+  if (rpl > rows) rpl = rows > 0 ? rows : 1;
+  g.rows_per_launch = rpl;
+  g.ws_bytes = rpl * g.nchunks * 8;
+  return g;
+}
+
+size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan) {
+  return plan.path == FK_PATH_SPLIT ? split_geometry(rows, cols, dtype).ws_bytes : 0;
+}
 
 fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out) {
   (void)rows;
@@ -60,10 +100,12 @@ fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax
       path = FK_PATH_CTA;
     else if (cols <= static_cast<size_t>(kMaxCluster) * block_cap(1024, kBlockEptLarge))
       path = FK_PATH_CLUSTER;
+    else if (rows < kSplitBelowRows || cols >= kSplitFromCols)
+      path = FK_PATH_SPLIT;
     else
       path = FK_PATH_TWOPHASE;
   }
-  fk_softmax_plan p = {path, 0, 0, 1};
+  fk_softmax_plan p = {path, 0, 0, 1, 1};
   switch (path) {
     case FK_PATH_WARP: {
       int vpt = 1;
@@ -108,6 +150,13 @@ fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax
       p.cluster = static_cast<int>(k);
       break;
     }
+    case FK_PATH_SPLIT: {
+      p.threads = kTwoPhaseThreads;
+      p.vpt = kTwoPhaseElemsPerThread / vec;
+      p.cluster = 1;
+      p.chunks = static_cast<int>(split_geometry(rows, cols, dtype).nchunks);
+      break;
+    }
     default:
       return FK_ERR_INVALID_ARG;
   }
@@ -115,11 +164,11 @@ fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax
   return FK_OK;
 }
 
-fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out) {
+fk_status check_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out) {
   if (!valid_dtype(dtype)) return FK_ERR_UNSUPPORTED_DTYPE;
   const int vec = vec_elems(dtype);
   fk_softmax_plan d;
-  const fk_status st = plan_softmax(1, cols, dtype, in.path, &d);
+  const fk_status st = plan_softmax(rows, cols, dtype, in.path, &d);
   if (st != FK_OK) {
     // the default for this path may not hold cols, but an explicit plan could
     if (in.path != FK_PATH_CTA && in.path != FK_PATH_CLUSTER) return st;
@@ -156,9 +205,17 @@ fk_status check_plan(size_t cols, int dtype, const fk_softmax_plan& in, fk_softm
         return FK_ERR_INVALID_ARG;
       if (p.cluster < 1 || p.cluster > kMaxCluster) return FK_ERR_INVALID_ARG;
       break;
+    case FK_PATH_SPLIT:
+      // the chunking is derived from the shape; only the defaults are accepted
+      if (p.threads != kTwoPhaseThreads || p.vpt != kTwoPhaseElemsPerThread / vec || p.cluster != 1)
+        return FK_ERR_INVALID_ARG;
+      if (in.chunks != 0 && in.chunks != d.chunks) return FK_ERR_INVALID_ARG;
+      p.chunks = d.chunks;
+      break;
     default:
       return FK_ERR_INVALID_ARG;
   }
+  if (p.path != FK_PATH_SPLIT) p.chunks = 1;
   *out = p;
   return FK_OK;
 }

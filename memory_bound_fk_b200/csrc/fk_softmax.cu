@@ -375,19 +375,71 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
   m = M;
 }
 
+// Streaming pass 1 over vectors [vb, ve) of a row: running (m, l) per thread
+// (the online recurrence of lecture 6, section 7.2), chunk by chunk.
+template <typename T, int THREADS, int VPT, bool ALIGNED>
+__device__ __forceinline__ void stream_stats(const T* xr, size_t vb, size_t ve, size_t cols, int t, float& m,
+                                             float& l) {
+  constexpr int E = VPT * Elem<T>::VEC;
+  constexpr size_t STEP = static_cast<size_t>(THREADS) * VPT;
+  for (size_t c = vb; c < ve; c += STEP) {
+    uint4 raw[VPT];
+    float v[E];
+    load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
+    const float mn = fmaxf(m, row_max<T, VPT>(raw, v));
+    const float acc = exp_sum<T, VPT, false>(raw, v, exp_ref(mn));
+    l = l * rescale(m, mn) + acc;
+    m = mn;
+  }
+}
+
+// Merge every thread's (m, l) of the block; all threads get the result.
+// `red` holds THREADS/32 entries; the caller must not reuse it before a
+// following __syncthreads.
+template <int THREADS>
+__device__ __forceinline__ void block_merge_ml(float& m, float& l, float2* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+    merge_ml(m, l, m2, l2);
+  }
+  if (lane == 0) red[warp] = make_float2(m, l);
+  __syncthreads();
+  m = red[0].x;
+  l = red[0].y;
+#pragma unroll
+  for (int w = 1; w < THREADS / 32; ++w) merge_ml(m, l, red[w].x, red[w].y);
+}
+
+// Streaming pass 2 over vectors [vb, ve): y = exp(x - M) / L.
+template <typename T, int THREADS, int VPT, bool ALIGNED>
+__device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, size_t ve, size_t cols, int t,
+                                                 float M, float L) {
+  constexpr int E = VPT * Elem<T>::VEC;
+  constexpr size_t STEP = static_cast<size_t>(THREADS) * VPT;
+  const float r = __frcp_rn(L);
+  const float ref = exp_ref(M);
+  for (size_t c = vb; c < ve; c += STEP) {
+    uint4 raw[VPT];
+    float v[E];
+    load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
+    exp_sum<T, VPT, false>(raw, v, ref);
+    store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
+  }
+}
+
 template <typename T, bool ALIGNED>
 __global__ void __launch_bounds__(kTwoPhaseThreads)
     softmax_twophase_kernel(const T* x, T* y, size_t rows, size_t cols) {
   constexpr int THREADS = kTwoPhaseThreads;
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
-  constexpr int E = VPT * VEC;
-  constexpr int NW = THREADS / 32;
-  constexpr size_t CHUNK = static_cast<size_t>(THREADS) * VPT;  // vectors per chunk
-  __shared__ float2 red[NW];
+  __shared__ float2 red[THREADS / 32];
   __shared__ __align__(16) ClusterExchange ex;
 
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int t = threadIdx.x;
   const int csize = static_cast<int>(cluster_nctarank());  // 1 without a cluster launch
   const int crank = static_cast<int>(cluster_ctarank());
   const size_t nvec = (cols + VEC - 1) / VEC;
@@ -402,54 +454,72 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
     if (t == 0) exchange_init(ex);
     cluster_arrive_relaxed();
   }
-  {
-    const T* xr = x + row * cols;
-    T* yr = y + row * cols;
+  const T* xr = x + row * cols;
+  T* yr = y + row * cols;
 
-    // pass 1: running (m, l) per thread over the streamed chunks
-    float m = -INFINITY, l = 0.0f;
-    for (size_t c = vb; c < ve; c += CHUNK) {
-      uint4 raw[VPT];
-      float v[E];
-      load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
-      const float mn = fmaxf(m, row_max<T, VPT>(raw, v));
-      const float acc = exp_sum<T, VPT, false>(raw, v, exp_ref(mn));
-      l = l * rescale(m, mn) + acc;
-      m = mn;
-    }
+  // pass 1: running (m, l) per thread, then merged over the block
+  float m = -INFINITY, l = 0.0f;
+  stream_stats<T, THREADS, VPT, ALIGNED>(xr, vb, ve, cols, t, m, l);
+  block_merge_ml<THREADS>(m, l, red);
 
-    // merge the threads' partials: warp, then block
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-      const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-      merge_ml(m, l, m2, l2);
-    }
-    if (lane == 0) red[warp] = make_float2(m, l);
-    __syncthreads();
-    m = red[0].x;
-    l = red[0].y;
-#pragma unroll
-    for (int w = 1; w < NW; ++w) merge_ml(m, l, red[w].x, red[w].y);
-
-    // merge the blocks' partials across the cluster
-    if (csize > 1) {
-      const float2 ML = exchange_merge(ex, m, l, csize, crank);
-      m = ML.x;
-      l = ML.y;
-    }
-
-    // pass 2: y = exp(x - M) / L
-    const float r = __frcp_rn(l);
-    const float ref = exp_ref(m);
-    for (size_t c = vb; c < ve; c += CHUNK) {
-      uint4 raw[VPT];
-      float v[E];
-      load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
-      exp_sum<T, VPT, false>(raw, v, ref);
-      store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
-    }
+  // merge the blocks' partials across the cluster
+  if (csize > 1) {
+    const float2 ML = exchange_merge(ex, m, l, csize, crank);
+    m = ML.x;
+    l = ML.y;
   }
+
+  // pass 2: y = exp(x - M) / L
+  stream_normalise<T, THREADS, VPT, ALIGNED>(xr, yr, vb, ve, cols, t, m, l);
+}
+
+// ---------------------------------------------------------------- split path
+
+// Rows longer than a cluster holds, split over the whole grid: block b covers
+// vectors [c * chunk, (c + 1) * chunk) of row b / nchunks, c = b % nchunks.
+// The stats kernel writes each chunk's (max, sum) partial to the workspace;
+// the normalise kernel (next on the stream) merges the row's partials with
+// the running-max rule and writes exp(x - M) / L for its chunk.  Every block
+// is independent (no waits), and the number of blocks does not depend on the
+// number of rows.
+
+template <typename T, bool ALIGNED>
+__global__ void __launch_bounds__(kTwoPhaseThreads)
+    softmax_split_stats_kernel(const T* x, float2* ws, size_t cols, size_t chunk, unsigned nchunks) {
+  constexpr int THREADS = kTwoPhaseThreads;
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
+  __shared__ float2 red[THREADS / 32];
+  const size_t row = blockIdx.x / nchunks;
+  const size_t c = blockIdx.x % nchunks;
+  const size_t nvec = (cols + VEC - 1) / VEC;
+  const size_t vb = imin(nvec, c * chunk);
+  const size_t ve = imin(nvec, vb + chunk);
+  float m = -INFINITY, l = 0.0f;
+  stream_stats<T, THREADS, VPT, ALIGNED>(x + row * cols, vb, ve, cols, threadIdx.x, m, l);
+  block_merge_ml<THREADS>(m, l, red);
+  if (threadIdx.x == 0) ws[blockIdx.x] = make_float2(m, l);
+}
+
+template <typename T, bool ALIGNED>
+__global__ void __launch_bounds__(kTwoPhaseThreads)
+    softmax_split_norm_kernel(const T* x, T* y, const float2* ws, size_t cols, size_t chunk,
+                              unsigned nchunks) {
+  constexpr int THREADS = kTwoPhaseThreads;
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
+  __shared__ float2 red[THREADS / 32];
+  const size_t row = blockIdx.x / nchunks;
+  const size_t c = blockIdx.x % nchunks;
+  const size_t nvec = (cols + VEC - 1) / VEC;
+  const size_t vb = imin(nvec, c * chunk);
+  const size_t ve = imin(nvec, vb + chunk);
+  // merge the row's partials
+  const float2* part = ws + row * nchunks;
+  float m = -INFINITY, l = 0.0f;
+  for (unsigned i = threadIdx.x; i < nchunks; i += THREADS) merge_ml(m, l, part[i].x, part[i].y);
+  block_merge_ml<THREADS>(m, l, red);
+  stream_normalise<T, THREADS, VPT, ALIGNED>(x + row * cols, y + row * cols, vb, ve, cols, threadIdx.x, m, l);
 }
 
 // A wait on an mbarrier that nothing ever arrives on: every thread gives up
@@ -595,15 +665,38 @@ cudaError_t launch_twophase(const void* x, void* y, size_t rows, size_t cols, in
   return cudaSuccess;
 }
 
+// Stats then normalise, batch by batch of rows (a batch's partials fit the
+// workspace; batches run in stream order, so the workspace is reused).
+template <typename T, bool ALIGNED>
+cudaError_t launch_split(const void* x, void* y, size_t rows, size_t cols, const SplitGeometry& g, void* ws,
+                         cudaStream_t s) {
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
+  float2* w = static_cast<float2*>(ws);
+  for (size_t r0 = 0; r0 < rows; r0 += g.rows_per_launch) {
+    const size_t n = (rows - r0 < g.rows_per_launch) ? rows - r0 : g.rows_per_launch;
+    const size_t blocks = n * g.nchunks;
+    cudaError_t e = launch(softmax_split_stats_kernel<T, ALIGNED>, blocks, kTwoPhaseThreads, 1, s,
+                           xp + r0 * cols, w, cols, g.chunk_vecs, g.nchunks);
+    if (e != cudaSuccess) return e;
+    e = launch(softmax_split_norm_kernel<T, ALIGNED>, blocks, kTwoPhaseThreads, 1, s, xp + r0 * cols,
+               yp + r0 * cols, static_cast<const float2*>(w), cols, g.chunk_vecs, g.nchunks);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 template <typename T, bool ALIGNED>
 cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
-                         const fk_softmax_plan& p, cudaStream_t s) {
+                         const fk_softmax_plan& p, void* ws, cudaStream_t s) {
   switch (p.path) {
     case FK_PATH_WARP: return launch_warp<T, ALIGNED>(x, y, rows, cols, p.vpt, s);
     case FK_PATH_CTA: return launch_block<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, s);
     case FK_PATH_CLUSTER:
       return launch_cluster<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, p.cluster, s);
     case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED>(x, y, rows, cols, p.cluster, s);
+    case FK_PATH_SPLIT:
+      return launch_split<T, ALIGNED>(x, y, rows, cols, split_geometry(rows, cols, Elem<T>::VEC == 8 ? FK_BF16 : FK_F32), ws, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -611,15 +704,15 @@ cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
 }  // namespace
 
 cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                           const fk_softmax_plan& plan, bool aligned, const DeviceInfo& dev,
+                           const fk_softmax_plan& plan, bool aligned, void* ws, const DeviceInfo& dev,
                            cudaStream_t stream) {
   (void)dev;
   if (dtype == FK_F32) {
-    return aligned ? launch_typed<float, true>(x, y, rows, cols, plan, stream)
-                   : launch_typed<float, false>(x, y, rows, cols, plan, stream);
+    return aligned ? launch_typed<float, true>(x, y, rows, cols, plan, ws, stream)
+                   : launch_typed<float, false>(x, y, rows, cols, plan, ws, stream);
   }
-  return aligned ? launch_typed<__nv_bfloat16, true>(x, y, rows, cols, plan, stream)
-                 : launch_typed<__nv_bfloat16, false>(x, y, rows, cols, plan, stream);
+  return aligned ? launch_typed<__nv_bfloat16, true>(x, y, rows, cols, plan, ws, stream)
+                 : launch_typed<__nv_bfloat16, false>(x, y, rows, cols, plan, ws, stream);
 }
 
 cudaError_t read_wait_timeouts(unsigned* out, bool reset) {

@@ -9,7 +9,8 @@ def test_library_exports_every_declared_entry_point(fk):
     names = fk.header_functions()
     assert set(names) >= {"fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex",
                           "fk_softmax_rows_plan", "fk_status_string", "fk_last_cuda_error",
-                          "fk_version", "fk_wait_timeouts", "fk_wait_selftest"}
+                          "fk_version", "fk_wait_timeouts", "fk_wait_selftest",
+                          "fk_softmax_rows_workspace", "fk_softmax_rows_ws"}
     lib = ctypes.CDLL(fk.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -39,8 +40,12 @@ def test_version_and_status_strings(fk):
     (4, 32769, 0, ("cluster", 128, 16, 5)),
     (4, 131073, 0, ("cluster", 256, 16, 9)),
     (4, 524288, 0, ("cluster", 512, 16, 16)),
+    (3, 524289, 0, ("split", 512, 4, 1)),
     (4, 524289, 0, ("twophase", 512, 4, 16)),
-    (4, 524289, 1, ("twophase", 512, 2, 16)),
+    (64, 524289, 0, ("twophase", 512, 4, 16)),
+    (64, 1 << 22, 0, ("split", 512, 4, 1)),
+    (2, 524289, 1, ("split", 512, 2, 1)),
+    (100, 524289, 1, ("twophase", 512, 2, 16)),
     (4, 524288, 1, ("cluster", 512, 8, 16)),
 ])
 def test_auto_plans(fk, rows, cols, dtype, expect):
@@ -131,3 +136,27 @@ def test_cluster_plan_validation(fk):
     bad = P.make_plan(P.FK_PATH_CLUSTER, threads=1024, vpt=16, cluster=16)
     assert P.fk_softmax_rows_ex(A, B, 4, 1000, 0, bad, 0) == P.FK_ERR_INVALID_ARG
     assert P.fk_softmax_rows_ex(A, B, 4, 1000, 0, ok, 0) in REJECT_NO_LAUNCH
+
+
+def test_split_plan_and_workspace(fk):
+    P = fk
+    p = P.fk_softmax_rows_plan(1, 64 << 20, P.FK_F32).as_dict()
+    assert p["path"] == "split" and p["chunks"] >= 148
+    # the workspace holds one (max, sum) pair per chunk of the rows of a launch
+    ws = P.fk_softmax_rows_workspace(1, 64 << 20, P.FK_F32)
+    assert ws == 8 * p["chunks"]
+    assert P.fk_softmax_rows_workspace(8192, 4096, P.FK_F32) == 0
+    assert P.fk_softmax_rows_workspace(512, 131072, P.FK_BF16) == 0
+    big = P.fk_softmax_rows_workspace(10 ** 6, 1 << 20, P.FK_F32, P.make_plan(P.FK_PATH_SPLIT))
+    assert 0 < big <= 8 << 20
+    # forced split for a short row: one chunk
+    q = P.fk_softmax_rows_plan(3, 100, P.FK_BF16, P.FK_PATH_SPLIT).as_dict()
+    assert q["path"] == "split" and q["chunks"] == 1
+    # explicit chunk counts other than the derived one are refused
+    assert P.fk_softmax_rows_ex(A, B, 3, 100, 0, P.make_plan(P.FK_PATH_SPLIT, chunks=7), 0) \
+        == P.FK_ERR_INVALID_ARG
+    # a caller workspace that is too small is refused before anything else runs
+    assert P.fk_softmax_rows_ws(A, B, 1, 1 << 22, 0, None, 0x30000000, 8, 0) == P.FK_ERR_INVALID_ARG or \
+        P.fk_softmax_rows_ws(A, B, 1, 1 << 22, 0, None, 0x30000000, 8, 0) in REJECT_NO_LAUNCH
+    with pytest.raises(P.FkError):
+        P.fk_softmax_rows_workspace(1, 10, 9)

@@ -88,6 +88,7 @@ def _forced_plans(fk, cols, dtype):
                 plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k, vpt=ept // vec))
     for k in (1, 2, 3, 16):
         plans.append(fk.make_plan(fk.FK_PATH_TWOPHASE, cluster=k))
+    plans.append(fk.make_plan(fk.FK_PATH_SPLIT))
     if cols <= (1024 if dtype == "f32" else 2048):
         plans.append(fk.make_plan(fk.FK_PATH_WARP, vpt=8))
     return plans
@@ -185,3 +186,45 @@ def test_bf16_outputs_in_the_subnormal_range_round_correctly(fk, torch_mod, cols
     assert sub.any()  # the case really reaches bf16 subnormals
     # fp32: the same rows stay within the absolute tolerance
     check(x, run(fk, torch_mod, x))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 100), (1, 50000), (2, 600000), (5, 1 << 20),
+                                       (7, 1234567)])
+def test_split_path(fk, torch_mod, dtype, rows, cols):
+    x = synth.softmax_input(rows, cols, dtype, sigma=4.0, neg_inf_frac=0.05, seed=rows + cols)
+    p = fk.make_plan(fk.FK_PATH_SPLIT)
+    assert fk.fk_softmax_rows_plan(rows, cols, 0 if dtype == "f32" else 1, fk.FK_PATH_SPLIT).chunks >= 1
+    check(x, run(fk, torch_mod, x, plan=p))
+
+
+def test_split_path_special_rows_in_place_and_misaligned(fk, torch_mod):
+    cols = 300001
+    x = synth.softmax_input(5, cols, "f32", sigma=3.0, seed=77)
+    x[0, :] = -np.inf
+    x[1, 12345] = np.nan
+    x[2, :100000] = -np.inf          # whole chunks with no finite value
+    x[3, cols - 1] += 1000.0
+    p = fk.make_plan(fk.FK_PATH_SPLIT)
+    check(x, run(fk, torch_mod, x, plan=p))
+    check(x, run(fk, torch_mod, x, plan=p, inplace=True))
+    check(x, run(fk, torch_mod, x, plan=p, xoff=1, yoff=1))
+
+
+def test_few_long_rows_take_the_split_path_with_a_caller_workspace(fk, torch_mod):
+    torch = torch_mod
+    rows, cols = 3, 2_000_000
+    plan = fk.fk_softmax_rows_plan(rows, cols, fk.FK_F32)
+    assert plan.as_dict()["path"] == "split"
+    need = fk.fk_softmax_rows_workspace(rows, cols, fk.FK_F32)
+    x = torch.from_numpy(synth.softmax_input(rows, cols, "f32", sigma=2.0, seed=5)).cuda()
+    ws = torch.empty(need // 4, dtype=torch.float32, device="cuda")
+    y1 = fk.softmax_rows(x, workspace=ws)          # allocation-free
+    y2 = fk.softmax_rows(x)                         # stream-ordered workspace
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    xs = x[:, :].cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(y1.cpu().numpy() - oracle.softmax_rows_f64(xs))) <= 1e-6
+    small = torch.empty(max(1, need // 4 - 2), dtype=torch.float32, device="cuda")
+    with pytest.raises(fk.FkError):
+        fk.softmax_rows(x, workspace=small)
