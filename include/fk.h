@@ -189,6 +189,32 @@ FK_API fk_status fk_softmax_rows_ws(const void *x, void *y, size_t rows, size_t 
                                     void *stream);
 
 /*
+ * fk_softmax_rows_noalloc -- fk_softmax_rows that never allocates device
+ * memory (the lecture pages have no counterpart; this is a library
+ * convenience).  For callers that cannot call cudaMalloc or let a library do
+ * so: code under a framework that has reserved nearly all device memory for
+ * its own allocator, latency-critical loops that cannot afford an allocation
+ * call (cudaMalloc may synchronise the device), environments whose policy
+ * forbids a library from allocating.
+ *   Arguments, plan and results as fk_softmax_rows.  Only the split path
+ *   (few or very long rows) needs scratch; here it is a fixed 1 MiB device
+ *   array inside the library (131072 (max, sum) pairs), which every GPU that
+ *   loads the library holds until the process exits.  Rows are processed in
+ *   batches whose partials fit it; a shape whose single row needs more than
+ *   131072 chunks (rows far beyond 2^33 elements) returns FK_ERR_INVALID_ARG.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, once per device, with that device current); make
+ *   that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents (nothing in it needs clearing: each call writes every partial
+ *   it reads before reading it).  Calls whose kernels overlap on the GPU --
+ *   on different streams without ordering between them -- race on it and
+ *   give wrong results; order them (one stream, or events).
+ */
+FK_API fk_status fk_softmax_rows_noalloc(const void *x, void *y, size_t rows, size_t cols, int dtype,
+                                         void *stream);
+
+/*
  * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a
  * cluster exchange their partial (max, sum) through mbarriers; every such
  * wait is bounded in time (1 s) and a wait that gives up is counted instead

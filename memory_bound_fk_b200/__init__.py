@@ -183,6 +183,17 @@ def fk_wait_selftest(timeout_us: int, stream: int = 0) -> int:
     return lib().fk_wait_selftest(timeout_us, stream)
 
 
+def fk_softmax_rows_noalloc(x: int, y: int, rows: int, cols: int, dtype: int, stream: int = 0) -> int:
+    """fk_softmax_rows that never allocates device memory (scratch is a fixed
+    1 MiB array inside the library; see include/fk.h)."""
+    f = lib().fk_softmax_rows_noalloc
+    if f.argtypes is None:
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        f.argtypes = [vp, vp, sz, sz, ctypes.c_int, vp]
+        f.restype = ctypes.c_int
+    return f(x, y, rows, cols, dtype, stream)
+
+
 def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0, chunks: int = 0) -> SoftmaxPlan:
     return SoftmaxPlan(path, threads, vpt, cluster, chunks)
 
@@ -259,7 +270,7 @@ __all__ = [
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
     "fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
-    "fk_softmax_rows_workspace", "fk_softmax_rows_ws",
+    "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
     "fk_wait_selftest", "make_plan", "gelu_tanh",
     "softmax_rows",
