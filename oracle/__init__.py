@@ -11,6 +11,8 @@ reordering); this module only marshals numpy arrays into it.
 Definitions followed:
   * GELU (tanh form): lecture-6 notes of CS336 (kyc001.github.io), section 4.2,
     0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+  * GELU (exact form): x Phi(x), the function the tanh form approximates
+    (the lecture's fusion example, section 6, calls PyTorch's default gelu).
   * Row softmax: "Lecture 6: GPU Kernels and Triton" (cs336.sjfarmltd.com),
     section 7.2 (standard two-pass form), and the lecture-6 notes, section 5.2
     (row max, then exponentials and their sum, then normalise).
@@ -46,7 +48,9 @@ def _load():
         lib.oracle_round_to_bf16.restype = u16
         lib.oracle_bf16_to_f64.argtypes = [u16]
         lib.oracle_bf16_to_f64.restype = d
-        for name in ("oracle_gelu_tanh_f64", "oracle_gelu_tanh_f32"):
+        lib.oracle_gelu_erf.argtypes = [d]
+        lib.oracle_gelu_erf.restype = d
+        for name in ("oracle_gelu_tanh_f64", "oracle_gelu_tanh_f32", "oracle_gelu_erf_f64"):
             getattr(lib, name).argtypes = [p, p, sz, i]
             getattr(lib, name).restype = None
         for name in ("oracle_softmax_rows_f64", "oracle_softmax_rows_f32",
@@ -98,6 +102,19 @@ def gelu_tanh_f64(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
     x = _c(x, np.float64)
     y = np.empty_like(x)
     _load().oracle_gelu_tanh_f64(_ptr(x), _ptr(y), x.size, nthreads or default_threads())
+    return y
+
+
+def gelu_erf(x: float) -> float:
+    """Exact GELU, x * Phi(x), of one double."""
+    return _load().oracle_gelu_erf(float(x))
+
+
+def gelu_erf_f64(x: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """Elementwise exact GELU, double in, double out."""
+    x = _c(x, np.float64)
+    y = np.empty_like(x)
+    _load().oracle_gelu_erf_f64(_ptr(x), _ptr(y), x.size, nthreads or default_threads())
     return y
 
 
@@ -167,7 +184,7 @@ def bf16_to_f64(b: np.ndarray) -> np.ndarray:
 
 
 __all__ = [
-    "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32",
+    "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32", "gelu_erf", "gelu_erf_f64",
     "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16",
     "round_to_f32", "round_to_bf16", "round_to_f32_scalar", "round_to_bf16_scalar",
     "bf16_to_f64", "default_threads",

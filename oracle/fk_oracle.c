@@ -60,6 +60,17 @@ double oracle_gelu_tanh(double x)
     return 0.5 * x * (1.0 + tanh(inner));
 }
 
+/* GELU, exact form: x * Phi(x), Phi the standard normal distribution
+ * function, Phi(x) = erfc(-x / sqrt(2)) / 2 -- the definition the tanh form
+ * approximates (the lecture's PyTorch fusion example calls gelu with its
+ * default, exact form).  erfc keeps Phi accurate in the far negative tail. */
+double oracle_gelu_erf(double x)
+{
+    if (isinf(x))
+        return x > 0.0 ? x : -0.0; /* limits at +-inf */
+    return x * 0.5 * erfc(-x / sqrt(2.0));
+}
+
 /* Softmax of one row, in place of nothing: reads x[0..n), writes y[0..n).
  * Two passes, as the lecture's section 7.2 states the standard algorithm. */
 static void softmax_row_f64(const double *x, double *y, size_t n)
@@ -226,6 +237,22 @@ static void gelu_f32_range(void *p, size_t b, size_t e)
     float *y = (float *)c->y;
     for (size_t i = b; i < e; ++i)
         y[i] = oracle_round_to_f32(oracle_gelu_tanh((double)x[i]));
+}
+
+static void gelu_erf_f64_range(void *p, size_t b, size_t e)
+{
+    gelu_ctx *c = (gelu_ctx *)p;
+    const double *x = (const double *)c->x;
+    double *y = (double *)c->y;
+    for (size_t i = b; i < e; ++i)
+        y[i] = oracle_gelu_erf(x[i]);
+}
+
+/* exact (erf) GELU, double in, double out */
+void oracle_gelu_erf_f64(const double *x, double *y, size_t n, int nthreads)
+{
+    gelu_ctx c = {x, y};
+    parallel_ranges(gelu_erf_f64_range, &c, n, nthreads);
 }
 
 /* double in, double out (no rounding) */

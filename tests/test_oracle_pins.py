@@ -116,6 +116,52 @@ def test_gelu_thread_count_invariance():
     assert np.array_equal(a, b)
 
 
+# =============================================================== exact GELU
+
+def test_gelu_erf_textbook_quantiles():
+    # Phi(1.959963985) = 0.975 and Phi(1.644853627) = 0.95 (standard normal
+    # table), Phi(0) = 1/2, Phi(-x) = 1 - Phi(x)
+    for z, p in ((1.959963984540054, 0.975), (1.6448536269514722, 0.95), (0.0, 0.5)):
+        if z != 0.0:
+            assert abs(oracle.gelu_erf(z) / z - p) <= 1e-15
+            assert abs(oracle.gelu_erf(-z) / -z - (1 - p)) <= 1e-15
+    assert oracle.gelu_erf(0.0) == 0.0
+
+
+def test_gelu_erf_odd_part_identity_and_limits():
+    x = np.concatenate([np.linspace(-30, 30, 60001), RNG.standard_normal(10000) * 5])
+    d = oracle.gelu_erf_f64(x) - oracle.gelu_erf_f64(-x)
+    assert np.all(np.abs(d - x) <= 4e-16 * np.maximum(np.abs(x), 1e-300) + 1e-300)
+    assert oracle.gelu_erf(math.inf) == math.inf
+    r = oracle.gelu_erf(-math.inf)
+    assert r == 0.0 and math.copysign(1.0, r) == -1.0
+    assert math.isnan(oracle.gelu_erf(math.nan))
+    assert np.all(np.abs(oracle.gelu_erf_f64(-np.linspace(40, 100, 61))) < 1e-300)
+
+
+def test_gelu_erf_matches_torch_exact_gelu_float64():
+    x = np.concatenate([np.linspace(-20, 20, 100001), RNG.standard_normal(100000) * 3])
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="none").numpy()
+    assert np.max(np.abs(oracle.gelu_erf_f64(x) - ref)) <= 1e-14
+
+
+def test_gelu_erf_brute_force_mpmath_in_the_tail():
+    # relative accuracy also deep in the negative tail, where 1 + erf loses it
+    mpmath.mp.dps = 50
+    for v in list(np.linspace(-38, 8, 461)):
+        xm = mpmath.mpf(float(v))
+        exact = xm * mpmath.ncdf(xm)
+        got = oracle.gelu_erf(float(v))
+        # error bound of the double evaluation: d ln erfc(z)/dz ~ -(2z + 1/z)
+        # in the tail, so a relative error d in z = -x/sqrt(2) moves the result
+        # by (2 z^2 + 1) d = (x^2 + 1) d; z carries two roundings (sqrt(2), the
+        # division), d <= 2 * 2^-53; erfc itself adds a few ulp; and an
+        # absolute 1e-300 where the double result nears underflow (far below
+        # the smallest fp32/bf16 output, 1.4e-45)
+        tol = (float(v) ** 2 + 5.0) * 2.3e-16 * abs(exact) + 1e-300
+        assert abs(mpmath.mpf(got) - exact) <= tol, v
+
+
 # =================================================================== softmax
 
 @pytest.mark.parametrize("cols", [1, 2, 3, 1000, 4096, 131072])
