@@ -50,14 +50,22 @@
 /* Scalar definitions                                                  */
 /* ------------------------------------------------------------------ */
 
-/* GELU, tanh approximation, lecture-6 notes section 4.2. */
+/* GELU, tanh approximation, lecture-6 notes section 4.2:
+ * 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3).
+ * For x < 0 the sum 1 + tanh(u) cancels -- in double it is 0 once u < -19,
+ * while GELU(-8) is about -3e-21 -- so there it is taken through the exact
+ * identity 1 + tanh(u) = 2 e^(2u) / (1 + e^(2u)), which keeps the result
+ * accurate relative to itself down to double's underflow. */
 double oracle_gelu_tanh(double x)
 {
     if (isinf(x))
         return x > 0.0 ? x : -0.0; /* limits at +-inf */
     const double k = sqrt(2.0 / M_PI);
-    const double inner = k * (x + 0.044715 * x * x * x);
-    return 0.5 * x * (1.0 + tanh(inner));
+    const double u = k * (x + 0.044715 * x * x * x);
+    if (x >= 0.0)
+        return 0.5 * x * (1.0 + tanh(u));
+    const double e = exp(2.0 * u); /* in [0, 1) for x < 0; NaN stays NaN */
+    return 0.5 * x * (2.0 * e / (1.0 + e));
 }
 
 /* GELU, exact form: x * Phi(x), Phi the standard normal distribution

@@ -103,6 +103,30 @@ def test_gelu_brute_force_mpmath():
         assert abs(mpmath.mpf(got) - exact) <= 8e-16 * max(abs(float(x)), 1.0), x
 
 
+def test_gelu_negative_tail_relative_accuracy_mpmath():
+    # For x < 0 GELU is tiny (GELU(-8) ~ -3e-21; GELU(-10.2) ~ -1e-39, a bf16
+    # subnormal), and a bf16 comparison needs it to relative accuracy, not
+    # merely within 1e-16 absolute.  mpmath evaluates the defining formula
+    # with enough digits that 1 + tanh(u) keeps ~40 significant ones.
+    xs = np.concatenate([-np.linspace(0.01, 21.5, 2150), -np.abs(RNG.standard_normal(300)) * 8])
+    for x in xs:
+        xm = mpmath.mpf(float(x))
+        with mpmath.workdps(40):
+            u0 = float(mpmath.sqrt(2 / mpmath.pi) * (xm + mpmath.mpf("0.044715") * xm ** 3))
+        with mpmath.workdps(40 + int(2 * abs(u0) / 2.302585) + 1):
+            c = mpmath.sqrt(2 / mpmath.pi)
+            u = c * (xm + mpmath.mpf("0.044715") * xm ** 3)
+            exact = mpmath.mpf("0.5") * xm * (1 + mpmath.tanh(u))
+            got = oracle.gelu_tanh(float(x))
+            # u carries up to ~6 roundings (sqrt(2/pi), the cube, the sum, the
+            # products), relative 6 * 2^-53 in all, so e^(2u) is off by up to
+            # 2|u| * 6 * 2^-53 = 6|u| * 2^-52 relative, plus a few roundings
+            # after it.  Once e^(2u) is a double subnormal (x < ~-20.5) it holds
+            # only to its spacing 2^-1074, which the product with x scales by |x|.
+            tol = (6 * abs(u0) + 6) * 2.3e-16 * abs(exact) + (abs(float(x)) + 1) * mpmath.mpf(2) ** -1074
+            assert abs(mpmath.mpf(got) - exact) <= tol, (x, got, exact)
+
+
 def test_gelu_f32_wrapper_rounds_the_double_result_once():
     x = (RNG.standard_normal(100000) * 6).astype(np.float32)
     via64 = oracle.round_to_f32(oracle.gelu_tanh_f64(x.astype(np.float64)))
