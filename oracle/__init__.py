@@ -16,6 +16,8 @@ Definitions followed:
   * Row softmax: "Lecture 6: GPU Kernels and Triton" (cs336.sjfarmltd.com),
     section 7.2 (standard two-pass form), and the lecture-6 notes, section 5.2
     (row max, then exponentials and their sum, then normalise).
+  * Scaled, causally masked softmax: the same lecture, section 8 (scores
+    scaled, -inf where the key comes after the query, then softmax).
 
 Parity pins: every function here is pinned by tests in
 ``tests/test_oracle_pins.py`` (closed forms, invariants, library routines
@@ -57,6 +59,8 @@ def _load():
                      "oracle_softmax_rows_bf16"):
             getattr(lib, name).argtypes = [p, p, sz, sz, i]
             getattr(lib, name).restype = None
+        lib.oracle_softmax_rows_causal.argtypes = [p, p, i, sz, sz, d, sz, sz, i]
+        lib.oracle_softmax_rows_causal.restype = None
         for name in ("oracle_round_to_f32_array", "oracle_round_to_bf16_array",
                      "oracle_bf16_to_f64_array"):
             getattr(lib, name).argtypes = [p, p, sz]
@@ -160,6 +164,31 @@ def softmax_rows_bf16(x_bits: np.ndarray, nthreads: int | None = None) -> np.nda
     return y
 
 
+def softmax_rows_causal(x: np.ndarray, scale: float, period: int, offset: int = 0,
+                        nthreads: int | None = None) -> np.ndarray:
+    """Scaled, causally masked row softmax of a [rows, cols] matrix: row r
+    keeps columns j <= (r mod period) + offset (all when period == 0), scores
+    scale * x_j, -inf elsewhere, then softmax.  float64 in -> float64 out;
+    float32 in -> float32 out; uint16 (bf16 patterns) in -> uint16 out, each
+    computed in double and rounded once."""
+    if x.dtype == np.float64:
+        kind = 0
+    elif x.dtype == np.float32:
+        kind = 1
+    elif x.dtype == np.uint16:
+        kind = 2
+    else:
+        raise TypeError("float64, float32 or uint16 (bf16 bits)")
+    x = np.ascontiguousarray(x)
+    rows, cols = _rows_cols(x)
+    if period < 0 or offset < 0:
+        raise ValueError("period and offset are non-negative")
+    y = np.empty_like(x)
+    _load().oracle_softmax_rows_causal(_ptr(x), _ptr(y), kind, rows, cols, float(scale), int(period), int(offset),
+                                       nthreads or default_threads())
+    return y
+
+
 def round_to_f32(v: np.ndarray) -> np.ndarray:
     v = _c(v, np.float64)
     out = np.empty(v.shape, np.float32)
@@ -185,7 +214,7 @@ def bf16_to_f64(b: np.ndarray) -> np.ndarray:
 
 __all__ = [
     "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32", "gelu_erf", "gelu_erf_f64",
-    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16",
+    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16", "softmax_rows_causal",
     "round_to_f32", "round_to_bf16", "round_to_f32_scalar", "round_to_bf16_scalar",
     "bf16_to_f64", "default_threads",
 ]

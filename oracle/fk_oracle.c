@@ -357,6 +357,72 @@ void oracle_softmax_rows_bf16(const uint16_t *x, uint16_t *y, size_t rows, size_
     parallel_ranges(softmax_bf16_range, &c, rows, nthreads);
 }
 
+/* ------------------------------------------------------------------ */
+/* Scaled, causally masked row softmax                                  */
+/* ------------------------------------------------------------------ */
+
+/* The score step of causal attention (lecture 6, "GPU Kernels and Triton",
+ * section 8): scores are scaled (by 1/sqrt(d_k) there), a score whose key
+ * position is after its query position is replaced by -inf, and softmax is
+ * taken over the row.  Here row r of a [rows, cols] matrix has query
+ * position q = (r mod period) + offset and column j is key position j, so
+ *     s_j = scale * x_j  for j <= q,   s_j = -inf  for j > q,
+ * and y = softmax(s) as softmax_row_f64 defines it; period == 0 means no
+ * mask.  Element kinds: 0 = double, 1 = fp32, 2 = bf16 patterns; outputs
+ * are of the input's kind, rounded once from double. */
+typedef struct {
+    const void *x;
+    void *y;
+    int kind;
+    size_t cols;
+    double scale;
+    size_t period, offset;
+} causal_ctx;
+
+static double causal_in(const causal_ctx *c, size_t i)
+{
+    if (c->kind == 0)
+        return ((const double *)c->x)[i];
+    if (c->kind == 1)
+        return (double)((const float *)c->x)[i];
+    return oracle_bf16_to_f64(((const uint16_t *)c->x)[i]);
+}
+
+static void causal_out(const causal_ctx *c, size_t i, double v)
+{
+    if (c->kind == 0)
+        ((double *)c->y)[i] = v;
+    else if (c->kind == 1)
+        ((float *)c->y)[i] = oracle_round_to_f32(v);
+    else
+        ((uint16_t *)c->y)[i] = oracle_round_to_bf16(v);
+}
+
+static void softmax_causal_range(void *p, size_t b, size_t e)
+{
+    causal_ctx *c = (causal_ctx *)p;
+    double *s = (double *)malloc(c->cols * sizeof(double) + 1);
+    double *out = (double *)malloc(c->cols * sizeof(double) + 1);
+    for (size_t r = b; r < e; ++r) {
+        for (size_t j = 0; j < c->cols; ++j) {
+            const int masked = c->period != 0 && j > (r % c->period) + c->offset;
+            s[j] = masked ? -INFINITY : c->scale * causal_in(c, r * c->cols + j);
+        }
+        softmax_row_f64(s, out, c->cols);
+        for (size_t j = 0; j < c->cols; ++j)
+            causal_out(c, r * c->cols + j, out[j]);
+    }
+    free(out);
+    free(s);
+}
+
+void oracle_softmax_rows_causal(const void *x, void *y, int kind, size_t rows, size_t cols, double scale,
+                                size_t period, size_t offset, int nthreads)
+{
+    causal_ctx c = {x, y, kind, cols, scale, period, offset};
+    parallel_ranges(softmax_causal_range, &c, rows, nthreads);
+}
+
 /* array forms of the rounding helpers */
 void oracle_round_to_f32_array(const double *v, float *out, size_t n)
 {

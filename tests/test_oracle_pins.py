@@ -337,6 +337,107 @@ def test_softmax_thread_count_invariance():
     assert np.array_equal(oracle.softmax_rows_f64(x, nthreads=1), oracle.softmax_rows_f64(x, nthreads=5))
 
 
+# ======================================================= causal softmax
+# Scaled, causally masked softmax (lecture 6, "GPU Kernels and Triton",
+# section 8): row r keeps columns j <= (r mod period) + offset, scores
+# scale * x_j, -inf for the rest, then softmax.
+
+
+def _torch_causal(x, scale, period, offset):
+    """Independent construction: a boolean mask from torch.triu over each
+    [period, cols] block (True strictly above the diagonal shifted by offset),
+    masked_fill with -inf, then torch.softmax, all in float64."""
+    t = torch.from_numpy(x) * scale
+    rows, cols = x.shape
+    if period:
+        block = torch.triu(torch.ones(period, cols, dtype=torch.bool), diagonal=offset + 1)
+        mask = block.repeat(-(-rows // period), 1)[:rows]
+        t = t.masked_fill(mask, float("-inf"))
+    return torch.softmax(t, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("rows,cols,scale,period,offset", [
+    (64, 64, 0.125, 64, 0), (96, 48, 1.0, 32, 0), (50, 80, 0.3, 50, 30), (40, 33, 2.5, 7, 3),
+    (17, 17, 1.0, 0, 0), (30, 20, 0.7, 100, 0), (12, 9, 1.3, 4, 50)])
+def test_causal_softmax_matches_torch_masked_fill(rows, cols, scale, period, offset):
+    x = RNG.standard_normal((rows, cols)) * 4
+    y = oracle.softmax_rows_causal(x, scale, period, offset)
+    ref = _torch_causal(x, scale, period, offset)
+    assert np.max(np.abs(y - ref)) <= 1e-14
+    assert np.array_equal(y == 0.0, ref == 0.0)
+
+
+def test_causal_softmax_first_rows_closed_form():
+    # row 0 of a block keeps offset + 1 columns; with offset 0 it is one-hot on
+    # column 0, and row 1 is the two-element softmax 1 / (1 + e^(s(x0 - x1)))
+    x = RNG.standard_normal((8, 6)) * 3
+    s = 0.4
+    y = oracle.softmax_rows_causal(x, s, period=4)
+    assert list(y[0]) == [1.0, 0, 0, 0, 0, 0] and list(y[4]) == [1.0, 0, 0, 0, 0, 0]
+    p0 = 1.0 / (1.0 + math.exp(s * (x[1, 1] - x[1, 0])))
+    assert abs(y[1, 0] - p0) <= 2e-16 and abs(y[1, 1] - (1 - p0)) <= 2e-16
+    assert np.all(y[1, 2:] == 0.0)
+    # with offset 2 the first row keeps 3 columns
+    y2 = oracle.softmax_rows_causal(x, s, period=4, offset=2)
+    assert np.all(y2[0, 3:] == 0.0) and np.all(y2[0, :3] > 0.0)
+
+
+def test_causal_softmax_invariants():
+    x = RNG.standard_normal((120, 70)) * 5
+    y = oracle.softmax_rows_causal(x, 0.25, period=40, offset=10)
+    q = (np.arange(120) % 40) + 10
+    kept = np.arange(70)[None, :] <= q[:, None]
+    assert np.all(y[~kept] == 0.0)            # masked: exactly 0
+    assert np.all(y[kept] > 0.0)
+    assert np.max(np.abs(y.sum(axis=1) - 1.0)) <= 1e-14
+    # the scale multiplies the scores: scaling x instead gives the same result
+    z = oracle.softmax_rows_causal(x * 0.25, 1.0, period=40, offset=10)
+    assert np.max(np.abs(y - z)) <= 1e-15
+    # a constant added to a row changes nothing (up to the rounding of x + c)
+    w = oracle.softmax_rows_causal(x + 3.0, 0.25, period=40, offset=10)
+    assert np.max(np.abs(y - w)) <= 1e-14
+
+
+def test_causal_softmax_never_reads_masked_entries():
+    x = RNG.standard_normal((32, 32))
+    q = np.arange(32)
+    x_bad = x.copy()
+    x_bad[np.arange(32)[None, :] > q[:, None]] = np.nan
+    a = oracle.softmax_rows_causal(x, 0.5, period=32)
+    b = oracle.softmax_rows_causal(x_bad, 0.5, period=32)
+    assert np.array_equal(a, b)
+
+
+def test_causal_softmax_without_mask_and_unit_scale_is_plain_softmax():
+    x = RNG.standard_normal((33, 257)) * 4
+    assert np.array_equal(oracle.softmax_rows_causal(x, 1.0, period=0), oracle.softmax_rows_f64(x))
+
+
+def test_causal_softmax_brute_force_mpmath():
+    mpmath.mp.dps = 50
+    x = RNG.standard_normal((7, 9)) * 3
+    scale, period, offset = 0.37, 5, 2
+    y = oracle.softmax_rows_causal(x, scale, period, offset)
+    for r in range(7):
+        q = r % period + offset
+        s = [mpmath.mpf(scale) * mpmath.mpf(float(v)) for v in x[r, :q + 1]]
+        m = max(s)
+        e = [mpmath.exp(v - m) for v in s]
+        tot = mpmath.fsum(e)
+        for j in range(9):
+            exact = e[j] / tot if j <= q else mpmath.mpf(0)
+            assert abs(mpmath.mpf(float(y[r, j])) - exact) <= 4e-16
+
+
+def test_causal_softmax_f32_and_bf16_round_the_double_result_once():
+    x = (RNG.standard_normal((40, 50)) * 4).astype(np.float32)
+    via64 = oracle.round_to_f32(oracle.softmax_rows_causal(x.astype(np.float64), 0.6, 16, 3))
+    assert np.array_equal(oracle.softmax_rows_causal(x, 0.6, 16, 3).view(np.uint32), via64.view(np.uint32))
+    b = oracle.round_to_bf16(x.astype(np.float64))
+    via64b = oracle.round_to_bf16(oracle.softmax_rows_causal(oracle.bf16_to_f64(b), 0.6, 16, 3))
+    assert np.array_equal(oracle.softmax_rows_causal(b, 0.6, 16, 3), via64b)
+
+
 # ================================================================= rounding
 
 def _all_finite_bf16():
