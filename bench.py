@@ -58,19 +58,42 @@ def log(*a):
 
 def kernel_name(w, plan: dict) -> str:
     """The libfk kernel a workload's plan launches."""
-    if w.op == "gelu":
-        return "gelu_tanh_kernel"
     t = "bf16" if w.dtype == "bf16" else "float"
+    if w.op in ("gelu", "gelu_erf"):
+        return f"gelu_kernel<{t},{'tanh' if w.op == 'gelu' else 'erf'}>"
+    sc = ",scaled" if w.op == "softmax_causal" else ""
     vec = 8 if w.dtype == "bf16" else 4
     p = plan["path"]
     if p == "warp":
-        return f"softmax_warp_kernel<{t},vpt={plan['vpt']}>"
+        return f"softmax_warp_kernel<{t},vpt={plan['vpt']}{sc}>"
     if p == "cta":
-        return f"softmax_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}>"
+        return f"softmax_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{sc}>"
     if p == "cluster":
-        return (f"softmax_cluster_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}>"
+        return (f"softmax_cluster_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{sc}>"
                 f" x cluster {plan['cluster']}")
-    return f"softmax_twophase_kernel<{t},cluster={plan['cluster']}>"
+    if p == "split":
+        return f"softmax_split_stats_kernel + softmax_split_norm_kernel<{t}{sc}>"
+    return f"softmax_twophase_kernel<{t},cluster={plan['cluster']}{sc}>"
+
+
+def launch_workload(fk, w, xp: int, yp: int, shape, stream: int) -> int:
+    """One call of a workload's operator through the C ABI; the status.
+    The causal softmax treats every `cols` rows as one block of queries
+    against `cols` keys (scale 1: the result equals plain softmax over the
+    same scores with the masked entries at -inf)."""
+    code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+    if w.op in ("gelu", "gelu_erf"):
+        kind = fk.FK_GELU_TANH if w.op == "gelu" else fk.FK_GELU_ERF
+        return fk.fk_gelu(xp, yp, shape[0], code, kind, stream)
+    rows, cols = shape
+    if w.op == "softmax_causal":
+        return fk.fk_softmax_rows_causal(xp, yp, rows, cols, code, 1.0, cols, 0, stream)
+    return fk.fk_softmax_rows(xp, yp, rows, cols, code, stream)
+
+
+def workload_bytes(w, shape) -> int:
+    from memory_bound_fk_b200 import synth
+    return synth.algorithmic_bytes(w.op, w.itemsize, tuple(shape))
 
 
 def hbm_traffic_bytes(tensor_bytes: int, n_elementwise_ops: int, fused: bool) -> int:
@@ -220,13 +243,19 @@ def oracle_run(names, inputs, frac, threads):
     for n in names:
         w = synth.WORKLOADS[n]
         x = _slice(n, inputs[n], frac)
-        if w.op == "gelu":
-            oracle.gelu_tanh_f32(x, nthreads=threads)
+        if w.op in ("gelu", "gelu_erf"):
+            f64 = oracle.gelu_tanh_f64 if w.op == "gelu" else oracle.gelu_erf_f64
+            if w.dtype == "f32":
+                oracle.round_to_f32(f64(x.astype(np.float64), nthreads=threads))
+            else:
+                oracle.round_to_bf16(f64(oracle.bf16_to_f64(x), nthreads=threads))
+        elif w.op == "softmax_causal":
+            oracle.softmax_rows_causal(x, 1.0, x.shape[1], 0, nthreads=threads)
         elif w.dtype == "f32":
             oracle.softmax_rows_f32(x, nthreads=threads)
         else:
             oracle.softmax_rows_bf16(x, nthreads=threads)
-        total_bytes += 2 * x.size * w.itemsize
+        total_bytes += workload_bytes(w, x.shape)
         elems += x.size
     dt = time.perf_counter() - t0
     return {"seconds": dt, "bytes": total_bytes, "elements": elems}
@@ -285,14 +314,8 @@ def run_ours(args) -> dict | None:
         dev_in[n] = t.to(device)
         dev_out[n] = torch.empty_like(dev_in[n])
         xp, yp = dev_in[n].data_ptr(), dev_out[n].data_ptr()
-        if w.op == "gelu":
-            calls.append((n, lambda xp=xp, yp=yp, k=host[n].size: fk.fk_gelu_tanh(xp, yp, k, sh)))
-        else:
-            r, c = shapes[n]
-            code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
-            calls.append((n, lambda xp=xp, yp=yp, r=r, c=c, code=code:
-                          fk.fk_softmax_rows(xp, yp, r, c, code, sh)))
-    bytes_step = sum(2 * host[n].nbytes for n in names)
+        calls.append((n, lambda w=w, xp=xp, yp=yp, shape=shapes[n]: launch_workload(fk, w, xp, yp, shape, sh)))
+    bytes_step = sum(workload_bytes(synth.WORKLOADS[n], shapes[n]) for n in names)
     elems_step = sum(host[n].size for n in names)
 
     def step(evs=None):
@@ -357,11 +380,11 @@ def run_ours(args) -> dict | None:
     for i, n in enumerate(names):
         w = synth.WORKLOADS[n]
         ms = kernel_ms[i] / args.steps
-        nbytes = 2 * host[n].nbytes
+        nbytes = workload_bytes(w, shapes[n])
         gbs = nbytes / (ms * 1e-3) / 1e9
         plan = (fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1],
                                         fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32).as_dict()
-                if w.op == "softmax" else {"path": "gelu"})
+                if w.op.startswith("softmax") else {"path": "gelu"})
         kernels.append({"workload": n, "kernel": kernel_name(w, plan), "plan": plan,
                         "shape": list(shapes[n]), "ms": round(ms, 5), "GB_s": round(gbs, 1),
                         "elements_per_s": round(host[n].size / (ms * 1e-3), 1),
@@ -429,7 +452,9 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
         row_bytes = a.itemsize * (a.shape[1] if a.ndim == 2 else 1)
         per = max(1, chunk_bytes // row_bytes)
         if a.ndim == 1:
-            per = max(4, per // 4 * 4)  # keep 16-byte chunk boundaries
+            per = max(8, per // 8 * 8)  # keep 16-byte chunk boundaries
+        elif synth.WORKLOADS[n].op == "softmax_causal":
+            per = max(1, per // a.shape[1]) * a.shape[1]  # whole query blocks per chunk
         for r0 in range(0, a.shape[0], per):
             chunks.append((n, r0, min(per, a.shape[0] - r0)))
     streams = [stream, torch.cuda.Stream(device)]
@@ -444,11 +469,7 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
                 raw_in[n][r0:r0 + cnt].copy_(pin_in[n][r0:r0 + cnt], non_blocking=True)
                 xp = raw_in[n][r0:r0 + cnt].data_ptr()
                 yp = raw_out[n][r0:r0 + cnt].data_ptr()
-                if w.op == "gelu":
-                    st = fk.fk_gelu_tanh(xp, yp, cnt, s.cuda_stream)
-                else:
-                    st = fk.fk_softmax_rows(xp, yp, cnt, host[n].shape[1],
-                                            fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32, s.cuda_stream)
+                st = launch_workload(fk, w, xp, yp, (cnt,) + tuple(host[n].shape[1:]), s.cuda_stream)
                 if st != fk.FK_OK:
                     raise fk.FkError(st, n)
                 pin_out[n][r0:r0 + cnt].copy_(raw_out[n][r0:r0 + cnt], non_blocking=True)
@@ -531,6 +552,8 @@ def run_unfused(args) -> dict | None:
     out = []
     for n in names:
         w = synth.WORKLOADS[n]
+        if w.op not in ("gelu", "softmax"):
+            raise SystemExit(f"--impl unfused covers tanh-GELU and plain softmax workloads, not {n}")
         a = host[n]
         x = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
              else torch.from_numpy(a)).to(device)
@@ -626,7 +649,8 @@ def parse_args(argv=None):
                         "eager op-by-op sequences timed against libfk (one GPU)")
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
-                        "cfg3_softmax, cfg4_softmax, cfg5_softmax")
+                        "cfg3_softmax, cfg4_softmax, cfg5_softmax, and the operator variants "
+                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal")
     p.add_argument("--rows", type=int, default=None,
                    help="profiling only: leading rows (elements for GELU) of each workload")
     p.add_argument("--no-e2e", action="store_true")

@@ -91,6 +91,27 @@ typedef enum fk_dtype {
  */
 FK_API fk_status fk_gelu_tanh(const float *x, float *y, size_t n, void *stream);
 
+/* GELU forms of fk_gelu. */
+typedef enum fk_gelu_kind {
+    FK_GELU_TANH = 0, /* 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) (lecture-6 notes, section 4.2) */
+    FK_GELU_ERF = 1   /* x Phi(x), the exact form the tanh one approximates */
+} fk_gelu_kind;
+
+/*
+ * fk_gelu -- elementwise GELU of either form, fp32 or bf16 in and out.
+ *   x  [in]  n values of `dtype`, device-accessible, aligned to the element size.
+ *   y  [out] n values of the same dtype; y == x allowed.
+ *   n        element count (0 = no-op).
+ *   dtype    FK_F32 or FK_BF16 (bf16: computed in fp32, rounded to nearest even).
+ *   kind     an fk_gelu_kind.
+ *   stream   cudaStream_t as void*.
+ * Accuracy: fp32 within 2e-6 absolute of the exact value; bf16 within 1 ulp
+ * of the correctly rounded value (subnormal outputs included).  GELU(+inf) =
+ * +inf, GELU(-inf) = -0, GELU(NaN) = NaN.  fk_gelu_tanh(x, y, n, s) is
+ * fk_gelu(x, y, n, FK_F32, FK_GELU_TANH, s).
+ */
+FK_API fk_status fk_gelu(const void *x, void *y, size_t n, int dtype, int kind, void *stream);
+
 /*
  * fk_softmax_rows -- softmax over each row of a row-major [rows, cols]
  * matrix (lecture 6, section 7.2; lecture-6 notes, section 5.2).
@@ -213,6 +234,41 @@ FK_API fk_status fk_softmax_rows_ws(const void *x, void *y, size_t rows, size_t 
  */
 FK_API fk_status fk_softmax_rows_noalloc(const void *x, void *y, size_t rows, size_t cols, int dtype,
                                          void *stream);
+
+/*
+ * fk_softmax_rows_causal -- scaled, causally masked row softmax: the score
+ * step of causal attention (lecture 6, "GPU Kernels and Triton", section 8:
+ * scores times 1/sqrt(d_k), -inf where the key position is after the query
+ * position, then softmax) in one pass, with the mask generated in the kernel
+ * instead of read from an -inf tensor.  Row r keeps the columns
+ *     j <= q(r) = (r mod period) + offset
+ * (every column when period == 0) and gets
+ *     y[r, j] = exp(scale (x[r, j] - m)) / sum_{i <= q(r)} exp(scale (x[r, i] - m)),
+ *     m = max_{i <= q(r)} x[r, i],
+ * and y[r, j] = 0 for j > q(r).  Masked inputs are never read (they may hold
+ * anything), so a causal [T, T] score block moves about 25% fewer bytes than
+ * softmax over an explicitly masked tensor.
+ *   x, y, rows, cols, dtype, stream   as for fk_softmax_rows.
+ *   scale   finite and > 0 (e.g. 1/sqrt(d_k)); applied in fp32 as
+ *           scale * log2(e) rounded once.
+ *   period  the rows per query block: for scores laid out [batch, heads, T_q,
+ *           T_k] as rows of T_k columns, period = T_q; 0 = no mask (a scaled
+ *           softmax).
+ *   offset  the query position of each block's first row: 0 when queries and
+ *           keys start together, T_k - T_q for the last T_q positions of a
+ *           T_k-long sequence.
+ * Paths, special values and errors as fk_softmax_rows (a kept -inf gives 0;
+ * every row keeps at least column 0, so no row is empty).  Values with
+ * |scale * x| beyond about 2^126 overflow the fp32 exponent arithmetic (NaN
+ * in that row).  scale not finite or <= 0 -> FK_ERR_INVALID_ARG.
+ */
+FK_API fk_status fk_softmax_rows_causal(const void *x, void *y, size_t rows, size_t cols, int dtype, float scale,
+                                        size_t period, size_t offset, void *stream);
+
+/* fk_softmax_rows_causal with an explicit plan, as fk_softmax_rows_ex. */
+FK_API fk_status fk_softmax_rows_causal_ex(const void *x, void *y, size_t rows, size_t cols, int dtype,
+                                           float scale, size_t period, size_t offset,
+                                           const fk_softmax_plan *plan, void *stream);
 
 /*
  * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a

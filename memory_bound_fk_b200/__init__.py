@@ -7,18 +7,23 @@ library's CUDA kernels.  PyTorch provides device memory and streams.
 Raw C-ABI mirrors (same names, pointers as integers, stream as a
 ``cudaStream_t`` integer):
     fk_gelu_tanh(x, y, n, stream) -> status
+    fk_gelu(x, y, n, dtype, kind, stream) -> status
     fk_softmax_rows(x, y, rows, cols, dtype, stream) -> status
     fk_softmax_rows_ex(x, y, rows, cols, dtype, plan, stream) -> status
     fk_softmax_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
     fk_softmax_rows_workspace(rows, cols, dtype, plan=None) -> bytes
     fk_softmax_rows_ws(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, stream) -> status
+    fk_softmax_rows_causal(x, y, rows, cols, dtype, scale, period, offset, stream) -> status
+    fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, plan, stream) -> status
     fk_status_string(status) -> str
     fk_wait_timeouts(reset=False) -> int     (bounded-wait give-ups, synchronous)
     fk_wait_selftest(timeout_us, stream) -> status
 
 Tensor conveniences (contiguous CUDA tensors; the current torch stream):
     gelu_tanh(x, out=None)
+    gelu(x, out=None, approximate="tanh")   # fp32 / bf16; "tanh" or "none" (exact)
     softmax_rows(x, out=None, plan=None)    # softmax over the last dimension
+    softmax_causal(x, scale, period=None, offset=0, out=None, plan=None)
 
 There is no fallback: if the library is missing or a call fails, an
 exception is raised.
@@ -42,6 +47,9 @@ FK_ERR_CUDA = 4
 # fk_dtype
 FK_F32 = 0
 FK_BF16 = 1
+# fk_gelu_kind
+FK_GELU_TANH = 0
+FK_GELU_ERF = 1
 # fk_softmax_path
 FK_PATH_AUTO = 0
 FK_PATH_WARP = 1
@@ -86,6 +94,8 @@ def lib() -> ctypes.CDLL:
         vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
         L.fk_gelu_tanh.argtypes = [vp, vp, sz, vp]
         L.fk_gelu_tanh.restype = ci
+        L.fk_gelu.argtypes = [vp, vp, sz, ci, ci, vp]
+        L.fk_gelu.restype = ci
         L.fk_softmax_rows.argtypes = [vp, vp, sz, sz, ci, vp]
         L.fk_softmax_rows.restype = ci
         L.fk_softmax_rows_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.POINTER(SoftmaxPlan), vp]
@@ -103,6 +113,11 @@ def lib() -> ctypes.CDLL:
         L.fk_softmax_rows_workspace.restype = ci
         L.fk_softmax_rows_ws.argtypes = [vp, vp, sz, sz, ci, ctypes.POINTER(SoftmaxPlan), vp, sz, vp]
         L.fk_softmax_rows_ws.restype = ci
+        L.fk_softmax_rows_causal.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz, vp]
+        L.fk_softmax_rows_causal.restype = ci
+        L.fk_softmax_rows_causal_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz,
+                                                ctypes.POINTER(SoftmaxPlan), vp]
+        L.fk_softmax_rows_causal_ex.restype = ci
         L.fk_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
         L.fk_wait_timeouts.restype = ci
         L.fk_wait_selftest.argtypes = [ctypes.c_uint, vp]
@@ -121,6 +136,10 @@ def header_functions() -> list[str]:
 
 def fk_gelu_tanh(x: int, y: int, n: int, stream: int = 0) -> int:
     return lib().fk_gelu_tanh(x, y, n, stream)
+
+
+def fk_gelu(x: int, y: int, n: int, dtype: int, kind: int, stream: int = 0) -> int:
+    return lib().fk_gelu(x, y, n, dtype, kind, stream)
 
 
 def fk_softmax_rows(x: int, y: int, rows: int, cols: int, dtype: int, stream: int = 0) -> int:
@@ -155,6 +174,17 @@ def fk_softmax_rows_ws(x: int, y: int, rows: int, cols: int, dtype: int, plan: S
                        workspace: int, workspace_bytes: int, stream: int = 0) -> int:
     return lib().fk_softmax_rows_ws(x, y, rows, cols, dtype, ctypes.byref(plan) if plan is not None else None,
                                     workspace, workspace_bytes, stream)
+
+
+def fk_softmax_rows_causal(x: int, y: int, rows: int, cols: int, dtype: int, scale: float, period: int,
+                           offset: int = 0, stream: int = 0) -> int:
+    return lib().fk_softmax_rows_causal(x, y, rows, cols, dtype, scale, period, offset, stream)
+
+
+def fk_softmax_rows_causal_ex(x: int, y: int, rows: int, cols: int, dtype: int, scale: float, period: int,
+                              offset: int, plan: SoftmaxPlan | None, stream: int = 0) -> int:
+    return lib().fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset,
+                                           ctypes.byref(plan) if plan is not None else None, stream)
 
 
 def fk_status_string(status: int) -> str:
@@ -236,7 +266,30 @@ def _dtype_code(dt) -> int:
         return FK_F32
     if dt == torch.bfloat16:
         return FK_BF16
-    raise TypeError("softmax_rows takes float32 or bfloat16")
+    raise TypeError("fk operators take float32 or bfloat16")
+
+
+_GELU_KINDS = {"tanh": FK_GELU_TANH, "none": FK_GELU_ERF}
+
+
+def gelu(x, out=None, approximate: str = "tanh"):
+    """GELU of a contiguous fp32/bf16 CUDA tensor; ``approximate`` is "tanh"
+    (the tanh form) or "none" (the exact x * Phi(x)), as in torch's gelu.
+    ``out`` may be ``x``."""
+    import torch
+    _check_tensor(x, "x")
+    code = _dtype_code(x.dtype)
+    if approximate not in _GELU_KINDS:
+        raise ValueError("approximate must be 'tanh' or 'none'")
+    if out is None:
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.dtype != x.dtype or out.numel() != x.numel() or out.device != x.device:
+        raise ValueError("out must match x in dtype, size and device")
+    st = fk_gelu(x.data_ptr(), out.data_ptr(), x.numel(), code, _GELU_KINDS[approximate], _stream_handle(x))
+    if st != FK_OK:
+        raise FkError(st, "fk_gelu")
+    return out
 
 
 def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None, workspace=None):
@@ -265,13 +318,40 @@ def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None, workspace=None):
     return out
 
 
+def softmax_causal(x, scale: float, period: int | None = None, offset: int = 0, out=None,
+                   plan: SoftmaxPlan | None = None):
+    """Scaled, causally masked softmax over the last dimension of a
+    contiguous fp32/bf16 CUDA tensor of attention scores [..., T_q, T_k]: row
+    i of each [T_q, T_k] block keeps keys j <= i + offset.  `period` defaults
+    to T_q (x.shape[-2]); 0 means no mask."""
+    import torch
+    _check_tensor(x, "x")
+    code = _dtype_code(x.dtype)
+    if x.dim() < 2 and period is None:
+        raise ValueError("period is needed for a 1-D tensor")
+    if out is None:
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.dtype != x.dtype or out.shape != x.shape or out.device != x.device:
+        raise ValueError("out must match x in dtype, shape and device")
+    cols = x.shape[-1] if x.dim() > 0 else 1
+    rows = x.numel() // cols if cols else 0
+    p = x.shape[-2] if period is None else period
+    st = fk_softmax_rows_causal_ex(x.data_ptr(), out.data_ptr(), rows, cols, code, scale, p, offset, plan,
+                                   _stream_handle(x))
+    if st != FK_OK:
+        raise FkError(st, "fk_softmax_rows_causal")
+    return out
+
+
 __all__ = [
     "FK_OK", "FK_ERR_INVALID_ARG", "FK_ERR_UNSUPPORTED_DTYPE", "FK_ERR_UNSUPPORTED_DEVICE",
-    "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
+    "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_GELU_TANH", "FK_GELU_ERF", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
-    "fk_gelu_tanh", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
+    "fk_gelu_tanh", "fk_gelu", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
     "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
+    "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
-    "fk_wait_selftest", "make_plan", "gelu_tanh",
+    "fk_wait_selftest", "make_plan", "gelu_tanh", "gelu",
     "softmax_rows",
 ]

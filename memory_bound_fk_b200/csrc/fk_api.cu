@@ -9,6 +9,7 @@
 // instead of a device fault.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cfloat>
 
 #include <stdint.h>
 
@@ -173,14 +174,19 @@ const DeviceInfo* current_device_info(int* device_out) {
 
 extern "C" {
 
-fk_status fk_gelu_tanh(const float* x, float* y, size_t n, void* stream) {
+fk_status fk_gelu(const void* x, void* y, size_t n, int dtype, int kind, void* stream) {
+  if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
+  if (kind != FK_GELU_TANH && kind != FK_GELU_ERF) return FK_ERR_INVALID_ARG;
   if (n == 0) return FK_OK;
   const fk::DeviceInfo* dev = nullptr;
-  const fk_status st = fk::check_call(x, y, n, sizeof(float), &dev);
+  const fk_status st = fk::check_call(x, y, n, dtype == FK_F32 ? 4 : 2, &dev);
   if (st != FK_OK) return st;
-  const cudaError_t e =
-      fk::launch_gelu_tanh(x, y, n, *dev, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = fk::launch_gelu(x, y, n, dtype, kind, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_gelu_tanh(const float* x, float* y, size_t n, void* stream) {
+  return fk_gelu(x, y, n, FK_F32, FK_GELU_TANH, stream);
 }
 
 fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out) {
@@ -197,8 +203,9 @@ fk_status resolve_plan(size_t rows, size_t cols, int dtype, const fk_softmax_pla
 
 // Shared body of the softmax entry points.  ws == nullptr and
 // allow_alloc: a needed workspace is allocated stream-ordered.
+// sc == nullptr: plain softmax.
 fk_status softmax_call(const void* x, void* y, size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan,
-                       void* ws, size_t ws_bytes, bool allow_alloc, void* stream) {
+                       void* ws, size_t ws_bytes, bool allow_alloc, const fk::SoftmaxScaling* sc, void* stream) {
   if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
   if (rows == 0 || cols == 0) return FK_OK;
   if (rows > SIZE_MAX / cols) return FK_ERR_INVALID_ARG;
@@ -237,7 +244,7 @@ fk_status softmax_call(const void* x, void* y, size_t rows, size_t cols, int dty
   // pitch that is a multiple of 16 bytes.
   const bool aligned = (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
                        (reinterpret_cast<uintptr_t>(y) % 16 == 0) && ((cols * esize) % 16 == 0);
-  cudaError_t e = fk::launch_softmax(x, y, rows, cols, dtype, p, aligned, ws, *dev, s);
+  cudaError_t e = fk::launch_softmax(x, y, rows, cols, dtype, p, aligned, ws, sc, *dev, s);
   if (owned) {
     const cudaError_t f = cudaFreeAsync(ws, s);
     if (e == cudaSuccess) e = f;
@@ -249,12 +256,31 @@ fk_status softmax_call(const void* x, void* y, size_t rows, size_t cols, int dty
 
 fk_status fk_softmax_rows_ex(const void* x, void* y, size_t rows, size_t cols, int dtype,
                              const fk_softmax_plan* plan, void* stream) {
-  return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, stream);
+  return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, nullptr, stream);
 }
 
 fk_status fk_softmax_rows_ws(const void* x, void* y, size_t rows, size_t cols, int dtype,
                              const fk_softmax_plan* plan, void* workspace, size_t workspace_bytes, void* stream) {
-  return softmax_call(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, false, stream);
+  return softmax_call(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, false, nullptr, stream);
+}
+
+fk_status fk_softmax_rows_causal_ex(const void* x, void* y, size_t rows, size_t cols, int dtype, float scale,
+                                    size_t period, size_t offset, const fk_softmax_plan* plan, void* stream) {
+  if (!(scale > 0.0f) || !(scale <= FLT_MAX)) return FK_ERR_INVALID_ARG;  // also rejects NaN
+  fk::SoftmaxScaling sc;
+  sc.k = static_cast<float>(static_cast<double>(scale) * 1.44269504088896340736);
+  // (r mod period) + offset: a period beyond the rows and an offset beyond
+  // the columns change nothing, and bounding them keeps the sum from wrapping
+  sc.period = period < rows ? period : rows;
+  sc.offset = offset < cols ? offset : cols;
+  sc.row0 = 0;
+  fk::set_period_division(&sc, rows);
+  return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, &sc, stream);
+}
+
+fk_status fk_softmax_rows_causal(const void* x, void* y, size_t rows, size_t cols, int dtype, float scale,
+                                 size_t period, size_t offset, void* stream) {
+  return fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, nullptr, stream);
 }
 
 fk_status fk_softmax_rows_workspace(size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan,

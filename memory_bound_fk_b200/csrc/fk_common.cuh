@@ -125,6 +125,14 @@ struct Elem<float> {
   }
   __device__ __forceinline__ static float load1(const float* p) { return __ldg(p); }
   __device__ __forceinline__ static void store1(float* p, float v) { *p = v; }
+  // Keep the first `keep` values of a vector, -inf in the rest.
+  __device__ __forceinline__ static uint4 keep_first(uint4 w, int keep) {
+    w.x = keep > 0 ? w.x : kNegInfWord;
+    w.y = keep > 1 ? w.y : kNegInfWord;
+    w.z = keep > 2 ? w.z : kNegInfWord;
+    w.w = keep > 3 ? w.w : kNegInfWord;
+    return w;
+  }
   // exp2 for softmax terms: results below 2^-126 flush to zero, an absolute
   // error under 1.2e-38 on an fp32 output (3% faster on 4096-column rows).
   __device__ __forceinline__ static float exp2(float a) { return ex2_ftz(a); }
@@ -178,6 +186,15 @@ struct Elem<__nv_bfloat16> {
   }
   __device__ __forceinline__ static void store1(__nv_bfloat16* p, float v) {
     *p = __float2bfloat16_rn(v);
+  }
+  // Keep the first `keep` values of a vector, -inf in the rest (word i holds
+  // values 2i in its low half and 2i+1 in its high half).
+  __device__ __forceinline__ static uint32_t keep_word(uint32_t w, int keep, int i) {
+    return keep > 2 * i + 1 ? w : (keep > 2 * i ? ((w & 0xffffu) | 0xff800000u) : kNegInfWord);
+  }
+  __device__ __forceinline__ static uint4 keep_first(uint4 w, int keep) {
+    return make_uint4(keep_word(w.x, keep, 0), keep_word(w.y, keep, 1), keep_word(w.z, keep, 2),
+                      keep_word(w.w, keep, 3));
   }
   // exp2 for softmax terms: subnormal results kept, because bf16 outputs
   // down to 2^-133 must still round correctly.

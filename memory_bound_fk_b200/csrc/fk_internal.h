@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <stdint.h>
 
 #include "fk.h"
 
@@ -22,9 +23,9 @@ struct DeviceInfo {
 const DeviceInfo* current_device_info(int* device_out);
 
 // ---- GELU --------------------------------------------------------------
-// y[i] = GELU_tanh(x[i]) for i < n.  Arguments already validated.
-cudaError_t launch_gelu_tanh(const float* x, float* y, size_t n, const DeviceInfo& dev,
-                             cudaStream_t stream);
+// y[i] = GELU(x[i]) for i < n, dtype FK_F32 / FK_BF16, kind FK_GELU_TANH /
+// FK_GELU_ERF.  Arguments already validated.
+cudaError_t launch_gelu(const void* x, void* y, size_t n, int dtype, int kind, cudaStream_t stream);
 
 // ---- softmax -----------------------------------------------------------
 constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
@@ -55,13 +56,35 @@ fk_status plan_softmax(size_t rows, size_t cols, int dtype, int path, fk_softmax
 // Validate a caller-provided plan and fill defaults.
 fk_status check_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan& in, fk_softmax_plan* out);
 
+// Scale and causal mask of fk_softmax_rows_causal.  Row r (counted from the
+// start of the whole call) keeps columns j < limit(r), limit(r) =
+// min(cols, (r mod period) + offset + 1), or every column when period == 0,
+// and computes softmax(scale * x_j) over them; the other columns are not
+// read and are written 0.
+struct SoftmaxScaling {
+  float k;        // scale * log2(e), rounded once to fp32
+  size_t period;  // 0: no mask; otherwise 1 <= period <= rows
+  size_t offset;  // <= cols
+  size_t row0;    // index of the launch's first row within the call (set by the launchers)
+  // r mod period by multiplication (Granlund and Montgomery, "Division by
+  // invariant integers using multiplication", 1994, unsigned 32-bit case):
+  // q = (t + ((n - t) >> shift1)) >> shift2 with t = mulhi(magic, n).  Used
+  // when fast32 is set (period and every row index below 2^32).
+  uint32_t magic, shift1, shift2;
+  int fast32;
+};
+
+// Fill the division fields of `sc` for its period and the call's rows.
+void set_period_division(SoftmaxScaling* sc, size_t rows);
+
 // Launch a validated plan.  `aligned` = rows and both pointers allow 16-byte
 // vector access.
 // `ws` is device workspace of at least workspace_bytes(plan) bytes (only the
-// split path uses it; may be null otherwise).
+// split path uses it; may be null otherwise).  `sc` == nullptr: plain
+// softmax; otherwise scaled and masked as above.
 cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                           const fk_softmax_plan& plan, bool aligned, void* ws, const DeviceInfo& dev,
-                           cudaStream_t stream);
+                           const fk_softmax_plan& plan, bool aligned, void* ws, const SoftmaxScaling* sc,
+                           const DeviceInfo& dev, cudaStream_t stream);
 
 // Workspace bytes a validated plan needs (0 except on the split path).
 size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan);

@@ -220,4 +220,20 @@ fk_status check_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan&
   return FK_OK;
 }
 
+void set_period_division(SoftmaxScaling* sc, size_t rows) {
+  sc->magic = 0;
+  sc->shift1 = 0;
+  sc->shift2 = 0;
+  sc->fast32 = 0;
+  const uint64_t d = sc->period;
+  if (d == 0 || d > 0xffffffffull || rows > 0xffffffffull) return;
+  // l = ceil(log2 d); magic = floor(2^32 (2^l - d) / d) + 1, which is < 2^32
+  unsigned l = 0;
+  while ((uint64_t{1} << l) < d) ++l;
+  sc->magic = static_cast<uint32_t>((((uint64_t{1} << l) - d) << 32) / d + 1);
+  sc->shift1 = l < 1 ? l : 1;
+  sc->shift2 = l > 1 ? l - 1 : 0;
+  sc->fast32 = 1;
+}
+
 }  // namespace fk

@@ -42,6 +42,14 @@
 // is skipped by fmaxf but poisons the sum; a +inf gives inf - inf = NaN.
 // Partial results of slices that are all -inf are merged without forming
 // (-inf) - (-inf): see rescale().
+//
+// Scaled and causal form (every kernel, template flag SC): the exponent of
+// x_j is scale * (x_j - m) and row r keeps only its first limit(r) columns
+// (see row_limit); masked columns are never loaded -- their loads are
+// predicated off, so they cost no HBM traffic -- and are written 0.  This is
+// the score step of causal attention (lecture 6, "GPU Kernels and Triton",
+// section 8: the scores times 1/sqrt(d_k), -inf where the key comes after
+// the query, then the softmax) done in one pass, without an -inf tensor.
 #include <cuda_bf16.h>
 
 #include "fk_common.cuh"
@@ -83,35 +91,63 @@ __device__ __forceinline__ I imin(I a, I b) {
 
 // ---------------------------------------------------------------- merge rule
 
-// exp(m_from - m_to) for m_from <= m_to: the factor that moves a partial sum
-// taken relative to max m_from onto max m_to.  Equal maxima give exactly 1,
-// which also covers (-inf, -inf) (an all -inf partial, whose sum is 0) and
-// (+inf, +inf) (whose sum is already NaN).
-__device__ __forceinline__ float rescale(float m_from, float m_to) {
-  return (m_from == m_to) ? 1.0f : ex2((m_from - m_to) * kLog2e);
+// exp(scale * (m_from - m_to)) for m_from <= m_to (k = scale * log2 e): the
+// factor that moves a partial sum taken relative to max m_from onto max m_to.
+// Equal maxima give exactly 1, which also covers (-inf, -inf) (an all -inf
+// partial, whose sum is 0) and (+inf, +inf) (whose sum is already NaN).
+__device__ __forceinline__ float rescale(float m_from, float m_to, float k) {
+  return (m_from == m_to) ? 1.0f : ex2((m_from - m_to) * k);
 }
 
 // Reference point for exponentials of a partial whose max is m: m itself,
 // or 0 for an all -inf partial (so that exp(-inf - ref) = 0, not NaN).
 __device__ __forceinline__ float exp_ref(float m) { return (m == -INFINITY) ? 0.0f : m; }
 
+// Columns kept in row `row` of the launch (see SoftmaxScaling): the query
+// position of the row is (row0 + row) mod period + offset, and keys up to it
+// are kept.  The host bounds period by the rows and offset by cols, so the
+// sum cannot wrap.
+__device__ __forceinline__ size_t row_limit(const SoftmaxScaling& sc, size_t row, size_t cols) {
+  if (sc.period == 0) return cols;
+  size_t rem;
+  if (sc.fast32) {
+    const uint32_t n = static_cast<uint32_t>(sc.row0 + row);
+    const uint32_t t = __umulhi(sc.magic, n);
+    const uint32_t quot = (t + ((n - t) >> sc.shift1)) >> sc.shift2;
+    rem = n - quot * static_cast<uint32_t>(sc.period);
+  } else {
+    rem = (sc.row0 + row) % sc.period;
+  }
+  const size_t q = rem + sc.offset;
+  return q < cols ? q + 1 : cols;
+}
+
 // ---------------------------------------------------------------- row I/O
 
 // Load VPT chunks of a team slice as raw 16-byte words (VPT * VEC values).
 // Vectors [vfirst, ve) of the row are the slice; anything outside is -inf.
+// MASK: elements at or after `lim` are -inf too and are not loaded.
 // The scalar (unaligned) path packs its scalar loads into the same layout.
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
-__device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, int t,
+template <typename T, int VPT, int TEAM, bool ALIGNED, bool MASK, typename Idx>
+__device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, Idx lim, int t,
                                             uint4* raw) {
   constexpr int VEC = Elem<T>::VEC;
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
     if constexpr (ALIGNED) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      raw[c] = ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, vi < ve, Elem<T>::kNegInfWord);
+      const Idx e = vi * VEC;
+      const bool live = MASK ? (vi < ve && e < lim) : (vi < ve);
+      raw[c] = ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, live, Elem<T>::kNegInfWord);
+      // vectors wholly past lim were not loaded (all -inf); only the one
+      // that straddles lim needs its tail masked
+      if constexpr (MASK) {
+        if (e < lim && lim - e < static_cast<Idx>(VEC)) raw[c] = Elem<T>::keep_first(raw[c], static_cast<int>(lim - e));
+      }
     } else {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
-      const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+      Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+      if constexpr (MASK) eend = imin(eend, lim);
       float f[VEC];
 #pragma unroll
       for (int k = 0; k < VEC; ++k) {
@@ -155,40 +191,55 @@ __device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx col
 // FOLD (every exponential of the row shares the reference): one FMA and one
 // flush-to-zero MUFU.EX2 per element, 2^(x log2 e - ref log2 e + bias); the
 // rounding of ref*log2(e) and the 2^bias scale are common factors that
-// cancel in the normalisation (bias: see Elem<T>::kFoldBias).
+// cancel in the normalisation (bias: see Elem<T>::kFoldBias; the caller
+// keeps |ref log2 e| below 2^24, see exp_sum_row).
 // Otherwise (blocks or chunks with different references are merged later):
 // (x - ref) is formed first, exact for the largest terms, and no bias is
 // applied, so the partial sums of different references compare directly.
+// k = scale * log2(e) (log2(e) for the plain softmax).
 template <typename T, int VPT, bool FOLD>
-__device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref) {
+__device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref, float k) {
   constexpr int VEC = Elem<T>::VEC;
   float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  const float c = Elem<T>::kFoldBias - ref * kLog2e;
+  const float c = Elem<T>::kFoldBias - ref * k;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     float f[VEC];
     if constexpr (sizeof(T) == 4) {
 #pragma unroll
-      for (int k = 0; k < VEC; ++k) f[k] = v[i * VEC + k];
+      for (int j = 0; j < VEC; ++j) f[j] = v[i * VEC + j];
     } else {
       Elem<T>::unpack(raw[i], f);
     }
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) {
-      const float e = FOLD ? ex2_ftz(fmaf(f[k], kLog2e, c)) : Elem<T>::exp2((f[k] - ref) * kLog2e);
-      v[i * VEC + k] = e;
-      s[k & 3] += e;
+    for (int j = 0; j < VEC; ++j) {
+      const float e = FOLD ? ex2_ftz(fmaf(f[j], k, c)) : Elem<T>::exp2((f[j] - ref) * k);
+      v[i * VEC + j] = e;
+      s[j & 3] += e;
     }
   }
   return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
+// Exponentials of values that all share the reference m, the max of the
+// whole row.  The folded form takes 2^(x k - fl(m k)): the rounding error of
+// fl(m k), up to |m k| 2^-24 in the exponent, scales every term of the row
+// alike and cancels in the normalisation -- but only while it is small, or
+// the terms overflow or flush.  So the row folds only when |m k| < 2^24 (an
+// error of at most 1/2 in the exponent); rows with larger maxima (beyond
+// about 1.2e7 at scale 1) take the unfolded form, one uniform branch per row.
+template <typename T, int VPT>
+__device__ __forceinline__ float exp_sum_row(const uint4* raw, float* v, float m, float k) {
+  if (fabsf(m * k) < 0x1p24f) return exp_sum<T, VPT, true>(raw, v, m, k);
+  return exp_sum<T, VPT, false>(raw, v, exp_ref(m), k);
+}
+
 // Row loads: raw 16-byte words; fp32 rows are unpacked into v at once (the
 // same bits), bf16 rows stay packed until exp_sum.
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
-__device__ __forceinline__ void load_row(const T* row, Idx vfirst, Idx ve, Idx cols, int t, uint4* raw,
-                                         float* v) {
-  load_chunks<T, VPT, TEAM, ALIGNED, Idx>(row, vfirst, ve, cols, t, raw);
+template <typename T, int VPT, int TEAM, bool ALIGNED, bool MASK, typename Idx>
+__device__ __forceinline__ void load_row(const T* row, Idx vfirst, Idx ve, Idx cols, Idx lim, int t,
+                                         uint4* raw, float* v) {
+  load_chunks<T, VPT, TEAM, ALIGNED, MASK, Idx>(row, vfirst, ve, cols, lim, t, raw);
   if constexpr (sizeof(T) == 4) {
 #pragma unroll
     for (int i = 0; i < VPT; ++i) Elem<T>::unpack(raw[i], v + i * Elem<T>::VEC);
@@ -207,13 +258,14 @@ __device__ __forceinline__ float row_max(const uint4* raw, const float* v) {
 
 // ---------------------------------------------------------------- warp path
 
-template <typename T, int VPT, bool ALIGNED>
+template <typename T, int VPT, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(kWarpThreads)
-    softmax_warp_kernel(const T* x, T* y, size_t rows, int cols) {
+    softmax_warp_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int E = VPT * VEC;
   const int lane = threadIdx.x & 31;
   const int nvec = (cols + VEC - 1) / VEC;
+  const float k = SC ? sc.k : kLog2e;
   const size_t stride = static_cast<size_t>(gridDim.x) * kWarpRowsPerBlock;
   for (size_t row = static_cast<size_t>(blockIdx.x) * kWarpRowsPerBlock + (threadIdx.x >> 5);
        row < rows; row += stride) {
@@ -221,9 +273,10 @@ __global__ void __launch_bounds__(kWarpThreads)
     T* yr = y + row * static_cast<size_t>(cols);
     uint4 raw[VPT];
     float v[E];
-    load_row<T, VPT, 32, ALIGNED, int>(xr, 0, nvec, cols, lane, raw, v);
+    const int lim = SC ? static_cast<int>(row_limit(sc, row, cols)) : cols;
+    load_row<T, VPT, 32, ALIGNED, SC, int>(xr, 0, nvec, cols, lim, lane, raw, v);
     const float m = warp_max(row_max<T, VPT>(raw, v));
-    const float s = warp_sum(exp_sum<T, VPT, true>(raw, v, m));
+    const float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k));
     store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, Elem<T>::recip(s));
   }
 }
@@ -251,7 +304,8 @@ __device__ __forceinline__ void exchange_init(ClusterExchange& ex) {
 // the row.  A block exits only after all pushes addressed to it have
 // landed, and it pushes only to blocks that are waiting for it, so no block
 // touches the shared memory of a block that has exited.
-__device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, float l, int csize, int crank) {
+__device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, float l, int csize, int crank,
+                                                 float k) {
   const int t = threadIdx.x, lane = t & 31;
   if (t == 0) mbar_arrive_expect_tx(&ex.bar, static_cast<uint32_t>(csize - 1) * 8u);
   cluster_wait();
@@ -265,16 +319,16 @@ __device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, f
     li = q.y;
   }
   const float M = warp_max(mi);
-  const float L = warp_sum(lane < csize ? li * rescale(mi, M) : 0.0f);
+  const float L = warp_sum(lane < csize ? li * rescale(mi, M, k) : 0.0f);
   return make_float2(M, L);
 }
 
 // ---------------------------------------------------------------- block path
 
 // One block per row; EPT = register-resident elements per thread.
-template <typename T, int THREADS, int EPT, bool ALIGNED>
+template <typename T, int THREADS, int EPT, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(THREADS)
-    softmax_block_kernel(const T* x, T* y, size_t rows, int cols) {
+    softmax_block_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = EPT / VEC;
   constexpr int E = VPT * VEC;
@@ -285,12 +339,14 @@ __global__ void __launch_bounds__(THREADS)
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int nvec = (cols + VEC - 1) / VEC;
+  const float k = SC ? sc.k : kLog2e;
   for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
     uint4 raw[VPT];
     float v[E];
-    load_row<T, VPT, THREADS, ALIGNED, int>(xr, 0, nvec, cols, t, raw, v);
+    const int lim = SC ? static_cast<int>(row_limit(sc, row, cols)) : cols;
+    load_row<T, VPT, THREADS, ALIGNED, SC, int>(xr, 0, nvec, cols, lim, t, raw, v);
 
     float m = warp_max(row_max<T, VPT>(raw, v));
     if (lane == 0) red_max[warp] = m;
@@ -299,7 +355,7 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
 
-    float s = warp_sum(exp_sum<T, VPT, true>(raw, v, m));
+    float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k));
     if (lane == 0) red_sum[warp] = s;
     __syncthreads();
     s = red_sum[0];
@@ -315,9 +371,9 @@ __global__ void __launch_bounds__(THREADS)
 
 // A cluster of csize blocks per row; block `rank` holds vectors
 // [rank*per, (rank+1)*per) of the row in registers, per = ceil(nvec / csize).
-template <typename T, int THREADS, int EPT, bool ALIGNED>
+template <typename T, int THREADS, int EPT, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(THREADS)
-    softmax_cluster_kernel(const T* x, T* y, size_t rows, int cols) {
+    softmax_cluster_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = EPT / VEC;
   constexpr int E = VPT * VEC;
@@ -343,9 +399,11 @@ __global__ void __launch_bounds__(THREADS)
 
   const T* xr = x + row * static_cast<size_t>(cols);
   T* yr = y + row * static_cast<size_t>(cols);
+  const float k = SC ? sc.k : kLog2e;
+  const int lim = SC ? static_cast<int>(row_limit(sc, row, cols)) : cols;
   uint4 raw[VPT];
   float v[E];
-  load_row<T, VPT, THREADS, ALIGNED, int>(xr, vb, ve, cols, t, raw, v);
+  load_row<T, VPT, THREADS, ALIGNED, SC, int>(xr, vb, ve, cols, lim, t, raw, v);
 
   float m = warp_max(row_max<T, VPT>(raw, v));
   if (lane == 0) red_max[warp] = m;
@@ -356,39 +414,42 @@ __global__ void __launch_bounds__(THREADS)
 
   // Blocks use different references, so the exponent difference is formed
   // first (exact for the largest terms) instead of folded into an FMA.
-  float s = warp_sum(exp_sum<T, VPT, false>(raw, v, exp_ref(m)));
+  float s = warp_sum(exp_sum<T, VPT, false>(raw, v, exp_ref(m), k));
   if (lane == 0) red_sum[warp] = s;
   __syncthreads();
   s = red_sum[0];
 #pragma unroll
   for (int w = 1; w < NW; ++w) s += red_sum[w];
 
-  const float2 ML = exchange_merge(ex, m, s, csize, crank);
-  store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, rescale(m, ML.x) * __frcp_rn(ML.y));
+  const float2 ML = exchange_merge(ex, m, s, csize, crank, k);
+  store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, rescale(m, ML.x, k) * __frcp_rn(ML.y));
 }
 
 // ---------------------------------------------------------------- two-phase path
 
-__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2, float k) {
   const float M = fmaxf(m, m2);
-  l = l * rescale(m, M) + l2 * rescale(m2, M);
+  l = l * rescale(m, M, k) + l2 * rescale(m2, M, k);
   m = M;
 }
 
 // Streaming pass 1 over vectors [vb, ve) of a row: running (m, l) per thread
 // (the online recurrence of lecture 6, section 7.2), chunk by chunk.
-template <typename T, int THREADS, int VPT, bool ALIGNED>
-__device__ __forceinline__ void stream_stats(const T* xr, size_t vb, size_t ve, size_t cols, int t, float& m,
-                                             float& l) {
-  constexpr int E = VPT * Elem<T>::VEC;
+// MASK: only elements before lim count; chunks wholly after it are skipped.
+template <typename T, int THREADS, int VPT, bool ALIGNED, bool MASK>
+__device__ __forceinline__ void stream_stats(const T* xr, size_t vb, size_t ve, size_t cols, size_t lim, int t,
+                                             float k, float& m, float& l) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int E = VPT * VEC;
   constexpr size_t STEP = static_cast<size_t>(THREADS) * VPT;
+  if constexpr (MASK) ve = imin(ve, (lim + VEC - 1) / VEC);
   for (size_t c = vb; c < ve; c += STEP) {
     uint4 raw[VPT];
     float v[E];
-    load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
+    load_row<T, VPT, THREADS, ALIGNED, MASK, size_t>(xr, c, ve, cols, lim, t, raw, v);
     const float mn = fmaxf(m, row_max<T, VPT>(raw, v));
-    const float acc = exp_sum<T, VPT, false>(raw, v, exp_ref(mn));
-    l = l * rescale(m, mn) + acc;
+    const float acc = exp_sum<T, VPT, false>(raw, v, exp_ref(mn), k);
+    l = l * rescale(m, mn, k) + acc;
     m = mn;
   }
 }
@@ -397,26 +458,27 @@ __device__ __forceinline__ void stream_stats(const T* xr, size_t vb, size_t ve, 
 // `red` holds THREADS/32 entries; the caller must not reuse it before a
 // following __syncthreads.
 template <int THREADS>
-__device__ __forceinline__ void block_merge_ml(float& m, float& l, float2* red) {
+__device__ __forceinline__ void block_merge_ml(float& m, float& l, float2* red, float k) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
     const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-    merge_ml(m, l, m2, l2);
+    merge_ml(m, l, m2, l2, k);
   }
   if (lane == 0) red[warp] = make_float2(m, l);
   __syncthreads();
   m = red[0].x;
   l = red[0].y;
 #pragma unroll
-  for (int w = 1; w < THREADS / 32; ++w) merge_ml(m, l, red[w].x, red[w].y);
+  for (int w = 1; w < THREADS / 32; ++w) merge_ml(m, l, red[w].x, red[w].y, k);
 }
 
-// Streaming pass 2 over vectors [vb, ve): y = exp(x - M) / L.
-template <typename T, int THREADS, int VPT, bool ALIGNED>
-__device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, size_t ve, size_t cols, int t,
-                                                 float M, float L) {
+// Streaming pass 2 over vectors [vb, ve): y = exp(x - M) / L (MASK: 0 at
+// and after lim, without loading those elements).
+template <typename T, int THREADS, int VPT, bool ALIGNED, bool MASK>
+__device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, size_t ve, size_t cols, size_t lim,
+                                                 int t, float k, float M, float L) {
   constexpr int E = VPT * Elem<T>::VEC;
   constexpr size_t STEP = static_cast<size_t>(THREADS) * VPT;
   const float r = __frcp_rn(L);
@@ -424,15 +486,15 @@ __device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, 
   for (size_t c = vb; c < ve; c += STEP) {
     uint4 raw[VPT];
     float v[E];
-    load_row<T, VPT, THREADS, ALIGNED, size_t>(xr, c, ve, cols, t, raw, v);
-    exp_sum<T, VPT, false>(raw, v, ref);
+    load_row<T, VPT, THREADS, ALIGNED, MASK, size_t>(xr, c, ve, cols, lim, t, raw, v);
+    exp_sum<T, VPT, false>(raw, v, ref, k);
     store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
   }
 }
 
-template <typename T, bool ALIGNED>
+template <typename T, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(kTwoPhaseThreads)
-    softmax_twophase_kernel(const T* x, T* y, size_t rows, size_t cols) {
+    softmax_twophase_kernel(const T* x, T* y, size_t rows, size_t cols, SoftmaxScaling sc) {
   constexpr int THREADS = kTwoPhaseThreads;
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
@@ -456,21 +518,23 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   }
   const T* xr = x + row * cols;
   T* yr = y + row * cols;
+  const float k = SC ? sc.k : kLog2e;
+  const size_t lim = SC ? row_limit(sc, row, cols) : cols;
 
   // pass 1: running (m, l) per thread, then merged over the block
   float m = -INFINITY, l = 0.0f;
-  stream_stats<T, THREADS, VPT, ALIGNED>(xr, vb, ve, cols, t, m, l);
-  block_merge_ml<THREADS>(m, l, red);
+  stream_stats<T, THREADS, VPT, ALIGNED, SC>(xr, vb, ve, cols, lim, t, k, m, l);
+  block_merge_ml<THREADS>(m, l, red, k);
 
   // merge the blocks' partials across the cluster
   if (csize > 1) {
-    const float2 ML = exchange_merge(ex, m, l, csize, crank);
+    const float2 ML = exchange_merge(ex, m, l, csize, crank, k);
     m = ML.x;
     l = ML.y;
   }
 
   // pass 2: y = exp(x - M) / L
-  stream_normalise<T, THREADS, VPT, ALIGNED>(xr, yr, vb, ve, cols, t, m, l);
+  stream_normalise<T, THREADS, VPT, ALIGNED, SC>(xr, yr, vb, ve, cols, lim, t, k, m, l);
 }
 
 // ---------------------------------------------------------------- split path
@@ -483,9 +547,10 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
 // is independent (no waits), and the number of blocks does not depend on the
 // number of rows.
 
-template <typename T, bool ALIGNED>
+template <typename T, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(kTwoPhaseThreads)
-    softmax_split_stats_kernel(const T* x, float2* ws, size_t cols, size_t chunk, unsigned nchunks) {
+    softmax_split_stats_kernel(const T* x, float2* ws, size_t cols, size_t chunk, unsigned nchunks,
+                               SoftmaxScaling sc) {
   constexpr int THREADS = kTwoPhaseThreads;
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
@@ -495,16 +560,18 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   const size_t nvec = (cols + VEC - 1) / VEC;
   const size_t vb = imin(nvec, c * chunk);
   const size_t ve = imin(nvec, vb + chunk);
+  const float k = SC ? sc.k : kLog2e;
+  const size_t lim = SC ? row_limit(sc, row, cols) : cols;
   float m = -INFINITY, l = 0.0f;
-  stream_stats<T, THREADS, VPT, ALIGNED>(x + row * cols, vb, ve, cols, threadIdx.x, m, l);
-  block_merge_ml<THREADS>(m, l, red);
+  stream_stats<T, THREADS, VPT, ALIGNED, SC>(x + row * cols, vb, ve, cols, lim, threadIdx.x, k, m, l);
+  block_merge_ml<THREADS>(m, l, red, k);
   if (threadIdx.x == 0) ws[blockIdx.x] = make_float2(m, l);
 }
 
-template <typename T, bool ALIGNED>
+template <typename T, bool ALIGNED, bool SC>
 __global__ void __launch_bounds__(kTwoPhaseThreads)
     softmax_split_norm_kernel(const T* x, T* y, const float2* ws, size_t cols, size_t chunk,
-                              unsigned nchunks) {
+                              unsigned nchunks, SoftmaxScaling sc) {
   constexpr int THREADS = kTwoPhaseThreads;
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = kTwoPhaseElemsPerThread / VEC;
@@ -514,12 +581,15 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   const size_t nvec = (cols + VEC - 1) / VEC;
   const size_t vb = imin(nvec, c * chunk);
   const size_t ve = imin(nvec, vb + chunk);
+  const float k = SC ? sc.k : kLog2e;
+  const size_t lim = SC ? row_limit(sc, row, cols) : cols;
   // merge the row's partials
   const float2* part = ws + row * nchunks;
   float m = -INFINITY, l = 0.0f;
-  for (unsigned i = threadIdx.x; i < nchunks; i += THREADS) merge_ml(m, l, part[i].x, part[i].y);
-  block_merge_ml<THREADS>(m, l, red);
-  stream_normalise<T, THREADS, VPT, ALIGNED>(x + row * cols, y + row * cols, vb, ve, cols, threadIdx.x, m, l);
+  for (unsigned i = threadIdx.x; i < nchunks; i += THREADS) merge_ml(m, l, part[i].x, part[i].y, k);
+  block_merge_ml<THREADS>(m, l, red, k);
+  stream_normalise<T, THREADS, VPT, ALIGNED, SC>(x + row * cols, y + row * cols, vb, ve, cols, lim, threadIdx.x, k,
+                                                 m, l);
 }
 
 // A wait on an mbarrier that nothing ever arrives on: every thread gives up
@@ -566,59 +636,59 @@ cudaError_t launch(void (*kernel)(KArgs...), size_t blocks, int threads, int clu
 
 constexpr size_t kMaxGrid = 0x7fffffffu;
 
-template <typename T, bool ALIGNED>
-cudaError_t launch_warp(const void* x, void* y, size_t rows, size_t cols, int vpt,
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_warp(const T* xp, T* yp, size_t rows, size_t cols, int vpt, SoftmaxScaling sc,
                         cudaStream_t s) {
   size_t blocks = (rows + kWarpRowsPerBlock - 1) / kWarpRowsPerBlock;
   if (blocks > kMaxGrid) blocks = kMaxGrid;
-  const T* xp = static_cast<const T*>(x);
-  T* yp = static_cast<T*>(y);
   const int c = static_cast<int>(cols);
   switch (vpt) {
-    case 1: return launch(softmax_warp_kernel<T, 1, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
-    case 2: return launch(softmax_warp_kernel<T, 2, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
-    case 4: return launch(softmax_warp_kernel<T, 4, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
-    case 8: return launch(softmax_warp_kernel<T, 8, ALIGNED>, blocks, kWarpThreads, 1, s, xp, yp, rows, c);
+    case 1: return launch(softmax_warp_kernel<T, 1, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
+    case 2: return launch(softmax_warp_kernel<T, 2, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
+    case 4: return launch(softmax_warp_kernel<T, 4, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
+    case 8: return launch(softmax_warp_kernel<T, 8, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, int EPT, bool ALIGNED>
-cudaError_t launch_block_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads,
+template <typename T, int EPT, bool ALIGNED, bool SC>
+cudaError_t launch_block_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads, SoftmaxScaling sc,
                              cudaStream_t s) {
   switch (threads) {
-    case 128: return launch(softmax_block_kernel<T, 128, EPT, ALIGNED>, blocks, 128, 1, s, xp, yp, rows, c);
-    case 256: return launch(softmax_block_kernel<T, 256, EPT, ALIGNED>, blocks, 256, 1, s, xp, yp, rows, c);
-    case 512: return launch(softmax_block_kernel<T, 512, EPT, ALIGNED>, blocks, 512, 1, s, xp, yp, rows, c);
-    case 1024: return launch(softmax_block_kernel<T, 1024, EPT, ALIGNED>, blocks, 1024, 1, s, xp, yp, rows, c);
+    case 128: return launch(softmax_block_kernel<T, 128, EPT, ALIGNED, SC>, blocks, 128, 1, s, xp, yp, rows, c, sc);
+    case 256: return launch(softmax_block_kernel<T, 256, EPT, ALIGNED, SC>, blocks, 256, 1, s, xp, yp, rows, c, sc);
+    case 512: return launch(softmax_block_kernel<T, 512, EPT, ALIGNED, SC>, blocks, 512, 1, s, xp, yp, rows, c, sc);
+    case 1024:
+      return launch(softmax_block_kernel<T, 1024, EPT, ALIGNED, SC>, blocks, 1024, 1, s, xp, yp, rows, c, sc);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, bool ALIGNED>
-cudaError_t launch_block(const void* x, void* y, size_t rows, size_t cols, int threads, int vpt,
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_block(const T* xp, T* yp, size_t rows, size_t cols, int threads, int vpt, SoftmaxScaling sc,
                          cudaStream_t s) {
   const size_t blocks = rows < kMaxGrid ? rows : kMaxGrid;
-  const T* xp = static_cast<const T*>(x);
-  T* yp = static_cast<T*>(y);
   const int c = static_cast<int>(cols);
   switch (vpt * Elem<T>::VEC) {
-    case 16: return launch_block_ept<T, 16, ALIGNED>(xp, yp, rows, c, blocks, threads, s);
-    case 32: return launch_block_ept<T, 32, ALIGNED>(xp, yp, rows, c, blocks, threads, s);
+    case 16: return launch_block_ept<T, 16, ALIGNED, SC>(xp, yp, rows, c, blocks, threads, sc, s);
+    case 32: return launch_block_ept<T, 32, ALIGNED, SC>(xp, yp, rows, c, blocks, threads, sc, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T, int EPT, bool ALIGNED>
-cudaError_t launch_cluster_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads,
-                               int k, cudaStream_t s) {
+template <typename T, int EPT, bool ALIGNED, bool SC>
+cudaError_t launch_cluster_ept(const T* xp, T* yp, size_t rows, int c, size_t blocks, int threads, int k,
+                               SoftmaxScaling sc, cudaStream_t s) {
   switch (threads) {
-    case 128: return launch(softmax_cluster_kernel<T, 128, EPT, ALIGNED>, blocks, 128, k, s, xp, yp, rows, c);
-    case 256: return launch(softmax_cluster_kernel<T, 256, EPT, ALIGNED>, blocks, 256, k, s, xp, yp, rows, c);
-    case 512: return launch(softmax_cluster_kernel<T, 512, EPT, ALIGNED>, blocks, 512, k, s, xp, yp, rows, c);
+    case 128:
+      return launch(softmax_cluster_kernel<T, 128, EPT, ALIGNED, SC>, blocks, 128, k, s, xp, yp, rows, c, sc);
+    case 256:
+      return launch(softmax_cluster_kernel<T, 256, EPT, ALIGNED, SC>, blocks, 256, k, s, xp, yp, rows, c, sc);
+    case 512:
+      return launch(softmax_cluster_kernel<T, 512, EPT, ALIGNED, SC>, blocks, 512, k, s, xp, yp, rows, c, sc);
     case 1024:
       if constexpr (EPT <= 32) {
-        return launch(softmax_cluster_kernel<T, 1024, EPT, ALIGNED>, blocks, 1024, k, s, xp, yp, rows, c);
+        return launch(softmax_cluster_kernel<T, 1024, EPT, ALIGNED, SC>, blocks, 1024, k, s, xp, yp, rows, c, sc);
       }
       return cudaErrorInvalidValue;  // 64 values per thread do not fit 1024 threads' registers
     default: return cudaErrorInvalidValue;
@@ -627,23 +697,23 @@ cudaError_t launch_cluster_ept(const T* xp, T* yp, size_t rows, int c, size_t bl
 
 // Cluster launches handle one row per cluster; rows beyond one grid's worth
 // of clusters go to further launches.
-template <typename T, bool ALIGNED>
-cudaError_t launch_cluster(const void* x, void* y, size_t rows, size_t cols, int threads, int vpt,
-                           int cluster, cudaStream_t s) {
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_cluster(const T* xp, T* yp, size_t rows, size_t cols, int threads, int vpt, int cluster,
+                           SoftmaxScaling sc, cudaStream_t s) {
   const size_t cl = static_cast<size_t>(cluster);
   const size_t max_rows = kMaxGrid / cl;
-  const T* xp = static_cast<const T*>(x);
-  T* yp = static_cast<T*>(y);
   const int c = static_cast<int>(cols);
+  const size_t row0 = sc.row0;
   for (size_t r0 = 0; r0 < rows; r0 += max_rows) {
     const size_t n = (rows - r0 < max_rows) ? rows - r0 : max_rows;
     const T* xs = xp + r0 * cols;
     T* ys = yp + r0 * cols;
+    sc.row0 = row0 + r0;
     cudaError_t e;
     switch (vpt * Elem<T>::VEC) {
-      case 16: e = launch_cluster_ept<T, 16, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
-      case 32: e = launch_cluster_ept<T, 32, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
-      case 64: e = launch_cluster_ept<T, 64, ALIGNED>(xs, ys, n, c, n * cl, threads, cluster, s); break;
+      case 16: e = launch_cluster_ept<T, 16, ALIGNED, SC>(xs, ys, n, c, n * cl, threads, cluster, sc, s); break;
+      case 32: e = launch_cluster_ept<T, 32, ALIGNED, SC>(xs, ys, n, c, n * cl, threads, cluster, sc, s); break;
+      case 64: e = launch_cluster_ept<T, 64, ALIGNED, SC>(xs, ys, n, c, n * cl, threads, cluster, sc, s); break;
       default: e = cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
@@ -651,15 +721,17 @@ cudaError_t launch_cluster(const void* x, void* y, size_t rows, size_t cols, int
   return cudaSuccess;
 }
 
-template <typename T, bool ALIGNED>
-cudaError_t launch_twophase(const void* x, void* y, size_t rows, size_t cols, int cluster,
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_twophase(const T* xp, T* yp, size_t rows, size_t cols, int cluster, SoftmaxScaling sc,
                             cudaStream_t s) {
   const size_t cl = static_cast<size_t>(cluster);
   const size_t max_rows = kMaxGrid / cl;
+  const size_t row0 = sc.row0;
   for (size_t r0 = 0; r0 < rows; r0 += max_rows) {
     const size_t n = (rows - r0 < max_rows) ? rows - r0 : max_rows;
-    const cudaError_t e = launch(softmax_twophase_kernel<T, ALIGNED>, n * cl, kTwoPhaseThreads, cluster, s,
-                                 static_cast<const T*>(x) + r0 * cols, static_cast<T*>(y) + r0 * cols, n, cols);
+    sc.row0 = row0 + r0;
+    const cudaError_t e = launch(softmax_twophase_kernel<T, ALIGNED, SC>, n * cl, kTwoPhaseThreads, cluster, s,
+                                 xp + r0 * cols, yp + r0 * cols, n, cols, sc);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -667,52 +739,63 @@ cudaError_t launch_twophase(const void* x, void* y, size_t rows, size_t cols, in
 
 // Stats then normalise, batch by batch of rows (a batch's partials fit the
 // workspace; batches run in stream order, so the workspace is reused).
-template <typename T, bool ALIGNED>
-cudaError_t launch_split(const void* x, void* y, size_t rows, size_t cols, const SplitGeometry& g, void* ws,
-                         cudaStream_t s) {
-  const T* xp = static_cast<const T*>(x);
-  T* yp = static_cast<T*>(y);
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_split(const T* xp, T* yp, size_t rows, size_t cols, const SplitGeometry& g, void* ws,
+                         SoftmaxScaling sc, cudaStream_t s) {
   float2* w = static_cast<float2*>(ws);
+  const size_t row0 = sc.row0;
   for (size_t r0 = 0; r0 < rows; r0 += g.rows_per_launch) {
     const size_t n = (rows - r0 < g.rows_per_launch) ? rows - r0 : g.rows_per_launch;
     const size_t blocks = n * g.nchunks;
-    cudaError_t e = launch(softmax_split_stats_kernel<T, ALIGNED>, blocks, kTwoPhaseThreads, 1, s,
-                           xp + r0 * cols, w, cols, g.chunk_vecs, g.nchunks);
+    sc.row0 = row0 + r0;
+    cudaError_t e = launch(softmax_split_stats_kernel<T, ALIGNED, SC>, blocks, kTwoPhaseThreads, 1, s,
+                           xp + r0 * cols, w, cols, g.chunk_vecs, g.nchunks, sc);
     if (e != cudaSuccess) return e;
-    e = launch(softmax_split_norm_kernel<T, ALIGNED>, blocks, kTwoPhaseThreads, 1, s, xp + r0 * cols,
-               yp + r0 * cols, static_cast<const float2*>(w), cols, g.chunk_vecs, g.nchunks);
+    e = launch(softmax_split_norm_kernel<T, ALIGNED, SC>, blocks, kTwoPhaseThreads, 1, s, xp + r0 * cols,
+               yp + r0 * cols, static_cast<const float2*>(w), cols, g.chunk_vecs, g.nchunks, sc);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
 
-template <typename T, bool ALIGNED>
-cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols,
-                         const fk_softmax_plan& p, void* ws, cudaStream_t s) {
+template <typename T, bool ALIGNED, bool SC>
+cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols, const fk_softmax_plan& p, void* ws,
+                         const SoftmaxScaling& sc, cudaStream_t s) {
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
   switch (p.path) {
-    case FK_PATH_WARP: return launch_warp<T, ALIGNED>(x, y, rows, cols, p.vpt, s);
-    case FK_PATH_CTA: return launch_block<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, s);
+    case FK_PATH_WARP: return launch_warp<T, ALIGNED, SC>(xp, yp, rows, cols, p.vpt, sc, s);
+    case FK_PATH_CTA: return launch_block<T, ALIGNED, SC>(xp, yp, rows, cols, p.threads, p.vpt, sc, s);
     case FK_PATH_CLUSTER:
-      return launch_cluster<T, ALIGNED>(x, y, rows, cols, p.threads, p.vpt, p.cluster, s);
-    case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED>(x, y, rows, cols, p.cluster, s);
+      return launch_cluster<T, ALIGNED, SC>(xp, yp, rows, cols, p.threads, p.vpt, p.cluster, sc, s);
+    case FK_PATH_TWOPHASE: return launch_twophase<T, ALIGNED, SC>(xp, yp, rows, cols, p.cluster, sc, s);
     case FK_PATH_SPLIT:
-      return launch_split<T, ALIGNED>(x, y, rows, cols, split_geometry(rows, cols, Elem<T>::VEC == 8 ? FK_BF16 : FK_F32), ws, s);
+      return launch_split<T, ALIGNED, SC>(xp, yp, rows, cols,
+                                          split_geometry(rows, cols, Elem<T>::VEC == 8 ? FK_BF16 : FK_F32), ws, sc, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <typename T>
+cudaError_t launch_dtype(const void* x, void* y, size_t rows, size_t cols, const fk_softmax_plan& p, bool aligned,
+                         void* ws, const SoftmaxScaling* sc, cudaStream_t s) {
+  if (sc == nullptr) {
+    const SoftmaxScaling none = {kLog2e, 0, 0, 0};
+    return aligned ? launch_typed<T, true, false>(x, y, rows, cols, p, ws, none, s)
+                   : launch_typed<T, false, false>(x, y, rows, cols, p, ws, none, s);
+  }
+  return aligned ? launch_typed<T, true, true>(x, y, rows, cols, p, ws, *sc, s)
+                 : launch_typed<T, false, true>(x, y, rows, cols, p, ws, *sc, s);
 }
 
 }  // namespace
 
 cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                           const fk_softmax_plan& plan, bool aligned, void* ws, const DeviceInfo& dev,
-                           cudaStream_t stream) {
+                           const fk_softmax_plan& plan, bool aligned, void* ws, const SoftmaxScaling* sc,
+                           const DeviceInfo& dev, cudaStream_t stream) {
   (void)dev;
-  if (dtype == FK_F32) {
-    return aligned ? launch_typed<float, true>(x, y, rows, cols, plan, ws, stream)
-                   : launch_typed<float, false>(x, y, rows, cols, plan, ws, stream);
-  }
-  return aligned ? launch_typed<__nv_bfloat16, true>(x, y, rows, cols, plan, ws, stream)
-                 : launch_typed<__nv_bfloat16, false>(x, y, rows, cols, plan, ws, stream);
+  if (dtype == FK_F32) return launch_dtype<float>(x, y, rows, cols, plan, aligned, ws, sc, stream);
+  return launch_dtype<__nv_bfloat16>(x, y, rows, cols, plan, aligned, ws, sc, stream);
 }
 
 cudaError_t read_wait_timeouts(unsigned* out, bool reset) {

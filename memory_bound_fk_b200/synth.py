@@ -63,8 +63,22 @@ class Workload:
 
     @property
     def algorithmic_bytes(self) -> int:
-        """One read of the input plus one write of the output."""
-        return 2 * self.numel * self.itemsize
+        return algorithmic_bytes(self.op, self.itemsize, self.shape)
+
+
+def algorithmic_bytes(op: str, itemsize: int, shape: tuple) -> int:
+    """One read of the input plus one write of the output.  For the causal
+    softmax (rows in blocks of T = cols queries against T keys) only the kept
+    entries are read: row i of a block reads i + 1 of its T values."""
+    if op == "softmax_causal":
+        rows, cols = shape
+        full, rem = divmod(rows, cols)
+        kept = full * cols * (cols + 1) // 2 + rem * (rem + 1) // 2
+        return (kept + rows * cols) * itemsize
+    n = 1
+    for d in shape:
+        n *= d
+    return 2 * n * itemsize
 
 
 WORKLOADS = {
@@ -81,6 +95,16 @@ WORKLOADS = {
                  "bf16 1048576x2048 (32x16 heads x 2048 queries), N(0,8^2), causal -inf"),
         Workload("cfg5_softmax", "softmax", "f32", (512, 131072), 4,
                  "fp32 512x131072, N(0,2^2), +50 at one position per row"),
+        # variants of the same operators (exact GELU, bf16 GELU, softmax with
+        # the causal mask generated in the kernel)
+        Workload("cfg2_gelu_erf", "gelu_erf", "f32", (8388608,), 1,
+                 "the cfg2_gelu values, exact GELU x*Phi(x)"),
+        Workload("gelu_bf16", "gelu", "bf16", (16777216,), 5,
+                 "bf16 16777216 (32 MiB), N(0,1) with 167772 positions redrawn U[-20,20]"),
+        Workload("gelu_erf_bf16", "gelu_erf", "bf16", (16777216,), 5,
+                 "the gelu_bf16 values, exact GELU x*Phi(x)"),
+        Workload("cfg4_causal", "softmax_causal", "bf16", (32 * 16 * 2048, 2048), 3,
+                 "the cfg4_softmax scores, causal mask generated in the kernel (masked entries not read)"),
     ]
 }
 
@@ -246,9 +270,13 @@ def make(name: str, threads: int | None = None, rows: int | None = None) -> np.n
     if name == "cfg3_softmax":
         r = rows or 8192
         return _cfg3(rows=-(-r // CFG3_ROWS_PER_CHUNK) * CFG3_ROWS_PER_CHUNK, threads=threads)[:r]
-    if name == "cfg4_softmax":
+    if name in ("cfg4_softmax", "cfg4_causal"):
         r = rows or CFG4_HEADS * CFG4_T
         return _cfg4(heads=-(-r // CFG4_T), threads=threads)[:r]
+    if name == "cfg2_gelu_erf":
+        return _cfg2()[:rows]
+    if name in ("gelu_bf16", "gelu_erf_bf16"):
+        return f32_to_bf16_bits(_cfg2(16777216, seed=5))[:rows]
     if name == "cfg5_softmax":
         r = rows or 512
         return _cfg5(rows=-(-r // CFG5_ROWS_PER_CHUNK) * CFG5_ROWS_PER_CHUNK, threads=threads)[:r]

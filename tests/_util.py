@@ -66,3 +66,27 @@ def check_softmax_bf16(y_bits: np.ndarray, ref_bits: np.ndarray, x_bits: np.ndar
     neg = (x_bits == 0xFF80) & ok
     assert np.all(y_bits[neg] == 0x0000), "-inf input did not give exactly +0"
     return int(d.max()) if d.size else 0
+
+
+def forced_plans(fk, cols, dtype):
+    """Every compiled softmax plan that can hold `cols` columns of `dtype`
+    ("f32" or "bf16"): CTA and cluster shapes, two-phase with 1..16 blocks,
+    split, and the warp path where a row fits a warp."""
+    plans = []
+    vec = 4 if dtype == "f32" else 8
+    for ept in (16, 32):
+        for t in (128, 256, 512, 1024):
+            if t * ept >= cols:
+                plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t, vpt=ept // vec))
+    for ept in (16, 32, 64):
+        for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (512, 16), (1024, 16)):
+            if ept == 64 and t > 512:
+                continue
+            if -(-(-(-cols // vec)) // k) * vec <= t * ept:
+                plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k, vpt=ept // vec))
+    for k in (1, 2, 3, 16):
+        plans.append(fk.make_plan(fk.FK_PATH_TWOPHASE, cluster=k))
+    plans.append(fk.make_plan(fk.FK_PATH_SPLIT))
+    if cols <= (1024 if dtype == "f32" else 2048):
+        plans.append(fk.make_plan(fk.FK_PATH_WARP, vpt=8))
+    return plans

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
-from _util import Guarded, check_softmax_bf16, check_softmax_f32
+from _util import Guarded, check_softmax_bf16, check_softmax_f32, forced_plans
 from memory_bound_fk_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -73,33 +73,12 @@ def test_auto_plan_bf16(fk, torch_mod, rows, cols):
     check(x, run(fk, torch_mod, x))
 
 
-def _forced_plans(fk, cols, dtype):
-    plans = []
-    vec = 4 if dtype == "f32" else 8
-    for ept in (16, 32):
-        for t in (128, 256, 512, 1024):
-            if t * ept >= cols:
-                plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t, vpt=ept // vec))
-    for ept in (16, 32, 64):
-        for t, k in ((128, 2), (128, 3), (256, 5), (128, 8), (128, 16), (512, 16), (1024, 16)):
-            if ept == 64 and t > 512:
-                continue
-            if -(-(-(-cols // vec)) // k) * vec <= t * ept:
-                plans.append(fk.make_plan(fk.FK_PATH_CLUSTER, threads=t, cluster=k, vpt=ept // vec))
-    for k in (1, 2, 3, 16):
-        plans.append(fk.make_plan(fk.FK_PATH_TWOPHASE, cluster=k))
-    plans.append(fk.make_plan(fk.FK_PATH_SPLIT))
-    if cols <= (1024 if dtype == "f32" else 2048):
-        plans.append(fk.make_plan(fk.FK_PATH_WARP, vpt=8))
-    return plans
-
-
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("cols", [1, 100, 1000, 1024, 4096, 50000])
 def test_every_path_on_the_same_input(fk, torch_mod, dtype, cols):
     rows = 6
     x = synth.softmax_input(rows, cols, dtype, sigma=5.0, neg_inf_frac=0.2, seed=cols)
-    for p in _forced_plans(fk, cols, dtype):
+    for p in forced_plans(fk, cols, dtype):
         check(x, run(fk, torch_mod, x, plan=p))
 
 
@@ -152,6 +131,33 @@ def test_large_magnitudes_split_across_blocks(fk, torch_mod, plan_kind):
     y = run(fk, torch_mod, x, plan=plan)
     check(x, y)
     assert abs(float(y[0, 10]) - 0.5) <= 1e-6 and abs(float(y[0, cols - 10]) - 0.5) <= 1e-6
+
+
+@pytest.mark.parametrize("cols", [3, 1000, 4096, 50000])
+def test_large_row_maxima(fk, torch_mod, cols):
+    # Rows whose max m is large: the single-reference form rounds m * log2(e)
+    # and that error (|m log2 e| 2^-24 in the exponent) must not overflow the
+    # terms; such rows take the unfolded form.  Maxima from just below the
+    # switch (1e7) to FLT_MAX, where m * log2(e) itself overflows, must give
+    # the softmax, not NaN, on every path.
+    fmax = np.finfo(np.float32).max
+    x = synth.softmax_input(8, cols, "f32", sigma=1.0, seed=cols)
+    x[0, cols // 2] = fmax                   # one-hot
+    x[1, 0], x[1, cols - 1] = fmax, fmax     # even split (cols >= 2)
+    x[2, :] = -fmax
+    x[2, cols // 3] = 2.5e38                 # one-hot
+    x[3, cols - 1] = 5e37                    # one-hot
+    x[4, cols - 1] = 1e12                    # one-hot
+    x[5] = np.float32(1e9) + np.float32(64) * np.arange(cols) % np.float32(256)  # spacing 64 near 1e9
+    x[6] = np.float32(1e7) + (np.arange(cols) % 5).astype(np.float32)      # below the switch: folded
+    x[7] = np.float32(2e7) + 2 * (np.arange(cols) % 5).astype(np.float32)  # above it: unfolded
+    for p in [None] + forced_plans(fk, cols, "f32"):
+        y = run(fk, torch_mod, x, plan=p)
+        check(x, y)
+        assert y[0, cols // 2] == 1.0 and y[2, cols // 3] == 1.0 and y[4, cols - 1] == 1.0
+    b = oracle.round_to_bf16(x.astype(np.float64))
+    for p in [None] + forced_plans(fk, cols, "bf16"):
+        check(b, run(fk, torch_mod, b, plan=p))
 
 
 def test_api_rejects_overlap_and_out_of_range(fk, torch_mod):
