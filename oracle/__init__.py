@@ -18,6 +18,8 @@ Definitions followed:
     (row max, then exponentials and their sum, then normalise).
   * Scaled, causally masked softmax: the same lecture, section 8 (scores
     scaled, -inf where the key comes after the query, then softmax).
+  * LayerNorm (+ GELU): the same lecture, sections 6.1-6.2 (the fused
+    LayerNorm -> Linear -> GELU example; F.layer_norm over the last axis).
 
 Parity pins: every function here is pinned by tests in
 ``tests/test_oracle_pins.py`` (closed forms, invariants, library routines
@@ -61,6 +63,8 @@ def _load():
             getattr(lib, name).restype = None
         lib.oracle_softmax_rows_causal.argtypes = [p, p, i, sz, sz, d, sz, sz, i]
         lib.oracle_softmax_rows_causal.restype = None
+        lib.oracle_layernorm_rows.argtypes = [p, p, i, sz, sz, p, p, d, i, i]
+        lib.oracle_layernorm_rows.restype = None
         for name in ("oracle_round_to_f32_array", "oracle_round_to_bf16_array",
                      "oracle_bf16_to_f64_array"):
             getattr(lib, name).argtypes = [p, p, sz]
@@ -189,6 +193,33 @@ def softmax_rows_causal(x: np.ndarray, scale: float, period: int, offset: int = 
     return y
 
 
+_GELU_CODES = {None: 0, "tanh": 1, "erf": 2}
+
+
+def layernorm_rows(x: np.ndarray, eps: float = 1e-5, gamma=None, beta=None, gelu: str | None = None,
+                   nthreads: int | None = None) -> np.ndarray:
+    """LayerNorm over the last axis of a [rows, cols] matrix (mean and biased
+    variance of each row, (x - mean) / sqrt(var + eps)), then * gamma + beta
+    (each optional, length cols), then GELU ("tanh", "erf" or None).  float64
+    in -> float64 out; float32 -> float32; uint16 (bf16 patterns) -> uint16;
+    computed in double and rounded once."""
+    kinds = {np.dtype(np.float64): 0, np.dtype(np.float32): 1, np.dtype(np.uint16): 2}
+    if x.dtype not in kinds:
+        raise TypeError("float64, float32 or uint16 (bf16 bits)")
+    x = np.ascontiguousarray(x)
+    rows, cols = _rows_cols(x)
+    g = None if gamma is None else _c(gamma, np.float64)
+    b = None if beta is None else _c(beta, np.float64)
+    for a in (g, b):
+        if a is not None and a.shape != (cols,):
+            raise ValueError("gamma / beta must have cols elements")
+    y = np.empty_like(x)
+    _load().oracle_layernorm_rows(_ptr(x), _ptr(y), kinds[x.dtype], rows, cols,
+                                  None if g is None else _ptr(g), None if b is None else _ptr(b),
+                                  float(eps), _GELU_CODES[gelu], nthreads or default_threads())
+    return y
+
+
 def round_to_f32(v: np.ndarray) -> np.ndarray:
     v = _c(v, np.float64)
     out = np.empty(v.shape, np.float32)
@@ -214,7 +245,7 @@ def bf16_to_f64(b: np.ndarray) -> np.ndarray:
 
 __all__ = [
     "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32", "gelu_erf", "gelu_erf_f64",
-    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16", "softmax_rows_causal",
+    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16", "softmax_rows_causal", "layernorm_rows",
     "round_to_f32", "round_to_bf16", "round_to_f32_scalar", "round_to_bf16_scalar",
     "bf16_to_f64", "default_threads",
 ]

@@ -36,6 +36,9 @@
  *     even (the bf16 rounding works from the double bits directly, so there
  *     is no intermediate fp32 rounding).
  *
+ *   LayerNorm (+ GELU) and the scaled, causally masked softmax: see their
+ *   sections below.
+ *
  * Rows (and GELU element ranges) are split across POSIX threads; each row
  * is computed by exactly one thread with the same sequential arithmetic,
  * so results do not depend on the thread count.
@@ -421,6 +424,80 @@ void oracle_softmax_rows_causal(const void *x, void *y, int kind, size_t rows, s
 {
     causal_ctx c = {x, y, kind, cols, scale, period, offset};
     parallel_ranges(softmax_causal_range, &c, rows, nthreads);
+}
+
+/* ------------------------------------------------------------------ */
+/* LayerNorm over rows (+ optional GELU)                                */
+/* ------------------------------------------------------------------ */
+
+/* The normalisation step of the fused LayerNorm -> Linear -> GELU example
+ * (lecture 6, "GPU Kernels and Triton", sections 6.1 and 6.2, where it is
+ * F.layer_norm(x, x.shape[-1:])): over each row of a [rows, cols] matrix,
+ *     mean = sum_j x_j / cols,   var = sum_j (x_j - mean)^2 / cols,
+ *     y_j  = (x_j - mean) / sqrt(var + eps),
+ * then y_j * gamma_j + beta_j when gamma / beta are given (either may be
+ * NULL: 1 / 0), then GELU when asked (1 = tanh form, 2 = exact form) -- the
+ * activation the same example applies.  Both sums are Neumaier-compensated;
+ * the variance is taken about the computed mean (two passes). */
+static void neumaier_add(double *s, double *c, double v)
+{
+    const double t = *s + v;
+    if (fabs(*s) >= fabs(v))
+        *c += (*s - t) + v;
+    else
+        *c += (v - t) + *s;
+    *s = t;
+}
+
+typedef struct {
+    const void *x;
+    void *y;
+    int kind; /* element kind as causal_ctx: 0 double, 1 fp32, 2 bf16 */
+    size_t cols;
+    const double *gamma, *beta;
+    double eps;
+    int gelu;
+} layernorm_ctx;
+
+static void layernorm_range(void *p, size_t b, size_t e)
+{
+    layernorm_ctx *c = (layernorm_ctx *)p;
+    causal_ctx io = {c->x, c->y, c->kind, c->cols, 1.0, 0, 0};
+    double *v = (double *)malloc(c->cols * sizeof(double) + 1);
+    for (size_t r = b; r < e; ++r) {
+        const size_t base = r * c->cols;
+        double s = 0.0, comp = 0.0;
+        for (size_t j = 0; j < c->cols; ++j) {
+            v[j] = causal_in(&io, base + j);
+            neumaier_add(&s, &comp, v[j]);
+        }
+        const double mean = (s + comp) / (double)c->cols;
+        double q = 0.0, qc = 0.0;
+        for (size_t j = 0; j < c->cols; ++j)
+            neumaier_add(&q, &qc, (v[j] - mean) * (v[j] - mean));
+        const double var = (q + qc) / (double)c->cols;
+        const double rstd = 1.0 / sqrt(var + c->eps);
+        for (size_t j = 0; j < c->cols; ++j) {
+            double y = (v[j] - mean) * rstd;
+            if (c->gamma)
+                y *= c->gamma[j];
+            if (c->beta)
+                y += c->beta[j];
+            if (c->gelu == 1)
+                y = oracle_gelu_tanh(y);
+            else if (c->gelu == 2)
+                y = oracle_gelu_erf(y);
+            causal_out(&io, base + j, y);
+        }
+    }
+    free(v);
+}
+
+void oracle_layernorm_rows(const void *x, void *y, int kind, size_t rows, size_t cols, const double *gamma,
+                           const double *beta, double eps, int gelu, int nthreads)
+{
+    layernorm_ctx c = {x, y, kind, cols, gamma, beta, eps, gelu};
+    parallel_ranges(layernorm_range, &c, rows, nthreads);
 }
 
 /* array forms of the rounding helpers */

@@ -438,6 +438,97 @@ def test_causal_softmax_f32_and_bf16_round_the_double_result_once():
     assert np.array_equal(oracle.softmax_rows_causal(b, 0.6, 16, 3), via64b)
 
 
+# ============================================================ LayerNorm
+# LayerNorm over rows (lecture 6, "GPU Kernels and Triton", sections 6.1-6.2:
+# F.layer_norm(x, x.shape[-1:])), optional affine, optional GELU.
+
+
+@pytest.mark.parametrize("rows,cols,eps,affine,gelu", [
+    (16, 7, 1e-5, False, None), (64, 4096, 1e-5, True, None), (33, 1000, 1e-6, True, "tanh"),
+    (9, 131, 1e-3, False, "erf"), (5, 1, 1e-5, True, None), (3, 65537, 1e-5, True, "erf")])
+def test_layernorm_matches_torch_float64(rows, cols, eps, affine, gelu):
+    x = RNG.standard_normal((rows, cols)) * RNG.uniform(0.1, 5, (rows, 1)) + RNG.uniform(-3, 3, (rows, 1))
+    g = RNG.standard_normal(cols) * 0.3 + 1 if affine else None
+    b = RNG.standard_normal(cols) * 0.3 if affine else None
+    y = oracle.layernorm_rows(x, eps, g, b, gelu)
+    t = torch.nn.functional.layer_norm(torch.from_numpy(x), (cols,),
+                                       None if g is None else torch.from_numpy(g),
+                                       None if b is None else torch.from_numpy(b), eps)
+    if gelu:
+        t = torch.nn.functional.gelu(t, approximate="tanh" if gelu == "tanh" else "none")
+    assert np.max(np.abs(y - t.numpy())) <= 1e-13
+
+
+def test_layernorm_moments_and_constant_rows():
+    # without affine and with eps = 0 each row has mean 0 and mean square 1;
+    # with eps the mean square is var / (var + eps); a constant row is 0
+    x = RNG.standard_normal((50, 300)) * 2.5 + 7.0
+    y = oracle.layernorm_rows(x, 0.0)
+    assert np.max(np.abs(y.mean(axis=1))) <= 1e-15 * 50
+    assert np.max(np.abs((y * y).mean(axis=1) - 1.0)) <= 1e-14
+    eps = 0.3
+    ye = oracle.layernorm_rows(x, eps)
+    var = x.var(axis=1)
+    assert np.max(np.abs((ye * ye).mean(axis=1) - var / (var + eps))) <= 1e-14
+    c = np.full((2, 10), 4.25)
+    assert np.all(oracle.layernorm_rows(c) == 0.0)
+    beta = np.arange(10.0)
+    assert np.array_equal(oracle.layernorm_rows(c, 1e-5, np.full(10, 3.0), beta), np.tile(beta, (2, 1)))
+
+
+def test_layernorm_two_element_closed_form():
+    # [a, b]: mean (a + b)/2, var ((a - b)/2)^2, y = +-d / sqrt(d^2 + eps), d = |a - b| / 2
+    for a, b, eps in ((1.0, 3.0, 1e-5), (-2.5, 4.0, 0.5), (10.0, 10.5, 1e-5)):
+        d = abs(a - b) / 2
+        v = d / math.sqrt(d * d + eps)
+        y = oracle.layernorm_rows(np.array([[a, b]]), eps)[0]
+        assert abs(y[0] - (-v if a < b else v)) <= 4e-16 and abs(y[1] - (v if a < b else -v)) <= 4e-16
+
+
+def test_layernorm_shift_and_scale_invariance():
+    x = RNG.standard_normal((40, 257))
+    y = oracle.layernorm_rows(x, 0.0)
+    assert np.max(np.abs(oracle.layernorm_rows(x + 1000.0, 0.0) - y)) <= 1e-11
+    assert np.max(np.abs(oracle.layernorm_rows(x * 37.0, 0.0) - y)) <= 1e-14
+    # with eps, scaling by a moves the result as sqrt(var / (var + eps / a^2))
+    ya = oracle.layernorm_rows(x * 4.0, 1e-2)
+    assert np.max(np.abs(ya - oracle.layernorm_rows(x, 1e-2 / 16.0))) <= 1e-14
+
+
+def test_layernorm_affine_and_gelu_are_applied_after_normalising():
+    x = RNG.standard_normal((8, 64)) * 3
+    g, b = RNG.standard_normal(64), RNG.standard_normal(64)
+    base = oracle.layernorm_rows(x, 1e-5)
+    assert np.max(np.abs(oracle.layernorm_rows(x, 1e-5, g, b) - (base * g + b))) <= 1e-15 * 8
+    z = base * g + b
+    assert np.max(np.abs(oracle.layernorm_rows(x, 1e-5, g, b, "erf") - oracle.gelu_erf_f64(z))) <= 1e-14
+    assert np.max(np.abs(oracle.layernorm_rows(x, 1e-5, g, b, "tanh") - oracle.gelu_tanh_f64(z))) <= 1e-14
+
+
+def test_layernorm_brute_force_mpmath():
+    mpmath.mp.dps = 50
+    x = RNG.standard_normal((4, 13)) * 3 + 5
+    eps = 1e-5
+    y = oracle.layernorm_rows(x, eps)
+    for r in range(4):
+        v = [mpmath.mpf(float(t)) for t in x[r]]
+        m = mpmath.fsum(v) / len(v)
+        var = mpmath.fsum([(t - m) ** 2 for t in v]) / len(v)
+        rs = 1 / mpmath.sqrt(var + mpmath.mpf(eps))
+        for j in range(13):
+            assert abs(mpmath.mpf(float(y[r, j])) - (v[j] - m) * rs) <= 2e-15
+
+
+def test_layernorm_f32_and_bf16_round_the_double_result_once():
+    x = (RNG.standard_normal((30, 200)) * 3).astype(np.float32)
+    g, b = RNG.standard_normal(200), RNG.standard_normal(200)
+    via = oracle.round_to_f32(oracle.layernorm_rows(x.astype(np.float64), 1e-5, g, b, "tanh"))
+    assert np.array_equal(oracle.layernorm_rows(x, 1e-5, g, b, "tanh").view(np.uint32), via.view(np.uint32))
+    xb = oracle.round_to_bf16(x.astype(np.float64))
+    viab = oracle.round_to_bf16(oracle.layernorm_rows(oracle.bf16_to_f64(xb), 1e-5, g, b))
+    assert np.array_equal(oracle.layernorm_rows(xb, 1e-5, g, b), viab)
+
+
 # ================================================================= rounding
 
 def _all_finite_bf16():
