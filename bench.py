@@ -61,6 +61,14 @@ def kernel_name(w, plan: dict) -> str:
     t = "bf16" if w.dtype == "bf16" else "float"
     if w.op in ("gelu", "gelu_erf"):
         return f"gelu_kernel<{t},{'tanh' if w.op == 'gelu' else 'erf'}>"
+    if w.op.startswith("layernorm"):
+        epi = ",gelu_tanh" if w.op == "layernorm_gelu" else ""
+        vec = 8 if w.dtype == "bf16" else 4
+        if plan["path"] == "warp":
+            return f"layernorm_warp_kernel<{t},vpt={plan['vpt']}{epi}>"
+        if plan["path"] == "cta":
+            return f"layernorm_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{epi}>"
+        return f"layernorm_stream_kernel<{t}{epi}>"
     sc = ",scaled" if w.op == "softmax_causal" else ""
     vec = 8 if w.dtype == "bf16" else 4
     p = plan["path"]
@@ -76,12 +84,19 @@ def kernel_name(w, plan: dict) -> str:
     return f"softmax_twophase_kernel<{t},cluster={plan['cluster']}{sc}>"
 
 
-def launch_workload(fk, w, xp: int, yp: int, shape, stream: int) -> int:
+LN_EPS = 1e-5
+
+
+def launch_workload(fk, w, xp: int, yp: int, shape, stream: int, params=None) -> int:
     """One call of a workload's operator through the C ABI; the status.
     The causal softmax treats every `cols` rows as one block of queries
     against `cols` keys (scale 1: the result equals plain softmax over the
-    same scores with the masked entries at -inf)."""
+    same scores with the masked entries at -inf).  LayerNorm takes
+    `params` = (gamma pointer, beta pointer) and eps 1e-5."""
     code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+    if w.op.startswith("layernorm"):
+        epi = fk.FK_EPILOGUE_GELU_TANH if w.op == "layernorm_gelu" else fk.FK_EPILOGUE_NONE
+        return fk.fk_layernorm_rows(xp, yp, params[0], params[1], shape[0], shape[1], code, LN_EPS, epi, stream)
     if w.op in ("gelu", "gelu_erf"):
         kind = fk.FK_GELU_TANH if w.op == "gelu" else fk.FK_GELU_ERF
         return fk.fk_gelu(xp, yp, shape[0], code, kind, stream)
@@ -251,6 +266,10 @@ def oracle_run(names, inputs, frac, threads):
                 oracle.round_to_bf16(f64(oracle.bf16_to_f64(x), nthreads=threads))
         elif w.op == "softmax_causal":
             oracle.softmax_rows_causal(x, 1.0, x.shape[1], 0, nthreads=threads)
+        elif w.op.startswith("layernorm"):
+            g, b = synth.layernorm_params(x.shape[1], w.seed)
+            oracle.layernorm_rows(x, LN_EPS, g, b, "tanh" if w.op == "layernorm_gelu" else None,
+                                  nthreads=threads)
         elif w.dtype == "f32":
             oracle.softmax_rows_f32(x, nthreads=threads)
         else:
@@ -304,7 +323,7 @@ def run_ours(args) -> dict | None:
     sh = stream.cuda_stream
 
     # device buffers, inputs resident in HBM before the timed region
-    dev_in, dev_out, calls = {}, {}, []
+    dev_in, dev_out, calls, params, keep = {}, {}, [], {}, []
     for n in names:
         w = synth.WORKLOADS[n]
         if w.dtype == "bf16":
@@ -314,7 +333,12 @@ def run_ours(args) -> dict | None:
         dev_in[n] = t.to(device)
         dev_out[n] = torch.empty_like(dev_in[n])
         xp, yp = dev_in[n].data_ptr(), dev_out[n].data_ptr()
-        calls.append((n, lambda w=w, xp=xp, yp=yp, shape=shapes[n]: launch_workload(fk, w, xp, yp, shape, sh)))
+        if w.op.startswith("layernorm"):
+            gb = [torch.from_numpy(a).to(device) for a in synth.layernorm_params(shapes[n][1], w.seed)]
+            keep += gb
+            params[n] = (gb[0].data_ptr(), gb[1].data_ptr())
+        calls.append((n, lambda w=w, xp=xp, yp=yp, shape=shapes[n], pr=params.get(n):
+                      launch_workload(fk, w, xp, yp, shape, sh, pr)))
     bytes_step = sum(workload_bytes(synth.WORKLOADS[n], shapes[n]) for n in names)
     elems_step = sum(host[n].size for n in names)
 
@@ -361,7 +385,7 @@ def run_ours(args) -> dict | None:
     # end to end: pinned host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step)
+        e2e = run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step, params)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -382,9 +406,13 @@ def run_ours(args) -> dict | None:
         ms = kernel_ms[i] / args.steps
         nbytes = workload_bytes(w, shapes[n])
         gbs = nbytes / (ms * 1e-3) / 1e9
-        plan = (fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1],
-                                        fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32).as_dict()
-                if w.op.startswith("softmax") else {"path": "gelu"})
+        code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+        if w.op.startswith("softmax"):
+            plan = fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
+        elif w.op.startswith("layernorm"):
+            plan = fk.fk_layernorm_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
+        else:
+            plan = {"path": "gelu"}
         kernels.append({"workload": n, "kernel": kernel_name(w, plan), "plan": plan,
                         "shape": list(shapes[n]), "ms": round(ms, 5), "GB_s": round(gbs, 1),
                         "elements_per_s": round(host[n].size / (ms * 1e-3), 1),
@@ -423,7 +451,7 @@ def run_ours(args) -> dict | None:
     return line
 
 
-def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step):
+def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step, params=None):
     """Same step through the C ABI from pinned host buffers: every step copies
     all inputs host->device and all outputs device->host inside the timed
     region.  Work is split into row chunks (about --e2e-chunk-mb of input
@@ -469,7 +497,8 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
                 raw_in[n][r0:r0 + cnt].copy_(pin_in[n][r0:r0 + cnt], non_blocking=True)
                 xp = raw_in[n][r0:r0 + cnt].data_ptr()
                 yp = raw_out[n][r0:r0 + cnt].data_ptr()
-                st = launch_workload(fk, w, xp, yp, (cnt,) + tuple(host[n].shape[1:]), s.cuda_stream)
+                st = launch_workload(fk, w, xp, yp, (cnt,) + tuple(host[n].shape[1:]), s.cuda_stream,
+                                     (params or {}).get(n))
                 if st != fk.FK_OK:
                     raise fk.FkError(st, n)
                 pin_out[n][r0:r0 + cnt].copy_(raw_out[n][r0:r0 + cnt], non_blocking=True)
@@ -650,7 +679,7 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
                         "cfg3_softmax, cfg4_softmax, cfg5_softmax, and the operator variants "
-                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal")
+                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal, ln_f32, ln_gelu_bf16")
     p.add_argument("--rows", type=int, default=None,
                    help="profiling only: leading rows (elements for GELU) of each workload")
     p.add_argument("--no-e2e", action="store_true")

@@ -270,6 +270,49 @@ FK_API fk_status fk_softmax_rows_causal_ex(const void *x, void *y, size_t rows, 
                                            float scale, size_t period, size_t offset,
                                            const fk_softmax_plan *plan, void *stream);
 
+/* Epilogues of fk_layernorm_rows. */
+typedef enum fk_epilogue {
+    FK_EPILOGUE_NONE = 0,
+    FK_EPILOGUE_GELU_TANH = 1, /* GELU, tanh form, of the normalised value */
+    FK_EPILOGUE_GELU_ERF = 2   /* GELU, exact form */
+} fk_epilogue;
+
+/*
+ * fk_layernorm_rows -- LayerNorm over each row of a row-major [rows, cols]
+ * matrix, optionally followed by GELU, in one pass over HBM: the
+ * normalisation and activation of the fused LayerNorm -> Linear -> GELU
+ * example (lecture 6, "GPU Kernels and Triton", sections 6.1-6.2, where it
+ * is F.layer_norm over the last axis).
+ *     mean = sum_j x_j / cols,   var = sum_j (x_j - mean)^2 / cols (biased),
+ *     y_j  = epilogue( (x_j - mean) / sqrt(var + eps) * gamma_j + beta_j ).
+ *   x, y    rows*cols elements of `dtype` (FK_F32 or FK_BF16), device
+ *           memory; y == x allowed, other overlap rejected.
+ *   gamma, beta  fp32 device arrays of cols values, or NULL (1 and 0); must
+ *           not overlap y.  16-byte alignment (with 16-byte-multiple rows)
+ *           selects the vector path; any 4-byte alignment works.
+ *   eps     finite, >= 0 (PyTorch's default is 1e-5).
+ *   epilogue  an fk_epilogue.
+ * Arithmetic in fp32 (bf16 widened exactly, rounded to nearest even on
+ * store).  The row is read once and written once up to 32768 columns; longer
+ * rows are read twice.  A row holding a NaN or an infinity gives NaN
+ * throughout; a constant row gives beta (or NaN when eps == 0).
+ * Errors: FK_ERR_INVALID_ARG for bad pointers, overlap, eps < 0 or not
+ * finite, or an unknown epilogue.
+ */
+FK_API fk_status fk_layernorm_rows(const void *x, void *y, const float *gamma, const float *beta, size_t rows,
+                                   size_t cols, int dtype, float eps, int epilogue, void *stream);
+
+/* The plan fk_layernorm_rows would use (host only; path FK_PATH_AUTO or one
+ * to force: FK_PATH_WARP, FK_PATH_CTA or FK_PATH_TWOPHASE). */
+FK_API fk_status fk_layernorm_rows_plan(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan *out);
+
+/* fk_layernorm_rows with an explicit plan: FK_PATH_WARP, FK_PATH_CTA (as for
+ * softmax) or FK_PATH_TWOPHASE (one 512-thread block per row, streamed
+ * twice); NULL or FK_PATH_AUTO = the automatic choice. */
+FK_API fk_status fk_layernorm_rows_ex(const void *x, void *y, const float *gamma, const float *beta,
+                                      size_t rows, size_t cols, int dtype, float eps, int epilogue,
+                                      const fk_softmax_plan *plan, void *stream);
+
 /*
  * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a
  * cluster exchange their partial (max, sum) through mbarriers; every such

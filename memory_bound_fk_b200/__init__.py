@@ -15,6 +15,9 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
     fk_softmax_rows_ws(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, stream) -> status
     fk_softmax_rows_causal(x, y, rows, cols, dtype, scale, period, offset, stream) -> status
     fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, plan, stream) -> status
+    fk_layernorm_rows(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, stream) -> status
+    fk_layernorm_rows_ex(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, plan, stream) -> status
+    fk_layernorm_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
     fk_status_string(status) -> str
     fk_wait_timeouts(reset=False) -> int     (bounded-wait give-ups, synchronous)
     fk_wait_selftest(timeout_us, stream) -> status
@@ -24,6 +27,7 @@ Tensor conveniences (contiguous CUDA tensors; the current torch stream):
     gelu(x, out=None, approximate="tanh")   # fp32 / bf16; "tanh" or "none" (exact)
     softmax_rows(x, out=None, plan=None)    # softmax over the last dimension
     softmax_causal(x, scale, period=None, offset=0, out=None, plan=None)
+    layernorm(x, eps=1e-5, weight=None, bias=None, gelu=None, out=None, plan=None)
 
 There is no fallback: if the library is missing or a call fails, an
 exception is raised.
@@ -50,6 +54,10 @@ FK_BF16 = 1
 # fk_gelu_kind
 FK_GELU_TANH = 0
 FK_GELU_ERF = 1
+# fk_epilogue
+FK_EPILOGUE_NONE = 0
+FK_EPILOGUE_GELU_TANH = 1
+FK_EPILOGUE_GELU_ERF = 2
 # fk_softmax_path
 FK_PATH_AUTO = 0
 FK_PATH_WARP = 1
@@ -118,6 +126,13 @@ def lib() -> ctypes.CDLL:
         L.fk_softmax_rows_causal_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz,
                                                 ctypes.POINTER(SoftmaxPlan), vp]
         L.fk_softmax_rows_causal_ex.restype = ci
+        L.fk_layernorm_rows.argtypes = [vp, vp, vp, vp, sz, sz, ci, ctypes.c_float, ci, vp]
+        L.fk_layernorm_rows.restype = ci
+        L.fk_layernorm_rows_ex.argtypes = [vp, vp, vp, vp, sz, sz, ci, ctypes.c_float, ci,
+                                           ctypes.POINTER(SoftmaxPlan), vp]
+        L.fk_layernorm_rows_ex.restype = ci
+        L.fk_layernorm_rows_plan.argtypes = [sz, sz, ci, ci, ctypes.POINTER(SoftmaxPlan)]
+        L.fk_layernorm_rows_plan.restype = ci
         L.fk_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
         L.fk_wait_timeouts.restype = ci
         L.fk_wait_selftest.argtypes = [ctypes.c_uint, vp]
@@ -185,6 +200,25 @@ def fk_softmax_rows_causal_ex(x: int, y: int, rows: int, cols: int, dtype: int, 
                               offset: int, plan: SoftmaxPlan | None, stream: int = 0) -> int:
     return lib().fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset,
                                            ctypes.byref(plan) if plan is not None else None, stream)
+
+
+def fk_layernorm_rows(x: int, y: int, gamma: int, beta: int, rows: int, cols: int, dtype: int, eps: float,
+                      epilogue: int = FK_EPILOGUE_NONE, stream: int = 0) -> int:
+    return lib().fk_layernorm_rows(x, y, gamma or None, beta or None, rows, cols, dtype, eps, epilogue, stream)
+
+
+def fk_layernorm_rows_ex(x: int, y: int, gamma: int, beta: int, rows: int, cols: int, dtype: int, eps: float,
+                         epilogue: int, plan: SoftmaxPlan | None, stream: int = 0) -> int:
+    return lib().fk_layernorm_rows_ex(x, y, gamma or None, beta or None, rows, cols, dtype, eps, epilogue,
+                                      ctypes.byref(plan) if plan is not None else None, stream)
+
+
+def fk_layernorm_rows_plan(rows: int, cols: int, dtype: int, path: int = FK_PATH_AUTO) -> SoftmaxPlan:
+    p = SoftmaxPlan()
+    st = lib().fk_layernorm_rows_plan(rows, cols, dtype, path, ctypes.byref(p))
+    if st != FK_OK:
+        raise FkError(st, "fk_layernorm_rows_plan")
+    return p
 
 
 def fk_status_string(status: int) -> str:
@@ -344,6 +378,44 @@ def softmax_causal(x, scale: float, period: int | None = None, offset: int = 0, 
     return out
 
 
+_EPILOGUES = {None: FK_EPILOGUE_NONE, "tanh": FK_EPILOGUE_GELU_TANH, "none": FK_EPILOGUE_GELU_ERF,
+              "erf": FK_EPILOGUE_GELU_ERF}
+
+
+def layernorm(x, eps: float = 1e-5, weight=None, bias=None, gelu: str | None = None, out=None,
+              plan: SoftmaxPlan | None = None):
+    """LayerNorm over the last dimension of a contiguous fp32/bf16 CUDA
+    tensor (as F.layer_norm(x, x.shape[-1:], weight, bias, eps)), then GELU
+    when `gelu` is "tanh" or "erf" (or torch's "none", the exact form).
+    weight / bias: contiguous fp32 CUDA tensors of x.shape[-1] values."""
+    import torch
+    _check_tensor(x, "x")
+    code = _dtype_code(x.dtype)
+    if gelu not in _EPILOGUES:
+        raise ValueError("gelu must be None, 'tanh' or 'erf'")
+    cols = x.shape[-1] if x.dim() > 0 else 1
+    rows = x.numel() // cols if cols else 0
+    ptrs = []
+    for name, p in (("weight", weight), ("bias", bias)):
+        if p is None:
+            ptrs.append(0)
+            continue
+        _check_tensor(p, name)
+        if p.dtype != torch.float32 or p.numel() != cols or p.device != x.device:
+            raise ValueError(f"{name} must be float32 with x.shape[-1] values on x's device")
+        ptrs.append(p.data_ptr())
+    if out is None:
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.dtype != x.dtype or out.shape != x.shape or out.device != x.device:
+        raise ValueError("out must match x in dtype, shape and device")
+    st = fk_layernorm_rows_ex(x.data_ptr(), out.data_ptr(), ptrs[0], ptrs[1], rows, cols, code, eps,
+                              _EPILOGUES[gelu], plan, _stream_handle(x))
+    if st != FK_OK:
+        raise FkError(st, "fk_layernorm_rows")
+    return out
+
+
 __all__ = [
     "FK_OK", "FK_ERR_INVALID_ARG", "FK_ERR_UNSUPPORTED_DTYPE", "FK_ERR_UNSUPPORTED_DEVICE",
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_GELU_TANH", "FK_GELU_ERF", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
@@ -351,6 +423,8 @@ __all__ = [
     "fk_gelu_tanh", "fk_gelu", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
     "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
     "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal",
+    "fk_layernorm_rows", "fk_layernorm_rows_ex", "fk_layernorm_rows_plan", "layernorm", "FK_EPILOGUE_NONE", "FK_EPILOGUE_GELU_TANH",
+    "FK_EPILOGUE_GELU_ERF",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
     "fk_wait_selftest", "make_plan", "gelu_tanh", "gelu",
     "softmax_rows",

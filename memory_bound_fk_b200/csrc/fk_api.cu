@@ -278,6 +278,54 @@ fk_status fk_softmax_rows_causal_ex(const void* x, void* y, size_t rows, size_t 
   return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, &sc, stream);
 }
 
+fk_status fk_layernorm_rows_ex(const void* x, void* y, const float* gamma, const float* beta, size_t rows,
+                               size_t cols, int dtype, float eps, int epilogue, const fk_softmax_plan* plan,
+                               void* stream) {
+  if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
+  if (!(eps >= 0.0f) || !(eps <= FLT_MAX)) return FK_ERR_INVALID_ARG;
+  if (epilogue != FK_EPILOGUE_NONE && epilogue != FK_EPILOGUE_GELU_TANH && epilogue != FK_EPILOGUE_GELU_ERF)
+    return FK_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return FK_OK;
+  if (rows > SIZE_MAX / cols) return FK_ERR_INVALID_ARG;
+  fk_softmax_plan p;
+  fk_status st = (plan == nullptr || plan->path == FK_PATH_AUTO)
+                     ? fk::plan_layernorm(rows, cols, dtype, FK_PATH_AUTO, &p)
+                     : fk::check_layernorm_plan(rows, cols, dtype, *plan, &p);
+  if (st != FK_OK) return st;
+  const size_t esize = dtype == FK_F32 ? 4 : 2;
+  const fk::DeviceInfo* dev = nullptr;
+  st = fk::check_call(x, y, rows * cols, esize, &dev);
+  if (st != FK_OK) return st;
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return FK_ERR_UNSUPPORTED_DEVICE;
+  const size_t pbytes = cols * sizeof(float);
+  const uintptr_t yb = reinterpret_cast<uintptr_t>(y);
+  const size_t ybytes = rows * cols * esize;
+  for (const float* q : {gamma, beta}) {
+    if (q == nullptr) continue;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(q);
+    if (a % sizeof(float) != 0 || a > UINTPTR_MAX - pbytes) return FK_ERR_INVALID_ARG;
+    if (a < yb + ybytes && yb < a + pbytes) return FK_ERR_INVALID_ARG;  // the output would overwrite it
+    st = fk::check_pointer(q, pbytes, d);
+    if (st != FK_OK) return st;
+  }
+  const bool aligned = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (yb % 16 == 0) &&
+                       ((cols * esize) % 16 == 0) && (reinterpret_cast<uintptr_t>(gamma) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(beta) % 16 == 0);
+  const cudaError_t e = fk::launch_layernorm(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, p, aligned,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_layernorm_rows_plan(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out) {
+  return fk::plan_layernorm(rows, cols, dtype, path, out);
+}
+
+fk_status fk_layernorm_rows(const void* x, void* y, const float* gamma, const float* beta, size_t rows,
+                            size_t cols, int dtype, float eps, int epilogue, void* stream) {
+  return fk_layernorm_rows_ex(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, nullptr, stream);
+}
+
 fk_status fk_softmax_rows_causal(const void* x, void* y, size_t rows, size_t cols, int dtype, float scale,
                                  size_t period, size_t offset, void* stream) {
   return fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, nullptr, stream);

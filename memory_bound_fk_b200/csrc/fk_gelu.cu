@@ -20,6 +20,7 @@
 // Errors stay within a few ulp of y: under 1e-6 absolute on [-20, 20] for
 // fp32 (bound 2e-6), and within 1 ulp of the correctly rounded value for bf16.
 #include "fk_common.cuh"
+#include "fk_gelu.cuh"
 #include "fk_internal.h"
 
 namespace fk {
@@ -33,34 +34,6 @@ namespace {
 constexpr int kGeluThreads = 256;
 constexpr int kGeluUnroll = 2;
 constexpr size_t kGeluMaxGrid = 0x7fffffffu;
-
-// -2 sqrt(2/pi) log2(e) and that times 0.044715, rounded once to fp32.
-constexpr float kA = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736);
-constexpr float kB = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736 * 0.044715);
-constexpr float kRsqrt2 = 0.70710678118654752440f;
-
-template <typename T>
-__device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float a = x * fmaf(kB, x * x, kA);  // -2u log2(e): <= 0 for x >= 0
-  const float t = Elem<T>::exp2(-fabsf(a)); // exp(-2|u|) in (0, 1]
-  const float r = rcp_approx(1.0f + t);
-  const float y = (a > 0.0f) ? x * t * r : x * r;
-  return (x == -INFINITY) ? -0.0f : y;
-}
-
-// h = P(Z > |x|) = 0.5 erfc(|x| / sqrt 2) keeps its relative accuracy when
-// tiny, so Phi(x) = 1 - h (x >= 0) or h (x < 0) is accurate to a rounding of
-// Phi and y = x Phi(x) to about one ulp of y over the whole range.
-__device__ __forceinline__ float gelu_erf_f(float x) {
-  const float h = 0.5f * erfcf(fabsf(x) * kRsqrt2);
-  const float y = x * ((x >= 0.0f) ? 1.0f - h : h);
-  return (x == -INFINITY) ? -0.0f : y;
-}
-
-template <typename T, int KIND>
-__device__ __forceinline__ float gelu_f(float x) {
-  return KIND == FK_GELU_TANH ? gelu_tanh_f<T>(x) : gelu_erf_f(x);
-}
 
 template <typename T, int KIND>
 __device__ __forceinline__ uint4 gelu_vec(uint4 v) {

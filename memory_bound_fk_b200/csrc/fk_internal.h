@@ -86,6 +86,22 @@ cudaError_t launch_softmax(const void* x, void* y, size_t rows, size_t cols, int
                            const fk_softmax_plan& plan, bool aligned, void* ws, const SoftmaxScaling* sc,
                            const DeviceInfo& dev, cudaStream_t stream);
 
+// ---- LayerNorm -----------------------------------------------------------
+// Plan of fk_layernorm_rows: FK_PATH_WARP (cols <= 1024 fp32 / 2048 bf16 on
+// demand), FK_PATH_CTA (<= 32768) or FK_PATH_TWOPHASE (any length: one
+// 512-thread block per row streams it twice).  `path` = FK_PATH_AUTO or one
+// of those; a caller plan is validated by check_layernorm_plan.
+fk_status plan_layernorm(size_t rows, size_t cols, int dtype, int path, fk_softmax_plan* out);
+fk_status check_layernorm_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan& in,
+                               fk_softmax_plan* out);
+
+// Launch a validated LayerNorm plan (gamma / beta: fp32 device arrays of
+// cols values, or nullptr; `aligned`: x, y, gamma and beta allow 16-byte
+// vector access along rows).
+cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, size_t rows,
+                             size_t cols, int dtype, float eps, int epilogue, const fk_softmax_plan& plan,
+                             bool aligned, cudaStream_t stream);
+
 // Workspace bytes a validated plan needs (0 except on the split path).
 size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan);
 

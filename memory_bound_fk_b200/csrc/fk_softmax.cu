@@ -54,6 +54,7 @@
 
 #include "fk_common.cuh"
 #include "fk_internal.h"
+#include "fk_rows.cuh"
 #include "fk_sync.cuh"
 
 namespace fk {
@@ -82,11 +83,6 @@ __device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, u
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
                                              uint64_t timeout_ns = kWaitTimeoutNs) {
   return mbar_try_wait(bar, parity) || bounded_wait_slow(bar, parity, timeout_ns);
-}
-
-template <typename I>
-__device__ __forceinline__ I imin(I a, I b) {
-  return a < b ? a : b;
 }
 
 // ---------------------------------------------------------------- merge rule
@@ -123,66 +119,6 @@ __device__ __forceinline__ size_t row_limit(const SoftmaxScaling& sc, size_t row
 }
 
 // ---------------------------------------------------------------- row I/O
-
-// Load VPT chunks of a team slice as raw 16-byte words (VPT * VEC values).
-// Vectors [vfirst, ve) of the row are the slice; anything outside is -inf.
-// MASK: elements at or after `lim` are -inf too and are not loaded.
-// The scalar (unaligned) path packs its scalar loads into the same layout.
-template <typename T, int VPT, int TEAM, bool ALIGNED, bool MASK, typename Idx>
-__device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Idx cols, Idx lim, int t,
-                                            uint4* raw) {
-  constexpr int VEC = Elem<T>::VEC;
-#pragma unroll
-  for (int c = 0; c < VPT; ++c) {
-    if constexpr (ALIGNED) {
-      const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      const Idx e = vi * VEC;
-      const bool live = MASK ? (vi < ve && e < lim) : (vi < ve);
-      raw[c] = ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, live, Elem<T>::kNegInfWord);
-      // vectors wholly past lim were not loaded (all -inf); only the one
-      // that straddles lim needs its tail masked
-      if constexpr (MASK) {
-        if (e < lim && lim - e < static_cast<Idx>(VEC)) raw[c] = Elem<T>::keep_first(raw[c], static_cast<int>(lim - e));
-      }
-    } else {
-      const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
-      Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
-      if constexpr (MASK) eend = imin(eend, lim);
-      float f[VEC];
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) {
-        const Idx e = e0 + static_cast<Idx>(k) * TEAM;
-        f[k] = (e < eend) ? Elem<T>::load1(row + e) : -INFINITY;
-      }
-      raw[c] = Elem<T>::pack(f);  // exact: the values are already of type T
-    }
-  }
-}
-
-// Store v * scale for the same placement as load_chunks.
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
-__device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx cols, int t,
-                                             const float* v, float scale) {
-  constexpr int VEC = Elem<T>::VEC;
-#pragma unroll
-  for (int c = 0; c < VPT; ++c) {
-    float o[VEC];
-#pragma unroll
-    for (int k = 0; k < VEC; ++k) o[k] = v[c * VEC + k] * scale;
-    if constexpr (ALIGNED) {
-      const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      st_stream_v4_if(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(o), vi < ve);
-    } else {
-      const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
-      const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) {
-        const Idx e = e0 + static_cast<Idx>(k) * TEAM;
-        if (e < eend) Elem<T>::store1(row + e, o[k]);
-      }
-    }
-  }
-}
 
 // Exponentials relative to ref, into v; returns their sum (four
 // accumulators).  fp32 works in place on v (already unpacked at load); bf16
@@ -232,18 +168,6 @@ template <typename T, int VPT>
 __device__ __forceinline__ float exp_sum_row(const uint4* raw, float* v, float m, float k) {
   if (fabsf(m * k) < 0x1p24f) return exp_sum<T, VPT, true>(raw, v, m, k);
   return exp_sum<T, VPT, false>(raw, v, exp_ref(m), k);
-}
-
-// Row loads: raw 16-byte words; fp32 rows are unpacked into v at once (the
-// same bits), bf16 rows stay packed until exp_sum.
-template <typename T, int VPT, int TEAM, bool ALIGNED, bool MASK, typename Idx>
-__device__ __forceinline__ void load_row(const T* row, Idx vfirst, Idx ve, Idx cols, Idx lim, int t,
-                                         uint4* raw, float* v) {
-  load_chunks<T, VPT, TEAM, ALIGNED, MASK, Idx>(row, vfirst, ve, cols, lim, t, raw);
-  if constexpr (sizeof(T) == 4) {
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) Elem<T>::unpack(raw[i], v + i * Elem<T>::VEC);
-  }
 }
 
 // Max of the values a thread holds (after load_row).

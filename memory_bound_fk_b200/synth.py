@@ -105,6 +105,12 @@ WORKLOADS = {
                  "the gelu_bf16 values, exact GELU x*Phi(x)"),
         Workload("cfg4_causal", "softmax_causal", "bf16", (32 * 16 * 2048, 2048), 3,
                  "the cfg4_softmax scores, causal mask generated in the kernel (masked entries not read)"),
+        # LayerNorm over transformer-shaped activations (hidden size 4096)
+        Workload("ln_f32", "layernorm", "f32", (16384, 4096), 6,
+                 "fp32 16384x4096, row r ~ N(mu_r, s_r^2), mu_r ~ U[-2,2], s_r ~ U[0.5,2]; "
+                 "gamma ~ 1+N(0,0.1^2), beta ~ N(0,0.1^2); eps 1e-5"),
+        Workload("ln_gelu_bf16", "layernorm_gelu", "bf16", (65536, 4096), 7,
+                 "bf16 65536x4096, same recipe, then tanh-GELU"),
     ]
 }
 
@@ -277,6 +283,10 @@ def make(name: str, threads: int | None = None, rows: int | None = None) -> np.n
         return _cfg2()[:rows]
     if name in ("gelu_bf16", "gelu_erf_bf16"):
         return f32_to_bf16_bits(_cfg2(16777216, seed=5))[:rows]
+    if name in ("ln_f32", "ln_gelu_bf16"):
+        w = WORKLOADS[name]
+        r = rows or w.shape[0]
+        return layernorm_input(r, w.shape[1], w.dtype, w.seed, threads=threads)
     if name == "cfg5_softmax":
         r = rows or 512
         return _cfg5(rows=-(-r // CFG5_ROWS_PER_CHUNK) * CFG5_ROWS_PER_CHUNK, threads=threads)[:r]
@@ -319,3 +329,39 @@ def softmax_input(rows: int, cols: int, dtype: str = "f32", sigma: float = 4.0,
     b = f32_to_bf16_bits(np.where(np.isneginf(x), 0.0, x))
     b[np.isneginf(x)] = NEG_INF_BF16
     return b
+
+
+# ------------------------------------------------------------------ LayerNorm
+
+LN_ROWS_PER_CHUNK = 256
+
+
+def _ln_chunk(out: np.ndarray, chunk: int, seed: int) -> None:
+    rows, cols = out.shape
+    g = chunk_rng(seed, chunk)
+    mu = g.uniform(-2.0, 2.0, size=(rows, 1)).astype(np.float32)
+    sd = g.uniform(0.5, 2.0, size=(rows, 1)).astype(np.float32)
+    g.standard_normal(out=out, dtype=np.float32)
+    out *= sd
+    out += mu
+
+
+def layernorm_input(rows: int, cols: int, dtype: str = "f32", seed: int = 6, threads=None) -> np.ndarray:
+    """LayerNorm activations: row r is N(mu_r, s_r^2) with mu_r ~ U[-2, 2]
+    and s_r ~ U[0.5, 2], generated in chunks of 256 rows (fp32, or bf16
+    bits)."""
+    nchunks = -(-rows // LN_ROWS_PER_CHUNK)
+    x = np.empty((nchunks * LN_ROWS_PER_CHUNK, cols), np.float32)
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(lambda c: _ln_chunk(x[c * LN_ROWS_PER_CHUNK:(c + 1) * LN_ROWS_PER_CHUNK], c, seed),
+                    range(nchunks)))
+    x = x[:rows]
+    return x if dtype == "f32" else f32_to_bf16_bits(x)
+
+
+def layernorm_params(cols: int, seed: int = 6) -> tuple[np.ndarray, np.ndarray]:
+    """gamma ~ 1 + N(0, 0.1^2) and beta ~ N(0, 0.1^2), fp32."""
+    g = chunk_rng(seed, 1 << 30)
+    gamma = (1.0 + 0.1 * g.standard_normal(cols)).astype(np.float32)
+    beta = (0.1 * g.standard_normal(cols)).astype(np.float32)
+    return gamma, beta
