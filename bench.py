@@ -69,7 +69,7 @@ def kernel_name(w, plan: dict) -> str:
         if plan["path"] == "cta":
             return f"layernorm_block_kernel<{t},{plan['threads']},ept={plan['vpt'] * vec}{epi}>"
         return f"layernorm_stream_kernel<{t}{epi}>"
-    sc = ",scaled" if w.op == "softmax_causal" else ""
+    sc = ",scaled" if w.op.startswith("softmax_causal") else ""
     vec = 8 if w.dtype == "bf16" else 4
     p = plan["path"]
     if p == "warp":
@@ -103,6 +103,9 @@ def launch_workload(fk, w, xp: int, yp: int, shape, stream: int, params=None) ->
     rows, cols = shape
     if w.op == "softmax_causal":
         return fk.fk_softmax_rows_causal(xp, yp, rows, cols, code, 1.0, cols, 0, stream)
+    if w.op == "softmax_causal_skip":
+        return fk.fk_softmax_rows_causal_ex(xp, yp, rows, cols, code, 1.0, cols, 0, None, stream,
+                                            fk.FK_SOFTMAX_SKIP_MASKED)
     return fk.fk_softmax_rows(xp, yp, rows, cols, code, stream)
 
 
@@ -264,7 +267,7 @@ def oracle_run(names, inputs, frac, threads):
                 oracle.round_to_f32(f64(x.astype(np.float64), nthreads=threads))
             else:
                 oracle.round_to_bf16(f64(oracle.bf16_to_f64(x), nthreads=threads))
-        elif w.op == "softmax_causal":
+        elif w.op.startswith("softmax_causal"):
             oracle.softmax_rows_causal(x, 1.0, x.shape[1], 0, nthreads=threads)
         elif w.op.startswith("layernorm"):
             g, b = synth.layernorm_params(x.shape[1], w.seed)
@@ -481,7 +484,7 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
         per = max(1, chunk_bytes // row_bytes)
         if a.ndim == 1:
             per = max(8, per // 8 * 8)  # keep 16-byte chunk boundaries
-        elif synth.WORKLOADS[n].op == "softmax_causal":
+        elif synth.WORKLOADS[n].op.startswith("softmax_causal"):
             per = max(1, per // a.shape[1]) * a.shape[1]  # whole query blocks per chunk
         for r0 in range(0, a.shape[0], per):
             chunks.append((n, r0, min(per, a.shape[0] - r0)))
@@ -679,7 +682,7 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
                         "cfg3_softmax, cfg4_softmax, cfg5_softmax, and the operator variants "
-                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal, ln_f32, ln_gelu_bf16")
+                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal, cfg4_causal_skip, ln_f32, ln_gelu_bf16")
     p.add_argument("--rows", type=int, default=None,
                    help="profiling only: leading rows (elements for GELU) of each workload")
     p.add_argument("--no-e2e", action="store_true")

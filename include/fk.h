@@ -265,9 +265,17 @@ FK_API fk_status fk_softmax_rows_noalloc(const void *x, void *y, size_t rows, si
 FK_API fk_status fk_softmax_rows_causal(const void *x, void *y, size_t rows, size_t cols, int dtype, float scale,
                                         size_t period, size_t offset, void *stream);
 
-/* fk_softmax_rows_causal with an explicit plan, as fk_softmax_rows_ex. */
+/* Flags of fk_softmax_rows_causal_ex. */
+#define FK_SOFTMAX_SKIP_MASKED 1u /* do not store masked outputs: each masked output is then
+                                     either left as it was or set to 0 (0 where it shares a
+                                     16-byte vector with a kept output).  For consumers that
+                                     never read the masked region: the output's write traffic
+                                     halves along with the reads. */
+
+/* fk_softmax_rows_causal with flags (0 or FK_SOFTMAX_SKIP_MASKED; other
+ * bits -> FK_ERR_INVALID_ARG) and an explicit plan, as fk_softmax_rows_ex. */
 FK_API fk_status fk_softmax_rows_causal_ex(const void *x, void *y, size_t rows, size_t cols, int dtype,
-                                           float scale, size_t period, size_t offset,
+                                           float scale, size_t period, size_t offset, unsigned int flags,
                                            const fk_softmax_plan *plan, void *stream);
 
 /* Epilogues of fk_layernorm_rows. */

@@ -14,7 +14,7 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
     fk_softmax_rows_workspace(rows, cols, dtype, plan=None) -> bytes
     fk_softmax_rows_ws(x, y, rows, cols, dtype, plan, workspace, workspace_bytes, stream) -> status
     fk_softmax_rows_causal(x, y, rows, cols, dtype, scale, period, offset, stream) -> status
-    fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, plan, stream) -> status
+    fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, flags, plan, stream) -> status
     fk_layernorm_rows(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, stream) -> status
     fk_layernorm_rows_ex(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, plan, stream) -> status
     fk_layernorm_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
@@ -54,6 +54,8 @@ FK_BF16 = 1
 # fk_gelu_kind
 FK_GELU_TANH = 0
 FK_GELU_ERF = 1
+# fk_softmax_rows_causal_ex flags
+FK_SOFTMAX_SKIP_MASKED = 1
 # fk_epilogue
 FK_EPILOGUE_NONE = 0
 FK_EPILOGUE_GELU_TANH = 1
@@ -123,7 +125,7 @@ def lib() -> ctypes.CDLL:
         L.fk_softmax_rows_ws.restype = ci
         L.fk_softmax_rows_causal.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz, vp]
         L.fk_softmax_rows_causal.restype = ci
-        L.fk_softmax_rows_causal_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz,
+        L.fk_softmax_rows_causal_ex.argtypes = [vp, vp, sz, sz, ci, ctypes.c_float, sz, sz, ctypes.c_uint,
                                                 ctypes.POINTER(SoftmaxPlan), vp]
         L.fk_softmax_rows_causal_ex.restype = ci
         L.fk_layernorm_rows.argtypes = [vp, vp, vp, vp, sz, sz, ci, ctypes.c_float, ci, vp]
@@ -197,8 +199,8 @@ def fk_softmax_rows_causal(x: int, y: int, rows: int, cols: int, dtype: int, sca
 
 
 def fk_softmax_rows_causal_ex(x: int, y: int, rows: int, cols: int, dtype: int, scale: float, period: int,
-                              offset: int, plan: SoftmaxPlan | None, stream: int = 0) -> int:
-    return lib().fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset,
+                              offset: int, plan: SoftmaxPlan | None, stream: int = 0, flags: int = 0) -> int:
+    return lib().fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, flags,
                                            ctypes.byref(plan) if plan is not None else None, stream)
 
 
@@ -353,11 +355,12 @@ def softmax_rows(x, out=None, plan: SoftmaxPlan | None = None, workspace=None):
 
 
 def softmax_causal(x, scale: float, period: int | None = None, offset: int = 0, out=None,
-                   plan: SoftmaxPlan | None = None):
+                   plan: SoftmaxPlan | None = None, skip_masked: bool = False):
     """Scaled, causally masked softmax over the last dimension of a
     contiguous fp32/bf16 CUDA tensor of attention scores [..., T_q, T_k]: row
     i of each [T_q, T_k] block keeps keys j <= i + offset.  `period` defaults
-    to T_q (x.shape[-2]); 0 means no mask."""
+    to T_q (x.shape[-2]); 0 means no mask.  skip_masked: masked outputs are
+    not stored (left as they were, or 0)."""
     import torch
     _check_tensor(x, "x")
     code = _dtype_code(x.dtype)
@@ -372,7 +375,7 @@ def softmax_causal(x, scale: float, period: int | None = None, offset: int = 0, 
     rows = x.numel() // cols if cols else 0
     p = x.shape[-2] if period is None else period
     st = fk_softmax_rows_causal_ex(x.data_ptr(), out.data_ptr(), rows, cols, code, scale, p, offset, plan,
-                                   _stream_handle(x))
+                                   _stream_handle(x), FK_SOFTMAX_SKIP_MASKED if skip_masked else 0)
     if st != FK_OK:
         raise FkError(st, "fk_softmax_rows_causal")
     return out
@@ -422,7 +425,7 @@ __all__ = [
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
     "fk_gelu_tanh", "fk_gelu", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
     "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
-    "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal",
+    "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal", "FK_SOFTMAX_SKIP_MASKED",
     "fk_layernorm_rows", "fk_layernorm_rows_ex", "fk_layernorm_rows_plan", "layernorm", "FK_EPILOGUE_NONE", "FK_EPILOGUE_GELU_TANH",
     "FK_EPILOGUE_GELU_ERF",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",

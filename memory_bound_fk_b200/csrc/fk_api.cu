@@ -265,8 +265,10 @@ fk_status fk_softmax_rows_ws(const void* x, void* y, size_t rows, size_t cols, i
 }
 
 fk_status fk_softmax_rows_causal_ex(const void* x, void* y, size_t rows, size_t cols, int dtype, float scale,
-                                    size_t period, size_t offset, const fk_softmax_plan* plan, void* stream) {
+                                    size_t period, size_t offset, unsigned int flags, const fk_softmax_plan* plan,
+                                    void* stream) {
   if (!(scale > 0.0f) || !(scale <= FLT_MAX)) return FK_ERR_INVALID_ARG;  // also rejects NaN
+  if ((flags & ~FK_SOFTMAX_SKIP_MASKED) != 0) return FK_ERR_INVALID_ARG;
   fk::SoftmaxScaling sc;
   sc.k = static_cast<float>(static_cast<double>(scale) * 1.44269504088896340736);
   // (r mod period) + offset: a period beyond the rows and an offset beyond
@@ -274,6 +276,7 @@ fk_status fk_softmax_rows_causal_ex(const void* x, void* y, size_t rows, size_t 
   sc.period = period < rows ? period : rows;
   sc.offset = offset < cols ? offset : cols;
   sc.row0 = 0;
+  sc.skip_masked = (flags & FK_SOFTMAX_SKIP_MASKED) ? 1 : 0;
   fk::set_period_division(&sc, rows);
   return softmax_call(x, y, rows, cols, dtype, plan, nullptr, 0, true, &sc, stream);
 }
@@ -328,7 +331,7 @@ fk_status fk_layernorm_rows(const void* x, void* y, const float* gamma, const fl
 
 fk_status fk_softmax_rows_causal(const void* x, void* y, size_t rows, size_t cols, int dtype, float scale,
                                  size_t period, size_t offset, void* stream) {
-  return fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, nullptr, stream);
+  return fk_softmax_rows_causal_ex(x, y, rows, cols, dtype, scale, period, offset, 0, nullptr, stream);
 }
 
 fk_status fk_softmax_rows_workspace(size_t rows, size_t cols, int dtype, const fk_softmax_plan* plan,

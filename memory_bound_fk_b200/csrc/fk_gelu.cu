@@ -14,8 +14,9 @@
 // subnormal for bf16 outputs, whose smallest value is 2^-133); x = -inf is
 // mapped to the limit -0.
 //
-// Exact form: x Phi(x), Phi the standard normal distribution function, from
-// CUDA's erfcf of |x| / sqrt(2).
+// Exact form: x Phi(x), Phi the standard normal distribution function, with
+// erfc in the form of Press et al. and coefficients fitted here (see
+// fk_gelu.cuh).
 //
 // Errors stay within a few ulp of y: under 1e-6 absolute on [-20, 20] for
 // fp32 (bound 2e-6), and within 1 ulp of the correctly rounded value for bf16.

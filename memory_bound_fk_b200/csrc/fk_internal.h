@@ -60,7 +60,8 @@ fk_status check_plan(size_t rows, size_t cols, int dtype, const fk_softmax_plan&
 // start of the whole call) keeps columns j < limit(r), limit(r) =
 // min(cols, (r mod period) + offset + 1), or every column when period == 0,
 // and computes softmax(scale * x_j) over them; the other columns are not
-// read and are written 0.
+// read and are written 0 (or, with skip_masked, not written where a whole
+// 16-byte vector is masked).
 struct SoftmaxScaling {
   float k;        // scale * log2(e), rounded once to fp32
   size_t period;  // 0: no mask; otherwise 1 <= period <= rows
@@ -72,6 +73,7 @@ struct SoftmaxScaling {
   // when fast32 is set (period and every row index below 2^32).
   uint32_t magic, shift1, shift2;
   int fast32;
+  int skip_masked;  // 1: masked columns are not stored (FK_SOFTMAX_SKIP_MASKED)
 };
 
 // Fill the division fields of `sc` for its period and the call's rows.

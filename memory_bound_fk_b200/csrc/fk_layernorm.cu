@@ -147,7 +147,7 @@ __device__ __forceinline__ float epilogue(float z) {
   if constexpr (EPI == FK_EPILOGUE_GELU_TANH) {
     return gelu_tanh_f<float>(z);
   } else if constexpr (EPI == FK_EPILOGUE_GELU_ERF) {
-    return gelu_erf_f(z);
+    return gelu_erf_f<float>(z);
   } else {
     return z;
   }

@@ -60,8 +60,10 @@ __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Id
 // Store, for the same placement as load_chunks, the values that
 // fn(c, o) writes into o[0..VEC) for chunk c (fn is called once per chunk,
 // in order, so callers can produce each chunk just before it is stored).
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx, typename Fn>
-__device__ __forceinline__ void store_chunks_fn(T* row, Idx vfirst, Idx ve, Idx cols, int t, Fn fn) {
+// WLIM: vectors (aligned path) or elements (scalar path) at or after wlim
+// are not stored.
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx, bool WLIM = false, typename Fn>
+__device__ __forceinline__ void store_chunks_fn(T* row, Idx vfirst, Idx ve, Idx cols, int t, Fn fn, Idx wlim = 0) {
   constexpr int VEC = Elem<T>::VEC;
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
@@ -69,10 +71,12 @@ __device__ __forceinline__ void store_chunks_fn(T* row, Idx vfirst, Idx ve, Idx 
     fn(c, o);
     if constexpr (ALIGNED) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      st_stream_v4_if(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(o), vi < ve);
+      const bool st = WLIM ? (vi < ve && vi * VEC < wlim) : (vi < ve);
+      st_stream_v4_if(row + static_cast<size_t>(vi) * VEC, Elem<T>::pack(o), st);
     } else {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
-      const Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+      Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
+      if constexpr (WLIM) eend = eend < wlim ? eend : wlim;
 #pragma unroll
       for (int k = 0; k < VEC; ++k) {
         const Idx e = e0 + static_cast<Idx>(k) * TEAM;
@@ -82,15 +86,18 @@ __device__ __forceinline__ void store_chunks_fn(T* row, Idx vfirst, Idx ve, Idx 
   }
 }
 
-// Store v * scale for the same placement as load_chunks.
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+// Store v * scale for the same placement as load_chunks (WLIM: as above).
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx, bool WLIM = false>
 __device__ __forceinline__ void store_chunks(T* row, Idx vfirst, Idx ve, Idx cols, int t, const float* v,
-                                             float scale) {
+                                             float scale, Idx wlim = 0) {
   constexpr int VEC = Elem<T>::VEC;
-  store_chunks_fn<T, VPT, TEAM, ALIGNED, Idx>(row, vfirst, ve, cols, t, [&](int c, float* o) {
+  store_chunks_fn<T, VPT, TEAM, ALIGNED, Idx, WLIM>(
+      row, vfirst, ve, cols, t,
+      [&](int c, float* o) {
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) o[k] = v[c * VEC + k] * scale;
-  });
+        for (int k = 0; k < VEC; ++k) o[k] = v[c * VEC + k] * scale;
+      },
+      wlim);
 }
 
 // Row loads: raw 16-byte words; fp32 rows are unpacked into v at once (the

@@ -132,14 +132,21 @@ __device__ __forceinline__ size_t row_limit(const SoftmaxScaling& sc, size_t row
 // Otherwise (blocks or chunks with different references are merged later):
 // (x - ref) is formed first, exact for the largest terms, and no bias is
 // applied, so the partial sums of different references compare directly.
-// k = scale * log2(e) (log2(e) for the plain softmax).
+// k = scale * log2(e) (log2(e) for the plain softmax).  live: bit i clear
+// when chunk i holds only masked columns (all -inf, see live_chunks); its
+// terms are 0 and are not computed.
 template <typename T, int VPT, bool FOLD>
-__device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref, float k) {
+__device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref, float k, unsigned live = ~0u) {
   constexpr int VEC = Elem<T>::VEC;
   float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const float c = Elem<T>::kFoldBias - ref * k;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
+    if (((live >> i) & 1u) == 0u) {
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) v[i * VEC + j] = 0.0f;
+      continue;
+    }
     float f[VEC];
     if constexpr (sizeof(T) == 4) {
 #pragma unroll
@@ -165,9 +172,26 @@ __device__ __forceinline__ float exp_sum(const uint4* raw, float* v, float ref, 
 // error of at most 1/2 in the exponent); rows with larger maxima (beyond
 // about 1.2e7 at scale 1) take the unfolded form, one uniform branch per row.
 template <typename T, int VPT>
-__device__ __forceinline__ float exp_sum_row(const uint4* raw, float* v, float m, float k) {
-  if (fabsf(m * k) < 0x1p24f) return exp_sum<T, VPT, true>(raw, v, m, k);
-  return exp_sum<T, VPT, false>(raw, v, exp_ref(m), k);
+__device__ __forceinline__ float exp_sum_row(const uint4* raw, float* v, float m, float k, unsigned live = ~0u) {
+  if (fabsf(m * k) < 0x1p24f) return exp_sum<T, VPT, true>(raw, v, m, k, live);
+  return exp_sum<T, VPT, false>(raw, v, exp_ref(m), k, live);
+}
+
+// Chunks of thread t that hold a column before lim (bit c for chunk c):
+// under a causal mask the rest are wholly masked, so their exponentials
+// need not be computed.  (Aligned rows: the thread's vector of the chunk;
+// the scalar path: its first element.)
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+__device__ __forceinline__ unsigned live_chunks(Idx vfirst, Idx lim, int t) {
+  constexpr int VEC = Elem<T>::VEC;
+  unsigned m = 0;
+#pragma unroll
+  for (int c = 0; c < VPT; ++c) {
+    const Idx first = ALIGNED ? (vfirst + static_cast<Idx>(c) * TEAM + t) * VEC
+                              : (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
+    m |= (first < lim ? 1u : 0u) << c;
+  }
+  return m;
 }
 
 // Max of the values a thread holds (after load_row).
@@ -200,8 +224,10 @@ __global__ void __launch_bounds__(kWarpThreads)
     const int lim = SC ? static_cast<int>(row_limit(sc, row, cols)) : cols;
     load_row<T, VPT, 32, ALIGNED, SC, int>(xr, 0, nvec, cols, lim, lane, raw, v);
     const float m = warp_max(row_max<T, VPT>(raw, v));
-    const float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k));
-    store_chunks<T, VPT, 32, ALIGNED, int>(yr, 0, nvec, cols, lane, v, Elem<T>::recip(s));
+    const unsigned live = SC ? live_chunks<T, VPT, 32, ALIGNED, int>(0, lim, lane) : ~0u;
+    const float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k, live));
+    store_chunks<T, VPT, 32, ALIGNED, int, SC>(yr, 0, nvec, cols, lane, v, Elem<T>::recip(s),
+                                               sc.skip_masked ? lim : cols);
   }
 }
 
@@ -249,9 +275,12 @@ __device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, f
 
 // ---------------------------------------------------------------- block path
 
-// One block per row; EPT = register-resident elements per thread.
+// One block per row; EPT = register-resident elements per thread.  Rows of
+// 32 bytes per thread (16 bf16 values) keep few loads in flight per thread,
+// so those kernels (up to 256 threads) are held to 2048 resident threads per
+// SM (32 registers).
 template <typename T, int THREADS, int EPT, bool ALIGNED, bool SC>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, (EPT * sizeof(T) <= 32 && THREADS <= 256 ? 2048 / THREADS : 1))
     softmax_block_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = EPT / VEC;
@@ -279,14 +308,16 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int w = 1; w < NW; ++w) m = fmaxf(m, red_max[w]);
 
-    float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k));
+    const unsigned live = SC ? live_chunks<T, VPT, THREADS, ALIGNED, int>(0, lim, t) : ~0u;
+    float s = warp_sum(exp_sum_row<T, VPT>(raw, v, m, k, live));
     if (lane == 0) red_sum[warp] = s;
     __syncthreads();
     s = red_sum[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) s += red_sum[w];
 
-    store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, 0, nvec, cols, t, v, Elem<T>::recip(s));
+    store_chunks<T, VPT, THREADS, ALIGNED, int, SC>(yr, 0, nvec, cols, t, v, Elem<T>::recip(s),
+                                                    sc.skip_masked ? lim : cols);
     __syncthreads();  // red_max / red_sum are rewritten by the next row
   }
 }
@@ -338,7 +369,8 @@ __global__ void __launch_bounds__(THREADS)
 
   // Blocks use different references, so the exponent difference is formed
   // first (exact for the largest terms) instead of folded into an FMA.
-  float s = warp_sum(exp_sum<T, VPT, false>(raw, v, exp_ref(m), k));
+  const unsigned live = SC ? live_chunks<T, VPT, THREADS, ALIGNED, int>(vb, lim, t) : ~0u;
+  float s = warp_sum(exp_sum<T, VPT, false>(raw, v, exp_ref(m), k, live));
   if (lane == 0) red_sum[warp] = s;
   __syncthreads();
   s = red_sum[0];
@@ -346,7 +378,8 @@ __global__ void __launch_bounds__(THREADS)
   for (int w = 1; w < NW; ++w) s += red_sum[w];
 
   const float2 ML = exchange_merge(ex, m, s, csize, crank, k);
-  store_chunks<T, VPT, THREADS, ALIGNED, int>(yr, vb, ve, cols, t, v, rescale(m, ML.x, k) * __frcp_rn(ML.y));
+  store_chunks<T, VPT, THREADS, ALIGNED, int, SC>(yr, vb, ve, cols, t, v, rescale(m, ML.x, k) * __frcp_rn(ML.y),
+                                                  sc.skip_masked ? lim : cols);
 }
 
 // ---------------------------------------------------------------- two-phase path
@@ -402,7 +435,7 @@ __device__ __forceinline__ void block_merge_ml(float& m, float& l, float2* red, 
 // and after lim, without loading those elements).
 template <typename T, int THREADS, int VPT, bool ALIGNED, bool MASK>
 __device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, size_t ve, size_t cols, size_t lim,
-                                                 int t, float k, float M, float L) {
+                                                 int t, float k, float M, float L, size_t wlim) {
   constexpr int E = VPT * Elem<T>::VEC;
   constexpr size_t STEP = static_cast<size_t>(THREADS) * VPT;
   const float r = __frcp_rn(L);
@@ -412,7 +445,7 @@ __device__ __forceinline__ void stream_normalise(const T* xr, T* yr, size_t vb, 
     float v[E];
     load_row<T, VPT, THREADS, ALIGNED, MASK, size_t>(xr, c, ve, cols, lim, t, raw, v);
     exp_sum<T, VPT, false>(raw, v, ref, k);
-    store_chunks<T, VPT, THREADS, ALIGNED, size_t>(yr, c, ve, cols, t, v, r);
+    store_chunks<T, VPT, THREADS, ALIGNED, size_t, MASK>(yr, c, ve, cols, t, v, r, wlim);
   }
 }
 
@@ -458,7 +491,8 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   }
 
   // pass 2: y = exp(x - M) / L
-  stream_normalise<T, THREADS, VPT, ALIGNED, SC>(xr, yr, vb, ve, cols, lim, t, k, m, l);
+  stream_normalise<T, THREADS, VPT, ALIGNED, SC>(xr, yr, vb, ve, cols, lim, t, k, m, l,
+                                                 sc.skip_masked ? lim : cols);
 }
 
 // ---------------------------------------------------------------- split path
@@ -513,7 +547,7 @@ __global__ void __launch_bounds__(kTwoPhaseThreads)
   for (unsigned i = threadIdx.x; i < nchunks; i += THREADS) merge_ml(m, l, part[i].x, part[i].y, k);
   block_merge_ml<THREADS>(m, l, red, k);
   stream_normalise<T, THREADS, VPT, ALIGNED, SC>(x + row * cols, y + row * cols, vb, ve, cols, lim, threadIdx.x, k,
-                                                 m, l);
+                                                 m, l, sc.skip_masked ? lim : cols);
 }
 
 // A wait on an mbarrier that nothing ever arrives on: every thread gives up
@@ -704,7 +738,7 @@ template <typename T>
 cudaError_t launch_dtype(const void* x, void* y, size_t rows, size_t cols, const fk_softmax_plan& p, bool aligned,
                          void* ws, const SoftmaxScaling* sc, cudaStream_t s) {
   if (sc == nullptr) {
-    const SoftmaxScaling none = {kLog2e, 0, 0, 0};
+    const SoftmaxScaling none = {kLog2e, 0, 0, 0, 0, 0, 0, 0, 0};
     return aligned ? launch_typed<T, true, false>(x, y, rows, cols, p, ws, none, s)
                    : launch_typed<T, false, false>(x, y, rows, cols, p, ws, none, s);
   }

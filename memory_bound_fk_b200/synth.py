@@ -69,12 +69,13 @@ class Workload:
 def algorithmic_bytes(op: str, itemsize: int, shape: tuple) -> int:
     """One read of the input plus one write of the output.  For the causal
     softmax (rows in blocks of T = cols queries against T keys) only the kept
-    entries are read: row i of a block reads i + 1 of its T values."""
-    if op == "softmax_causal":
+    entries are read: row i of a block reads i + 1 of its T values; with
+    masked stores skipped, only those are written too."""
+    if op in ("softmax_causal", "softmax_causal_skip"):
         rows, cols = shape
         full, rem = divmod(rows, cols)
         kept = full * cols * (cols + 1) // 2 + rem * (rem + 1) // 2
-        return (kept + rows * cols) * itemsize
+        return (kept + (kept if op == "softmax_causal_skip" else rows * cols)) * itemsize
     n = 1
     for d in shape:
         n *= d
@@ -105,6 +106,8 @@ WORKLOADS = {
                  "the gelu_bf16 values, exact GELU x*Phi(x)"),
         Workload("cfg4_causal", "softmax_causal", "bf16", (32 * 16 * 2048, 2048), 3,
                  "the cfg4_softmax scores, causal mask generated in the kernel (masked entries not read)"),
+        Workload("cfg4_causal_skip", "softmax_causal_skip", "bf16", (32 * 16 * 2048, 2048), 3,
+                 "as cfg4_causal, masked outputs not stored either (FK_SOFTMAX_SKIP_MASKED)"),
         # LayerNorm over transformer-shaped activations (hidden size 4096)
         Workload("ln_f32", "layernorm", "f32", (16384, 4096), 6,
                  "fp32 16384x4096, row r ~ N(mu_r, s_r^2), mu_r ~ U[-2,2], s_r ~ U[0.5,2]; "
@@ -276,7 +279,7 @@ def make(name: str, threads: int | None = None, rows: int | None = None) -> np.n
     if name == "cfg3_softmax":
         r = rows or 8192
         return _cfg3(rows=-(-r // CFG3_ROWS_PER_CHUNK) * CFG3_ROWS_PER_CHUNK, threads=threads)[:r]
-    if name in ("cfg4_softmax", "cfg4_causal"):
+    if name in ("cfg4_softmax", "cfg4_causal", "cfg4_causal_skip"):
         r = rows or CFG4_HEADS * CFG4_T
         return _cfg4(heads=-(-r // CFG4_T), threads=threads)[:r]
     if name == "cfg2_gelu_erf":

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 
 import oracle
-from _util import Guarded, check_softmax_bf16, check_softmax_f32, forced_plans
+from _util import Guarded, bf16_ordinal, check_softmax_bf16, check_softmax_f32, forced_plans
 from memory_bound_fk_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -203,3 +203,59 @@ def test_row_indices_beyond_32_bits(fk, torch_mod):
     one, half = 0x3F80, 0x3F00
     expect = np.where((idx % 3 == 0)[:, None], np.array([[one, 0]], np.uint16), np.array([[half, half]], np.uint16))
     assert np.array_equal(got, expect)
+
+
+def run_skip(fk, torch, x, scale, period, offset, plan=None, sentinel=7.0):
+    """FK_SOFTMAX_SKIP_MASKED into an output pre-filled with `sentinel`."""
+    rows, cols = x.shape
+    bf16 = x.dtype == np.uint16
+    tdt = torch.bfloat16 if bf16 else torch.float32
+    host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if bf16 else torch.from_numpy(x)
+    dev = torch.device("cuda:0")
+    xin = Guarded(torch, x.size, tdt, dev, fill=host.reshape(-1))
+    out = Guarded(torch, x.size, tdt, dev)
+    out.view.fill_(sentinel)
+    st = fk.fk_softmax_rows_causal_ex(xin.view.data_ptr(), out.view.data_ptr(), rows, cols,
+                                      fk.FK_BF16 if bf16 else fk.FK_F32, scale, period, offset, plan,
+                                      torch.cuda.current_stream().cuda_stream, fk.FK_SOFTMAX_SKIP_MASKED)
+    assert st == fk.FK_OK, fk.fk_status_string(st)
+    torch.cuda.synchronize()
+    assert out.canaries_intact() and xin.canaries_intact()
+    y = out.view.cpu()
+    if bf16:
+        return y.view(torch.int16).numpy().view(np.uint16).reshape(rows, cols)
+    return y.numpy().reshape(rows, cols)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("cols", [96, 2048, 50000, 200000, 700000])
+def test_skip_masked_stores(fk, torch_mod, dtype, cols):
+    """Kept outputs equal the oracle's; a masked output is left as it was,
+    or is 0 -- and it is always left as it was when its whole 16-byte vector
+    is masked (aligned rows), so the masked region costs no writes."""
+    rows, period, offset = 6, 6, cols // 3
+    x = synth.softmax_input(rows, cols, dtype, sigma=3.0, seed=cols + 11)
+    keep = kept_mask(rows, cols, period, offset)
+    vec = 4 if dtype == "f32" else 8
+    whole = np.zeros_like(keep)
+    q = np.arange(rows) % period + offset
+    whole[:] = (np.arange(cols)[None, :] // vec * vec) > q[:, None]   # vector starts after the last kept column
+    ref = oracle.softmax_rows_causal(x if dtype == "bf16" else x.astype(np.float64), 0.5, period, offset)
+    sent = 7.0
+    sent_bits = oracle.round_to_bf16(np.array([sent]))[0]
+    for p in [None] + forced_plans(fk, cols, dtype):
+        y = run_skip(fk, torch_mod, x, 0.5, period, offset, plan=p, sentinel=sent)
+        if dtype == "bf16":
+            d = np.abs(bf16_ordinal(y[keep]) - bf16_ordinal(ref[keep]))
+            assert d.max() <= 1
+            assert np.all((y[~keep] == sent_bits) | (y[~keep] == 0))
+            assert np.all(y[whole] == sent_bits)
+        else:
+            assert np.max(np.abs(y[keep].astype(np.float64) - ref[keep])) <= 1e-6
+            assert np.all((y[~keep] == sent) | (y[~keep] == 0.0))
+            assert np.all(y[whole] == sent)
+    # an unknown flag is rejected
+    import torch
+    t = torch.zeros(4, 4, device="cuda")
+    assert fk.fk_softmax_rows_causal_ex(t.data_ptr(), t.data_ptr(), 4, 4, fk.FK_F32, 1.0, 4, 0, None, 0, 2) \
+        == fk.FK_ERR_INVALID_ARG
