@@ -20,6 +20,8 @@ Definitions followed:
     scaled, -inf where the key comes after the query, then softmax).
   * LayerNorm (+ GELU): the same lecture, sections 6.1-6.2 (the fused
     LayerNorm -> Linear -> GELU example; F.layer_norm over the last axis).
+  * Attention forward: the same lecture, sections 7.3 and 8 (what Flash
+    Attention computes: softmax(scale Q K^T, causal mask) V).
 
 Parity pins: every function here is pinned by tests in
 ``tests/test_oracle_pins.py`` (closed forms, invariants, library routines
@@ -65,6 +67,8 @@ def _load():
         lib.oracle_softmax_rows_causal.restype = None
         lib.oracle_layernorm_rows.argtypes = [p, p, i, sz, sz, p, p, d, i, i]
         lib.oracle_layernorm_rows.restype = None
+        lib.oracle_attention.argtypes = [p, p, p, p, i, sz, sz, sz, sz, d, i, i]
+        lib.oracle_attention.restype = None
         for name in ("oracle_round_to_f32_array", "oracle_round_to_bf16_array",
                      "oracle_bf16_to_f64_array"):
             getattr(lib, name).argtypes = [p, p, sz]
@@ -220,6 +224,28 @@ def layernorm_rows(x: np.ndarray, eps: float = 1e-5, gamma=None, beta=None, gelu
     return y
 
 
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, causal: bool,
+              nthreads: int | None = None) -> np.ndarray:
+    """Attention forward over [bh, t, d] arrays (q: [bh, tq, d]; k, v:
+    [bh, tk, d]): softmax(scale * q k^T, causal mask with query i at key
+    position i + tk - tq) v.  float64 in -> float64 out; float32 -> float32;
+    uint16 (bf16 patterns) -> uint16; computed in double, rounded once."""
+    kinds = {np.dtype(np.float64): 0, np.dtype(np.float32): 1, np.dtype(np.uint16): 2}
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in kinds:
+        raise TypeError("q, k, v: one of float64, float32, uint16 (bf16 bits)")
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    if q.ndim != 3 or k.shape != v.shape or k.ndim != 3 or q.shape[0] != k.shape[0] or q.shape[2] != k.shape[2]:
+        raise ValueError("shapes [bh, tq, d], [bh, tk, d], [bh, tk, d]")
+    bh, tq, d = q.shape
+    tk = k.shape[1]
+    if causal and tk < tq:
+        raise ValueError("causal attention needs tk >= tq")
+    o = np.empty_like(q)
+    _load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), kinds[q.dtype], bh, tq, tk, d, float(scale),
+                             int(bool(causal)), nthreads or default_threads())
+    return o
+
+
 def round_to_f32(v: np.ndarray) -> np.ndarray:
     v = _c(v, np.float64)
     out = np.empty(v.shape, np.float32)
@@ -245,7 +271,7 @@ def bf16_to_f64(b: np.ndarray) -> np.ndarray:
 
 __all__ = [
     "gelu_tanh", "gelu_tanh_f64", "gelu_tanh_f32", "gelu_erf", "gelu_erf_f64",
-    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16", "softmax_rows_causal", "layernorm_rows",
+    "softmax_rows_f64", "softmax_rows_f32", "softmax_rows_bf16", "softmax_rows_causal", "layernorm_rows", "attention",
     "round_to_f32", "round_to_bf16", "round_to_f32_scalar", "round_to_bf16_scalar",
     "bf16_to_f64", "default_threads",
 ]

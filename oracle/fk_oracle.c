@@ -500,6 +500,76 @@ void oracle_layernorm_rows(const void *x, void *y, int kind, size_t rows, size_t
     parallel_ranges(layernorm_range, &c, rows, nthreads);
 }
 
+/* ------------------------------------------------------------------ */
+/* Attention forward                                                    */
+/* ------------------------------------------------------------------ */
+
+/* The attention that Flash Attention computes (lecture 6, "GPU Kernels and
+ * Triton", sections 7.3 and 8): for each of `bh` independent (batch, head)
+ * slices, with Q [tq, d], K [tk, d], V [tk, d] row-major,
+ *     S = scale * Q K^T,
+ *     S[i, j] = -inf where the key comes after the query (causal: query i
+ *               sits at position i + (tk - tq) of the key sequence),
+ *     P = softmax over each row of S (softmax_row_f64),
+ *     O = P V.
+ * Plain loops in double, no blocking; kinds as causal_ctx (0 double,
+ * 1 fp32, 2 bf16 patterns) for Q, K, V and O alike, O rounded once. */
+typedef struct {
+    const void *q, *k, *v;
+    void *o;
+    int kind;
+    size_t tq, tk, d;
+    double scale;
+    int causal;
+} attn_ctx;
+
+static double attn_in(const void *p, int kind, size_t i)
+{
+    causal_ctx io = {p, NULL, kind, 0, 1.0, 0, 0};
+    return causal_in(&io, i);
+}
+
+static void attention_range(void *p, size_t b, size_t e)
+{
+    attn_ctx *c = (attn_ctx *)p;
+    double *s = (double *)malloc(c->tk * sizeof(double) + 1);
+    double *pr = (double *)malloc(c->tk * sizeof(double) + 1);
+    causal_ctx out = {NULL, c->o, c->kind, 0, 1.0, 0, 0};
+    /* one (slice, query) pair per unit of work */
+    for (size_t u = b; u < e; ++u) {
+        const size_t h = u / c->tq, i = u % c->tq;
+        const size_t qb = (h * c->tq + i) * c->d;
+        for (size_t j = 0; j < c->tk; ++j) {
+            if (c->causal && j > i + (c->tk - c->tq)) {
+                s[j] = -INFINITY;
+                continue;
+            }
+            const size_t kb = (h * c->tk + j) * c->d;
+            double dot = 0.0;
+            for (size_t t = 0; t < c->d; ++t)
+                dot += attn_in(c->q, c->kind, qb + t) * attn_in(c->k, c->kind, kb + t);
+            s[j] = c->scale * dot;
+        }
+        softmax_row_f64(s, pr, c->tk);
+        for (size_t t = 0; t < c->d; ++t) {
+            double acc = 0.0;
+            for (size_t j = 0; j < c->tk; ++j)
+                if (pr[j] != 0.0)
+                    acc += pr[j] * attn_in(c->v, c->kind, (h * c->tk + j) * c->d + t);
+            causal_out(&out, qb + t, acc);
+        }
+    }
+    free(pr);
+    free(s);
+}
+
+void oracle_attention(const void *q, const void *k, const void *v, void *o, int kind, size_t bh, size_t tq,
+                      size_t tk, size_t d, double scale, int causal, int nthreads)
+{
+    attn_ctx c = {q, k, v, o, kind, tq, tk, d, scale, causal};
+    parallel_ranges(attention_range, &c, bh * tq, nthreads);
+}
+
 /* array forms of the rounding helpers */
 void oracle_round_to_f32_array(const double *v, float *out, size_t n)
 {

@@ -529,6 +529,73 @@ def test_layernorm_f32_and_bf16_round_the_double_result_once():
     assert np.array_equal(oracle.layernorm_rows(xb, 1e-5, g, b), viab)
 
 
+# ============================================================ attention
+# Attention forward (lecture 6, "GPU Kernels and Triton", sections 7.3 and 8):
+# softmax(scale Q K^T with the causal mask) V per (batch, head) slice.
+
+
+def _torch_attention(q, k, v, scale, causal):
+    s = torch.from_numpy(q) @ torch.from_numpy(k).transpose(1, 2) * scale
+    if causal:
+        tq, tk = q.shape[1], k.shape[1]
+        s = s.masked_fill(torch.ones(tq, tk, dtype=torch.bool).triu(1 + tk - tq), float("-inf"))
+    return (torch.softmax(s, dim=-1) @ torch.from_numpy(v)).numpy()
+
+
+@pytest.mark.parametrize("bh,tq,tk,d,causal", [(3, 16, 16, 8, True), (2, 9, 23, 16, True), (2, 17, 17, 64, False),
+                                                (1, 40, 40, 128, True), (2, 5, 31, 32, False)])
+def test_attention_matches_torch_float64(bh, tq, tk, d, causal):
+    q, k, v = (RNG.standard_normal((bh, t, d)) for t in (tq, tk, tk))
+    scale = 1.0 / math.sqrt(d)
+    o = oracle.attention(q, k, v, scale, causal)
+    assert np.max(np.abs(o - _torch_attention(q, k, v, scale, causal))) <= 1e-13
+
+
+def test_attention_closed_forms():
+    # constant value rows: every output row is that row (the weights sum to 1)
+    bh, t, d = 2, 12, 8
+    q, k = RNG.standard_normal((bh, t, d)), RNG.standard_normal((bh, t, d))
+    v = np.tile(RNG.standard_normal((bh, 1, d)), (1, t, 1))
+    o = oracle.attention(q, k, v, 0.7, True)
+    assert np.max(np.abs(o - v)) <= 1e-14
+    # causal: query 0 sees key 0 only; identical keys give the mean of the visible values
+    v = RNG.standard_normal((bh, t, d))
+    o = oracle.attention(q, k, v, 0.7, True)
+    assert np.max(np.abs(o[:, 0] - v[:, 0])) <= 1e-15
+    kk = np.tile(RNG.standard_normal((bh, 1, d)), (1, t, 1))
+    o = oracle.attention(q, kk, v, 0.7, True)
+    means = np.cumsum(v, axis=1) / np.arange(1, t + 1)[None, :, None]
+    assert np.max(np.abs(o - means)) <= 1e-14
+    o = oracle.attention(q, kk, v, 0.7, False)
+    assert np.max(np.abs(o - v.mean(axis=1, keepdims=True))) <= 1e-14
+    # one key far ahead of the others: the output is its value row
+    k2 = RNG.standard_normal((1, t, d)) * 0.01
+    k2[0, 5] = q[0, 3] * 1000.0
+    o = oracle.attention(q[:1], k2, v[:1], 1.0, False)
+    assert np.max(np.abs(o[0, 3] - v[0, 5])) <= 1e-12
+
+
+def test_attention_brute_force_mpmath():
+    mpmath.mp.dps = 40
+    q, k, v = (RNG.standard_normal((1, 4, 3)) for _ in range(3))
+    o = oracle.attention(q, k, v, 0.5, True)
+    for i in range(4):
+        s = [mpmath.mpf(0.5) * mpmath.fsum(mpmath.mpf(float(a)) * mpmath.mpf(float(b)) for a, b in zip(q[0, i], k[0, j]))
+             for j in range(i + 1)]
+        m = max(s)
+        e = [mpmath.exp(x - m) for x in s]
+        tot = mpmath.fsum(e)
+        for t in range(3):
+            exact = mpmath.fsum(e[j] * mpmath.mpf(float(v[0, j, t])) for j in range(i + 1)) / tot
+            assert abs(mpmath.mpf(float(o[0, i, t])) - exact) <= 1e-15
+
+
+def test_attention_bf16_rounds_the_double_result_once():
+    q, k, v = (oracle.round_to_bf16(RNG.standard_normal((2, 10, 16))) for _ in range(3))
+    via = oracle.round_to_bf16(oracle.attention(*(oracle.bf16_to_f64(a) for a in (q, k, v)), 0.25, True))
+    assert np.array_equal(oracle.attention(q, k, v, 0.25, True), via)
+
+
 # ================================================================= rounding
 
 def _all_finite_bf16():
