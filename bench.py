@@ -385,6 +385,11 @@ def run_ours(args) -> dict | None:
     reduced = max_over_ranks([total_ms] + per_kernel_ms, world, device)
     max_ms, kernel_ms = reduced[0], reduced[1:]
 
+    # copy ceiling for the dominant kernel's bytes: cudaMemcpy D2D and
+    # libfk's plain 16-byte copy, same buffers, timed the same way
+    dom_i = max(range(len(names)), key=lambda i: kernel_ms[i])
+    copy_ceiling = copy_reference(fk, dev_in[names[dom_i]], dev_out[names[dom_i]], stream, device, world)
+
     # end to end: pinned host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
@@ -395,7 +400,9 @@ def run_ours(args) -> dict | None:
         threads = host_threads()
         f = oracle_sample_plan(names, host, args.cpu_budget, threads)
         res = oracle_run(names, host, f, threads)
+        one = oracle_run(names, host, f / max(1, threads), 1)
         cpu = {"value": res["bytes"] / res["seconds"] / 1e9, "unit": UNIT, "cores": threads,
+               "value_1_thread": one["bytes"] / one["seconds"] / 1e9,
                "kind": "oracle",
                "sample": f"leading {100 * f:.3f}% of every workload ({res['elements']} elements, "
                          f"{res['bytes'] / 1e9:.3f} GB algorithmic, {res['seconds']:.1f} s)"}
@@ -445,13 +452,42 @@ def run_ours(args) -> dict | None:
                      "frac": round(dk["GB_s"] / peaks["hbm_gbs"], 4),
                      "peak_source": peaks["source"],
                      "traffic": traffic, "traffic_source": traffic_src,
-                     "algorithmic_bytes_per_launch": dk["bytes_per_launch"]},
+                     "algorithmic_bytes_per_launch": dk["bytes_per_launch"],
+                     "copy_ceiling": copy_ceiling,
+                     "frac_of_copy_ceiling": (round(dk["GB_s"] / copy_ceiling["fk_copy_GB_s"], 4)
+                                              if copy_ceiling else None)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": len(calls) * args.steps,
         "clocks": clocks,
     }
     return line
+
+
+def copy_reference(fk, src, dst, stream, device, world, reps: int = 7) -> dict | None:
+    """Median time of copying src's bytes into dst with cudaMemcpyAsync
+    (torch's copy_) and with libfk's fk_copy: the achievable-bandwidth
+    reference of the same byte count (read + write counted)."""
+    import torch
+    nbytes = src.numel() * src.element_size()
+    if nbytes % 16:
+        return None
+    out = {}
+    for label, fn in (("cudaMemcpy", lambda: dst.copy_(src)),
+                      ("fk_copy", lambda: fk.fk_copy(src.data_ptr(), dst.data_ptr(), nbytes, stream.cuda_stream))):
+        fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            ts.append(a.elapsed_time(b))
+        ms = max_over_ranks([sorted(ts)[len(ts) // 2]], world, device)[0]
+        out[f"{label}_GB_s"] = round(2 * nbytes / (ms * 1e-3) / 1e9, 1)
+    out["bytes_copied"] = nbytes
+    return out
 
 
 def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step, params=None):

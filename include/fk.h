@@ -113,6 +113,17 @@ typedef enum fk_gelu_kind {
 FK_API fk_status fk_gelu(const void *x, void *y, size_t n, int dtype, int kind, void *stream);
 
 /*
+ * fk_copy -- the bandwidth reference: a plain 16-byte streaming copy with
+ * the GELU kernel's access pattern (no arithmetic).  The fused kernels are
+ * reported against it (the lectures' bandwidth-utilisation metric).
+ *   src, dst  device memory, 16-byte aligned, not overlapping.
+ *   bytes     a multiple of 16 (0 = no-op).
+ * FK_ERR_INVALID_ARG for misalignment, overlap or a size outside either
+ * allocation.
+ */
+FK_API fk_status fk_copy(const void *src, void *dst, size_t bytes, void *stream);
+
+/*
  * fk_softmax_rows -- softmax over each row of a row-major [rows, cols]
  * matrix (lecture 6, section 7.2; lecture-6 notes, section 5.2).
  *   x      [in]  rows*cols elements of `dtype`, device-accessible, aligned to
@@ -320,6 +331,27 @@ FK_API fk_status fk_layernorm_rows_plan(size_t rows, size_t cols, int dtype, int
 FK_API fk_status fk_layernorm_rows_ex(const void *x, void *y, const float *gamma, const float *beta,
                                       size_t rows, size_t cols, int dtype, float eps, int epilogue,
                                       const fk_softmax_plan *plan, void *stream);
+
+/*
+ * fk_attention_fwd -- attention forward on the tensor cores, the computation
+ * Flash Attention tiles (lecture 6, "GPU Kernels and Triton", sections 7.3
+ * and 8):
+ *     O = softmax(scale * Q K^T  [+ causal mask: key j > query i is -inf]) V
+ * for bh independent (batch, head) slices; S and P stay on chip (tensor
+ * memory and shared memory), with the running max / sum of section 7.2.
+ *   q, k, v  [bh, t, d] bf16, contiguous, device memory, 16-byte aligned.
+ *   o        [bh, t, d] bf16 output; must not overlap q, k or v.
+ *   t        a multiple of 128 (queries and keys per slice); d = 64 or 128.
+ *   causal   0 or 1.
+ *   scale    finite, > 0 (e.g. 1 / sqrt(d)).
+ * Arithmetic: S and the O accumulator in fp32 (tcgen05, TMEM), P rounded to
+ * bf16 for the second product, O rounded to bf16 at the end.
+ * Errors: FK_ERR_INVALID_ARG for a shape or argument outside the above,
+ * bh * t >= 2^31, bad pointers or overlap.  A wait that gives up (see
+ * fk_wait_timeouts) leaves that block of O unwritten.
+ */
+FK_API fk_status fk_attention_fwd(const void *q, const void *k, const void *v, void *o, size_t bh, size_t t,
+                                  size_t d, int causal, float scale, void *stream);
 
 /*
  * fk_wait_timeouts -- health check of the cluster paths.  Blocks of a

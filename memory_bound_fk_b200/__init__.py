@@ -8,6 +8,7 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
 ``cudaStream_t`` integer):
     fk_gelu_tanh(x, y, n, stream) -> status
     fk_gelu(x, y, n, dtype, kind, stream) -> status
+    fk_copy(src, dst, bytes, stream) -> status     (bandwidth reference)
     fk_softmax_rows(x, y, rows, cols, dtype, stream) -> status
     fk_softmax_rows_ex(x, y, rows, cols, dtype, plan, stream) -> status
     fk_softmax_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
@@ -18,6 +19,7 @@ Raw C-ABI mirrors (same names, pointers as integers, stream as a
     fk_layernorm_rows(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, stream) -> status
     fk_layernorm_rows_ex(x, y, gamma, beta, rows, cols, dtype, eps, epilogue, plan, stream) -> status
     fk_layernorm_rows_plan(rows, cols, dtype, path=FK_PATH_AUTO) -> SoftmaxPlan
+    fk_attention_fwd(q, k, v, o, bh, t, d, causal, scale, stream) -> status
     fk_status_string(status) -> str
     fk_wait_timeouts(reset=False) -> int     (bounded-wait give-ups, synchronous)
     fk_wait_selftest(timeout_us, stream) -> status
@@ -28,6 +30,7 @@ Tensor conveniences (contiguous CUDA tensors; the current torch stream):
     softmax_rows(x, out=None, plan=None)    # softmax over the last dimension
     softmax_causal(x, scale, period=None, offset=0, out=None, plan=None)
     layernorm(x, eps=1e-5, weight=None, bias=None, gelu=None, out=None, plan=None)
+    attention(q, k, v, causal=True, scale=None, out=None)   # [..., t, d] bf16
 
 There is no fallback: if the library is missing or a call fails, an
 exception is raised.
@@ -104,6 +107,8 @@ def lib() -> ctypes.CDLL:
         vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
         L.fk_gelu_tanh.argtypes = [vp, vp, sz, vp]
         L.fk_gelu_tanh.restype = ci
+        L.fk_copy.argtypes = [vp, vp, sz, vp]
+        L.fk_copy.restype = ci
         L.fk_gelu.argtypes = [vp, vp, sz, ci, ci, vp]
         L.fk_gelu.restype = ci
         L.fk_softmax_rows.argtypes = [vp, vp, sz, sz, ci, vp]
@@ -133,6 +138,8 @@ def lib() -> ctypes.CDLL:
         L.fk_layernorm_rows_ex.argtypes = [vp, vp, vp, vp, sz, sz, ci, ctypes.c_float, ci,
                                            ctypes.POINTER(SoftmaxPlan), vp]
         L.fk_layernorm_rows_ex.restype = ci
+        L.fk_attention_fwd.argtypes = [vp, vp, vp, vp, sz, sz, sz, ci, ctypes.c_float, vp]
+        L.fk_attention_fwd.restype = ci
         L.fk_layernorm_rows_plan.argtypes = [sz, sz, ci, ci, ctypes.POINTER(SoftmaxPlan)]
         L.fk_layernorm_rows_plan.restype = ci
         L.fk_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), ci]
@@ -153,6 +160,10 @@ def header_functions() -> list[str]:
 
 def fk_gelu_tanh(x: int, y: int, n: int, stream: int = 0) -> int:
     return lib().fk_gelu_tanh(x, y, n, stream)
+
+
+def fk_copy(src: int, dst: int, nbytes: int, stream: int = 0) -> int:
+    return lib().fk_copy(src, dst, nbytes, stream)
 
 
 def fk_gelu(x: int, y: int, n: int, dtype: int, kind: int, stream: int = 0) -> int:
@@ -221,6 +232,11 @@ def fk_layernorm_rows_plan(rows: int, cols: int, dtype: int, path: int = FK_PATH
     if st != FK_OK:
         raise FkError(st, "fk_layernorm_rows_plan")
     return p
+
+
+def fk_attention_fwd(q: int, k: int, v: int, o: int, bh: int, t: int, d: int, causal: int, scale: float,
+                     stream: int = 0) -> int:
+    return lib().fk_attention_fwd(q, k, v, o, bh, t, d, causal, scale, stream)
 
 
 def fk_status_string(status: int) -> str:
@@ -419,14 +435,38 @@ def layernorm(x, eps: float = 1e-5, weight=None, bias=None, gelu: str | None = N
     return out
 
 
+def attention(q, k, v, causal: bool = True, scale: float | None = None, out=None):
+    """Attention forward on contiguous bf16 CUDA tensors [..., t, d] (all
+    leading dimensions are independent slices): softmax(scale q k^T, causal)
+    v, with scale = 1/sqrt(d) by default."""
+    import math
+
+    import torch
+    for name, a in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(a, name)
+        if a.dtype != torch.bfloat16 or a.shape != q.shape:
+            raise ValueError(f"{name} must be bfloat16 with q's shape")
+    t, d = q.shape[-2], q.shape[-1]
+    bh = q.numel() // (t * d) if t * d else 0
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor(out, "out")
+    st = fk_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), bh, t, d, int(bool(causal)),
+                          1.0 / math.sqrt(d) if scale is None else scale, _stream_handle(q))
+    if st != FK_OK:
+        raise FkError(st, "fk_attention_fwd")
+    return out
+
+
 __all__ = [
     "FK_OK", "FK_ERR_INVALID_ARG", "FK_ERR_UNSUPPORTED_DTYPE", "FK_ERR_UNSUPPORTED_DEVICE",
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_GELU_TANH", "FK_GELU_ERF", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
-    "fk_gelu_tanh", "fk_gelu", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
+    "fk_gelu_tanh", "fk_gelu", "fk_copy", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
     "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
     "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal", "FK_SOFTMAX_SKIP_MASKED",
-    "fk_layernorm_rows", "fk_layernorm_rows_ex", "fk_layernorm_rows_plan", "layernorm", "FK_EPILOGUE_NONE", "FK_EPILOGUE_GELU_TANH",
+    "fk_layernorm_rows", "fk_layernorm_rows_ex", "fk_layernorm_rows_plan", "layernorm",
+    "fk_attention_fwd", "attention", "FK_EPILOGUE_NONE", "FK_EPILOGUE_GELU_TANH",
     "FK_EPILOGUE_GELU_ERF",
     "fk_status_string", "fk_last_cuda_error", "fk_version", "fk_wait_timeouts",
     "fk_wait_selftest", "make_plan", "gelu_tanh", "gelu",

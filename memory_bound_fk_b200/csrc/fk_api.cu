@@ -185,6 +185,18 @@ fk_status fk_gelu(const void* x, void* y, size_t n, int dtype, int kind, void* s
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 
+fk_status fk_copy(const void* src, void* dst, size_t bytes, void* stream) {
+  if (bytes == 0) return FK_OK;
+  if (bytes % 16 != 0 || reinterpret_cast<uintptr_t>(src) % 16 != 0 || reinterpret_cast<uintptr_t>(dst) % 16 != 0)
+    return FK_ERR_INVALID_ARG;
+  if (src == dst) return FK_ERR_INVALID_ARG;
+  const fk::DeviceInfo* dev = nullptr;
+  const fk_status st = fk::check_call(src, dst, bytes / 16, 16, &dev);
+  if (st != FK_OK) return st;
+  const cudaError_t e = fk::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
 fk_status fk_gelu_tanh(const float* x, float* y, size_t n, void* stream) {
   return fk_gelu(x, y, n, FK_F32, FK_GELU_TANH, stream);
 }
@@ -359,7 +371,40 @@ fk_status fk_wait_timeouts(unsigned int* count, int reset) {
   const fk::DeviceInfo* info = fk::current_device_info(&dev);
   if (info == nullptr || !info->ok) return FK_ERR_UNSUPPORTED_DEVICE;
   if (info->major != 10 || info->minor != 0) return FK_ERR_UNSUPPORTED_DEVICE;
-  const cudaError_t e = fk::read_wait_timeouts(count, reset != 0);
+  unsigned a = 0, b = 0;
+  cudaError_t e = fk::read_wait_timeouts(&a, reset != 0);
+  if (e == cudaSuccess) e = fk::read_attention_wait_timeouts(&b, reset != 0);
+  *count = a + b;
+  return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
+}
+
+fk_status fk_attention_fwd(const void* q, const void* k, const void* v, void* o, size_t bh, size_t t, size_t d,
+                           int causal, float scale, void* stream) {
+  if (causal != 0 && causal != 1) return FK_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !(scale <= FLT_MAX)) return FK_ERR_INVALID_ARG;
+  if (bh == 0 || t == 0) return FK_OK;
+  if ((d != 64 && d != 128) || t % 128 != 0) return FK_ERR_INVALID_ARG;
+  if (bh > (size_t{1} << 31) / t || bh * t >= (size_t{1} << 31)) return FK_ERR_INVALID_ARG;
+  const size_t n = bh * t * d;
+  const size_t bytes = n * 2;
+  for (const void* p : {q, k, v, static_cast<const void*>(o)})
+    if (p == nullptr || reinterpret_cast<uintptr_t>(p) % 16 != 0) return FK_ERR_INVALID_ARG;
+  const uintptr_t ob = reinterpret_cast<uintptr_t>(o);
+  for (const void* p : {q, k, v}) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    if (a < ob + bytes && ob < a + bytes) return FK_ERR_INVALID_ARG;  // the output may not overlap an input
+  }
+  const fk::DeviceInfo* dev = nullptr;
+  fk_status st = fk::check_call(q, o, n, 2, &dev);
+  if (st != FK_OK) return st;
+  int di = -1;
+  if (cudaGetDevice(&di) != cudaSuccess) return FK_ERR_UNSUPPORTED_DEVICE;
+  for (const void* p : {k, v}) {
+    st = fk::check_pointer(p, bytes, di);
+    if (st != FK_OK) return st;
+  }
+  const cudaError_t e = fk::launch_attention(q, k, v, o, bh, t, static_cast<int>(d), causal != 0, scale,
+                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 

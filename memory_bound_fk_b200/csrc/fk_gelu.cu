@@ -118,3 +118,43 @@ cudaError_t launch_gelu(const void* x, void* y, size_t n, int dtype, int kind, c
 }
 
 }  // namespace fk
+
+// ---------------------------------------------------------------- copy reference
+// A plain 16-byte streaming copy with the same access pattern as the GELU
+// kernel (one batch of two vectors per thread): the achievable-bandwidth
+// reference that the fused kernels are measured against.
+namespace fk {
+namespace {
+
+__global__ void __launch_bounds__(kGeluThreads) copy_kernel(const uint4* src, uint4* dst, size_t nvec) {
+  constexpr size_t kPerBlock = static_cast<size_t>(kGeluThreads) * kGeluUnroll;
+  for (size_t b = blockIdx.x; b * kPerBlock < nvec; b += gridDim.x) {
+    const size_t base = b * kPerBlock + threadIdx.x;
+    uint4 v[kGeluUnroll];
+#pragma unroll
+    for (int u = 0; u < kGeluUnroll; ++u) {
+      const size_t i = base + static_cast<size_t>(u) * kGeluThreads;
+      v[u] = ld_stream_v4_if(src + i, i < nvec, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kGeluUnroll; ++u) {
+      const size_t i = base + static_cast<size_t>(u) * kGeluThreads;
+      st_stream_v4_if(dst + i, v[u], i < nvec);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t stream) {
+  const size_t nvec = bytes / 16;
+  const size_t per_block = static_cast<size_t>(kGeluThreads) * kGeluUnroll;
+  size_t blocks = (nvec + per_block - 1) / per_block;
+  if (blocks > kGeluMaxGrid) blocks = kGeluMaxGrid;
+  if (blocks < 1) return cudaSuccess;
+  copy_kernel<<<static_cast<unsigned>(blocks), kGeluThreads, 0, stream>>>(static_cast<const uint4*>(src),
+                                                                          static_cast<uint4*>(dst), nvec);
+  return cudaGetLastError();
+}
+
+}  // namespace fk

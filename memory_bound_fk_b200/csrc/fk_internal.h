@@ -27,6 +27,9 @@ const DeviceInfo* current_device_info(int* device_out);
 // FK_GELU_ERF.  Arguments already validated.
 cudaError_t launch_gelu(const void* x, void* y, size_t n, int dtype, int kind, cudaStream_t stream);
 
+// dst <- src, bytes a multiple of 16 and both 16-byte aligned (validated).
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t stream);
+
 // ---- softmax -----------------------------------------------------------
 constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
 constexpr int kWarpThreads = 32 * kWarpRowsPerBlock;
@@ -106,6 +109,13 @@ cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const f
 
 // Workspace bytes a validated plan needs (0 except on the split path).
 size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan);
+
+// ---- attention ------------------------------------------------------------
+// O = softmax(scale Q K^T, causal) V over bh slices of [t, d] bf16 rows
+// (validated: t % 128 == 0, d in {64, 128}, 16-byte aligned, bh * t < 2^31).
+cudaError_t launch_attention(const void* q, const void* k, const void* v, void* o, size_t bh, size_t t, int d,
+                             bool causal, float scale, cudaStream_t stream);
+cudaError_t read_attention_wait_timeouts(unsigned* out, bool reset);
 
 // Number of threads whose bounded mbarrier wait gave up, on the current
 // device; optionally reset to 0.  Synchronous.

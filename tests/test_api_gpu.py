@@ -79,3 +79,18 @@ def test_host_cost_per_call_is_small(fk, cuda_device):
     torch.cuda.synchronize()
     print(f"host time per fk_softmax_rows call (incl. ctypes): {dt * 1e6:.2f} us")
     assert dt < 50e-6
+
+
+def test_fk_copy_reference(fk, cuda_device):
+    import torch
+    x = torch.randint(0, 1 << 30, ((1 << 22) + 4,), dtype=torch.int32, device="cuda")
+    y = torch.zeros_like(x)
+    nb = x.numel() * 4
+    assert fk.fk_copy(x.data_ptr(), y.data_ptr(), nb, 0) == fk.FK_OK
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
+    assert fk.fk_copy(x.data_ptr(), y.data_ptr(), 0, 0) == fk.FK_OK
+    assert fk.fk_copy(x.data_ptr(), y.data_ptr(), 24, 0) == fk.FK_ERR_INVALID_ARG      # not a multiple of 16
+    assert fk.fk_copy(x.data_ptr() + 4, y.data_ptr(), 32, 0) == fk.FK_ERR_INVALID_ARG  # misaligned
+    assert fk.fk_copy(x.data_ptr(), x.data_ptr() + 16, 64, 0) == fk.FK_ERR_INVALID_ARG  # overlap
+    assert fk.fk_copy(x.data_ptr(), y.data_ptr(), nb + (1 << 30), 0) == fk.FK_ERR_INVALID_ARG  # past the allocation

@@ -1,0 +1,114 @@
+"""fk_attention_fwd (tcgen05 tensor cores) against the double-precision
+oracle of softmax(scale Q K^T, causal) V.
+
+Tolerance, derived from the kernel's arithmetic: S and O accumulate in fp32
+(errors ~1e-6 relative), P is rounded to bf16 before the second product
+(relative error <= 2^-9 per weight, so O moves by at most 2^-9 max|v|), and
+O is rounded to bf16 (2^-9 |O|).  The test allows twice that:
+|O - O_ref| <= 2^-8 (|O_ref| + max |v| of the slice).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from _util import Guarded
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_mod(cuda_device):
+    import torch
+    return torch
+
+
+def _bf16(torch, bits, dev):
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def run(fk, torch, q, k, v, causal, scale):
+    """q, k, v: uint16 bf16 bits [bh, t, d].  Returns O bits."""
+    bh, t, d = q.shape
+    dev = torch.device("cuda:0")
+    tq, tk, tv = (_bf16(torch, a, dev) for a in (q, k, v))
+    out = Guarded(torch, q.size, torch.bfloat16, dev)
+    st = fk.fk_attention_fwd(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), out.view.data_ptr(), bh, t, d,
+                             int(causal), scale, torch.cuda.current_stream().cuda_stream)
+    assert st == fk.FK_OK, fk.fk_status_string(st)
+    torch.cuda.synchronize()
+    assert out.canaries_intact()
+    return out.view.cpu().view(torch.int16).numpy().view(np.uint16).reshape(bh, t, d)
+
+
+def check(o_bits, q, k, v, causal, scale):
+    ref = oracle.attention(*(oracle.bf16_to_f64(a) for a in (q, k, v)), scale, causal)
+    o = oracle.bf16_to_f64(o_bits)
+    vmax = np.abs(oracle.bf16_to_f64(v)).max(axis=(1, 2))[:, None, None]
+    tol = 2.0 ** -8 * (np.abs(ref) + vmax)
+    err = np.abs(o - ref)
+    assert np.all(np.isfinite(o))
+    assert np.all(err <= tol), f"max err {err.max():.3e}, worst ratio {(err / tol).max():.2f}"
+    return float((err / tol).max())
+
+
+def inputs(bh, t, d, seed, sigma=1.0):
+    g = np.random.default_rng(seed)
+    return tuple(oracle.round_to_bf16(g.standard_normal((bh, t, d)) * sigma) for _ in range(3))
+
+
+@pytest.mark.parametrize("bh,t,d,causal", [(1, 128, 64, False), (1, 128, 64, True), (2, 256, 64, True),
+                                            (2, 256, 128, False), (3, 384, 128, True), (2, 512, 64, False),
+                                            (1, 1024, 128, True), (4, 256, 128, True)])
+def test_parity(fk, torch_mod, bh, t, d, causal):
+    q, k, v = inputs(bh, t, d, seed=bh * 1000 + t + d)
+    scale = 1.0 / math.sqrt(d)
+    check(run(fk, torch_mod, q, k, v, causal, scale), q, k, v, causal, scale)
+    assert fk.fk_wait_timeouts(reset=True) == 0
+
+
+@pytest.mark.parametrize("sigma,scale", [(3.0, 0.125), (1.0, 1.0), (0.2, 0.05)])
+def test_score_ranges(fk, torch_mod, sigma, scale):
+    """Peaked and flat attention: large scores (the running max moves often)
+    and small ones (nearly uniform weights)."""
+    q, k, v = inputs(2, 384, 64, seed=int(sigma * 100), sigma=sigma)
+    check(run(fk, torch_mod, q, k, v, True, scale), q, k, v, True, scale)
+
+
+def test_constant_values_and_first_row(fk, torch_mod):
+    """With every value row equal, every output row is that row; causal row
+    0 sees key 0 only."""
+    bh, t, d = 2, 256, 128
+    q, k, v = inputs(bh, t, d, seed=5)
+    vc = np.repeat(v[:, :1], t, axis=1)
+    o = oracle.bf16_to_f64(run(fk, torch_mod, q, k, vc, True, 0.1))
+    assert np.max(np.abs(o - oracle.bf16_to_f64(vc))) <= 2.0 ** -8 * np.abs(oracle.bf16_to_f64(vc)).max()
+    o = oracle.bf16_to_f64(run(fk, torch_mod, q, k, v, True, 0.1))
+    v0 = oracle.bf16_to_f64(v[:, 0])
+    assert np.all(np.abs(o[:, 0] - v0) <= 2.0 ** -8 * np.abs(v0))
+
+
+def test_rejects_bad_arguments(fk, torch_mod):
+    torch = torch_mod
+    x = torch.zeros(2, 256, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(x)
+    p = x.data_ptr()
+    E = fk.FK_ERR_INVALID_ARG
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 2, 200, 64, 1, 0.1, 0) == E      # t not a multiple of 128
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 2, 256, 96, 1, 0.1, 0) == E      # d not 64 / 128
+    assert fk.fk_attention_fwd(p, p, p, p, 2, 256, 64, 1, 0.1, 0) == E                 # output overlaps an input
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 2, 256, 64, 2, 0.1, 0) == E      # causal not 0/1
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 2, 256, 64, 1, 0.0, 0) == E      # scale
+    assert fk.fk_attention_fwd(p + 2, p, p, y.data_ptr(), 1, 128, 64, 1, 0.1, 0) == E  # misaligned
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 4, 256, 64, 1, 0.1, 0) == E      # past the allocation
+    assert fk.fk_attention_fwd(p, p, p, y.data_ptr(), 0, 256, 64, 1, 0.1, 0) == fk.FK_OK
+
+
+def test_tensor_wrapper_against_torch_sdpa(fk, torch_mod):
+    """Sanity against torch's own scaled_dot_product_attention on the GPU."""
+    torch = torch_mod
+    q, k, v = (torch.randn(2, 4, 512, 128, device="cuda", dtype=torch.bfloat16) for _ in range(3))
+    o = fk.attention(q, k, v, causal=True)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(), is_causal=True)
+    assert torch.max(torch.abs(o.float() - ref)).item() <= 2e-2
