@@ -464,6 +464,123 @@ def run_ours(args) -> dict | None:
     return line
 
 
+def run_attention(args) -> dict | None:
+    """bench.py --workload attn_causal_bf16 | attn_bf16: the tcgen05 attention
+    forward, timed as the other workloads (W warm-ups, K steps between
+    barriers, CUDA events on the stream, max over ranks), reported in
+    algorithmic TFLOP/s (unmasked pairs only) against the measured bf16
+    tensor-core peak."""
+    import math
+
+    import torch
+
+    import memory_bound_fk_b200 as fk
+    from memory_bound_fk_b200 import synth
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    fk.lib()
+    n = args.workload
+    w = synth.WORKLOADS[n]
+    causal = w.op == "attention"
+    host = synth.make(n, rows=args.rows)
+    _, bh, t, d = host.shape
+    scale = 1.0 / math.sqrt(d)
+    flops = synth.attention_flops(bh, t, d, causal)
+    qkv = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16).to(device)
+    o = torch.empty(bh, t, d, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+
+    def call(src=qkv, dst=o):
+        st = fk.fk_attention_fwd(src[0].data_ptr(), src[1].data_ptr(), src[2].data_ptr(), dst.data_ptr(), bh, t, d,
+                                 int(causal), scale, sh)
+        if st != fk.FK_OK:
+            raise fk.FkError(st, n)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        call()
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    barrier()
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    max_ms = max_over_ranks([a.elapsed_time(b)], world, device)[0]
+    tflops = flops * args.steps * world / (max_ms * 1e-3) / 1e12
+
+    # end to end: q, k, v from pinned host memory in, o back out, every step
+    e2e = None
+    if not args.no_e2e:
+        pin_in = torch.empty(qkv.shape, dtype=torch.int16, pin_memory=True)
+        pin_in.copy_(torch.from_numpy(host.view(np.int16)))
+        pin_out = torch.empty(o.shape, dtype=torch.int16, pin_memory=True)
+        steps = max(3, min(args.steps, args.e2e_steps))
+        barrier()
+        a.record(stream)
+        for _ in range(steps):
+            qkv.view(torch.int16).copy_(pin_in, non_blocking=True)
+            call()
+            pin_out.copy_(o.view(torch.int16), non_blocking=True)
+        b.record(stream)
+        barrier()
+        ms_e = max_over_ranks([a.elapsed_time(b)], world, device)[0]
+        e2e = {"value": round(flops * steps * world / (ms_e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": pin_in.numel() * 2, "d2h_bytes_per_step": pin_out.numel() * 2,
+               "steps": steps, "ms_per_step": round(ms_e / steps, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = host_threads()
+        nb = 1
+        t0 = time.perf_counter()
+        oracle.attention(*(host[i, :nb] for i in range(3)), scale, causal, nthreads=threads)
+        dt = time.perf_counter() - t0
+        cpu = {"value": synth.attention_flops(nb, t, d, causal) / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+               "kind": "oracle", "sample": f"{nb} of {bh} (batch, head) slices ({dt:.1f} s)"}
+    if rank != 0:
+        return None
+    d_all = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = float(d_all.get("bf16_tflops", 1590.0))
+    ms = max_ms / args.steps
+    kname = f"attention_fwd_kernel<d={d},causal={int(causal)}>"
+    return {
+        "metric": "attention forward TFLOP/s (bf16 in, fp32 accumulate) at 1 B200", "value": round(tflops, 2),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": n, "detail": w.recipe, "bh": bh, "t": t, "d": d, "causal": causal,
+                   "algorithmic_flops_per_step": flops,
+                   "l2": "q, k, v total %.0f MB; every launch reads them from HBM or L2" % (qkv.numel() * 2 / 1e6),
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "kernels": [{"workload": n, "kernel": kname, "ms": round(ms, 5), "TFLOP_s": round(flops / ms / 1e9, 1)}],
+        "roofline": {"bound": "tensor", "kernel": kname, "workload": n, "achieved": round(flops / ms / 1e9, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(flops / ms / 1e9 / peak, 4),
+                     "peak_source": "measured (cuBLAS bf16 burst)" if d_all else "fallback",
+                     "traffic": None},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 def copy_reference(fk, src, dst, stream, device, world, reps: int = 7) -> dict | None:
     """Median time of copying src's bytes into dst with cudaMemcpyAsync
     (torch's copy_) and with libfk's fk_copy: the achievable-bandwidth
@@ -718,7 +835,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="suite",
                    help="suite (default) or one of cfg1_gelu, cfg1_softmax, cfg2_gelu, "
                         "cfg3_softmax, cfg4_softmax, cfg5_softmax, and the operator variants "
-                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal, cfg4_causal_skip, ln_f32, ln_gelu_bf16")
+                        "cfg2_gelu_erf, gelu_bf16, gelu_erf_bf16, cfg4_causal, cfg4_causal_skip, ln_f32, ln_gelu_bf16, "
+                        "attn_causal_bf16, attn_bf16")
     p.add_argument("--rows", type=int, default=None,
                    help="profiling only: leading rows (elements for GELU) of each workload")
     p.add_argument("--no-e2e", action="store_true")
@@ -741,11 +859,13 @@ def main(argv=None):
         line = run_reference(args)
     elif args.impl == "unfused":
         line = run_unfused(args)
+    elif args.workload in ("attn_causal_bf16", "attn_bf16"):
+        line = run_attention(args)
     else:
         line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
-    if args.impl == "ours" and dist_env()[1] > 1:
+    if args.impl in ("ours",) and dist_env()[1] > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 

@@ -383,7 +383,7 @@ fk_status fk_attention_fwd(const void* q, const void* k, const void* v, void* o,
   if (causal != 0 && causal != 1) return FK_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !(scale <= FLT_MAX)) return FK_ERR_INVALID_ARG;
   if (bh == 0 || t == 0) return FK_OK;
-  if ((d != 64 && d != 128) || t % 128 != 0) return FK_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || t % 128 != 0 || t / 128 > 65535) return FK_ERR_INVALID_ARG;
   if (bh > (size_t{1} << 31) / t || bh * t >= (size_t{1} << 31)) return FK_ERR_INVALID_ARG;
   const size_t n = bh * t * d;
   const size_t bytes = n * 2;

@@ -5,18 +5,25 @@
 // sum l, rescale the output accumulator when m grows, and divide by l at the
 // end -- the online recurrence of section 7.2 -- so S and P never reach HBM.
 //
-// One CTA of 128 threads per (128-query block, batch*head).  Thread r owns
-// query row r, which is TMEM lane r of both accumulators:
-//   S (128 x 128 fp32, TMEM columns 0..127)   = Q K_j^T      (tcgen05.mma)
-//   O (128 x D   fp32, TMEM columns 128..)   += P_j V_j       (tcgen05.mma)
+// One CTA of 256 threads per (128-query block, batch*head): two warpgroups
+// that both serve query rows 0..127 (TMEM lanes; warp w reaches lanes
+// 32 (w % 4) ..), warpgroup g taking columns g*64 .. g*64+63 of S and its
+// half of O.  The row max is exchanged once per key block through shared
+// memory; the partial sums are added at the end.
+//   S_j (128 x 128 fp32, TMEM columns (j % 2) * 128 ..) = Q K_j^T   (tcgen05.mma)
+//   O   (128 x D   fp32, TMEM columns 256 ..)          += P_j V_j   (tcgen05.mma)
 // Q, K_j, V_j arrive by TMA in 128-byte-swizzled tiles; P_j is written by the
 // threads into a K-major swizzled shared-memory tile (bf16) for the second
 // MMA.  One thread issues the MMAs; completion arrives on an mbarrier
 // (tcgen05.commit).  Every mbarrier wait is bounded (1 s); a wait that gives
 // up is counted, the whole CTA stops, frees its TMEM and returns.
 //
-// This first version runs the steps of one key block in sequence (TMA ->
-// MMA -> softmax -> MMA); overlapping them across key blocks is the next step.
+// Pipelining: S is double-buffered in TMEM, so the tensor cores compute
+// S_{j+1} while the threads run the softmax of block j; P is
+// double-buffered in shared memory; K and V each have two buffers and their
+// own barriers, and each buffer is refilled by TMA as soon as the MMA that
+// read it has completed (K after S_j, V after O_{j-1}).  Causal grids hand
+// out the longest query blocks (most key blocks) first.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,10 +40,10 @@ __device__ unsigned int g_attn_wait_timeouts = 0;
 
 namespace {
 
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 256;  // two warpgroups on the same 128 rows
 constexpr int kAttnBlock = 128;                // queries per CTA = keys per step
 constexpr uint32_t kChunkBytes = 128 * 128;    // 128 rows x 64 bf16 columns
-constexpr uint32_t kTmemCols = 256;            // S: 128 columns, O: up to 128
+constexpr uint32_t kTmemCols = 512;            // S0, S1: 128 columns each; O: up to 128
 constexpr uint64_t kAttnWaitNs = 1000000000ull;
 
 __device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity) {
@@ -63,148 +70,215 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          float scale_log2) {
   constexpr int KC = D / 64;                     // 64-column chunks of a head row
   constexpr uint32_t TILE = KC * kChunkBytes;    // bytes of a 128 x D tile
+  constexpr uint32_t PTILE = 2 * kChunkBytes;    // bytes of a 128 x 128 P tile
   constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_kv, bar_mma;
+  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_o;
   __shared__ uint32_t tmem_slot;
+  // per-warpgroup row maxima of a key block; at the end, the row sums (the
+  // whole CTA fits the 227 KB of shared memory with ~1 KB to spare at D = 128)
+  __shared__ float xred[2][128];
 
+  // Q | K0 | K1 | V0 | V1 | P0 | P1, every tile 1024-byte aligned
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   uint8_t* sQ = base;
-  uint8_t* sK = base + TILE;
-  uint8_t* sV = base + 2 * TILE;
-  uint8_t* sP = base + 3 * TILE;  // 2 chunks: keys 0..63, 64..127
-  const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aP = smem_addr(sP);
+  uint8_t* sK[2] = {base + TILE, base + 2 * TILE};
+  uint8_t* sV[2] = {base + 3 * TILE, base + 4 * TILE};
+  uint8_t* sP[2] = {base + 5 * TILE, base + 5 * TILE + PTILE};
+  const uint32_t aQ = smem_addr(sQ);
 
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
-  const int qblk = blockIdx.x;
-  const int row0 = blockIdx.y * t + qblk * kAttnBlock;  // first query row in the [bh * t, D] view
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int wg = warp >> 2;                        // warpgroup: S columns wg*64.., O columns wg*D/2..
+  const int r = ((warp & 3) << 5) | (tid & 31);    // query row = TMEM lane
+  const int slice = blockIdx.x;
+  const int nq = static_cast<int>(gridDim.y);
+  const int qblk = CAUSAL ? nq - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
+  const int row0 = slice * t + qblk * kAttnBlock;  // first query row in the [bh * t, D] view
+  const int nkv = CAUSAL ? qblk + 1 : t / kAttnBlock;
 
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
   if (tid == 0) {
     mbar_init(&bar_q, 1);
-    mbar_init(&bar_kv, 1);
-    mbar_init(&bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_k[i], 1);
+      mbar_init(&bar_v[i], 1);
+      mbar_init(&bar_s[i], 1);
+    }
+    mbar_init(&bar_o, 1);
     fence_mbarrier_init();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = tmem_slot;
-  const uint32_t lane = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem + lane, tO = tmem + lane + 128;
+  const uint32_t tmem = tmem_slot;                        // S0 | S1 | O
+  const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tO = tmem + lane + 256 + wg * (D / 2);
 
+  // producer side, thread 0 only
+  auto load_k = [&](int j) {
+    const int b = j & 1;
+    mbar_arrive_expect_tx(&bar_k[b], TILE);
+#pragma unroll
+    for (int c = 0; c < KC; ++c) tc::tma_load_2d(sK[b] + c * kChunkBytes, &tmk, &bar_k[b], c * 64, slice * t + j * 128);
+  };
+  auto load_v = [&](int j) {
+    const int b = j & 1;
+    mbar_arrive_expect_tx(&bar_v[b], TILE);
+#pragma unroll
+    for (int c = 0; c < KC; ++c) tc::tma_load_2d(sV[b] + c * kChunkBytes, &tmv, &bar_v[b], c * 64, slice * t + j * 128);
+  };
+  // S_j = Q K_j^T into TMEM columns (j & 1) * 128, once K_j has landed
+  auto issue_s = [&](int j) -> bool {
+    const int b = j & 1;
+    if (!attn_wait(&bar_k[b], (j >> 1) & 1)) return false;
+    tc::fence_after_sync();
+    const uint32_t aK = smem_addr(sK[b]);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t off = (ks / 4) * kChunkBytes + (ks % 4) * 32;
+      tc::mma_bf16(tmem + b * 128, tc::smem_desc(aQ + off, 16, 1024), tc::smem_desc(aK + off, 16, 1024), IDESC_S,
+                   ks > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&bar_s[b]);
+    return true;
+  };
+
+  bool ok = true;
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar_q, TILE);
 #pragma unroll
     for (int c = 0; c < KC; ++c) tc::tma_load_2d(sQ + c * kChunkBytes, &tmq, &bar_q, c * 64, row0);
+    load_k(0);
+    load_v(0);
+    if (nkv > 1) {
+      load_k(1);
+      load_v(1);
+    }
+    ok = attn_wait(&bar_q, 0) && issue_s(0);
   }
-  const int nkv = CAUSAL ? qblk + 1 : t / kAttnBlock;
   float m_i = -INFINITY, l_i = 0.0f;
-  bool ok = __syncthreads_and(attn_wait(&bar_q, 0)) != 0;
 
-  for (int j = 0; j < nkv && ok; ++j) {
-    const int krow = blockIdx.y * t + j * kAttnBlock;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bar_kv, 2 * TILE);
-#pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        tc::tma_load_2d(sK + c * kChunkBytes, &tmk, &bar_kv, c * 64, krow);
-        tc::tma_load_2d(sV + c * kChunkBytes, &tmv, &bar_kv, c * 64, krow);
-      }
-    }
-    ok = __syncthreads_and(attn_wait(&bar_kv, j & 1)) != 0;
-    if (!ok) break;
-
-    // S = Q K_j^T: D/16 MMAs of K = 16, both operands K-major
-    if (tid == 0) {
-      tc::fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (ks / 4) * kChunkBytes + (ks % 4) * 32;
-        tc::mma_bf16(tmem, tc::smem_desc(aQ + off, 16, 1024), tc::smem_desc(aK + off, 16, 1024), IDESC_S,
-                     ks > 0 ? 1u : 0u);
-      }
-      tc::mma_commit(&bar_mma);
-    }
-    ok = __syncthreads_and(attn_wait(&bar_mma, 0)) != 0;
-    if (!ok) break;
-    tc::fence_after_sync();
-
-    // softmax step on row r: max, then p = 2^(s scale log2e - m), sum, P
+  for (int j = 0; j < nkv; ++j) {
+    const int b = j & 1;
+    // the tensor cores start on S_{j+1} while the threads work on S_j (its
+    // buffer was last read by block j - 1's softmax, finished at the last
+    // barrier)
+    if (tid == 0 && ok && j + 1 < nkv) ok = issue_s(j + 1);
+    ok = attn_wait(&bar_s[b], (j >> 1) & 1) && ok;
+    // K_j is consumed: refill its buffer with K_{j+2}
+    if (tid == 0 && ok && j + 2 < nkv) load_k(j + 2);
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05 loads below are warp-wide
     const bool diag = CAUSAL && j == qblk;
-    float mx = -INFINITY;
+    float corr = 1.0f;
+    const uint32_t tS = tmem + lane + b * 128 + wg * 64;
+    const int kbase = wg * 64;  // key index of sr[0] within the block
+    uint32_t sr[64];
+    if (ok) {
+      tc::fence_after_sync();
+      // this warpgroup's 64 columns of the row in registers: two loads, one wait
+      tc::tmem_ld32_async(tS, sr);
+      tc::tmem_ld32_async(tS + 32, sr + 32);
+      tc::tmem_wait_ld();
+      float mx8[8];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tc::tmem_ld32(tS + c * 32, s);
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, (diag && c * 32 + i > r) ? -INFINITY : s[i]);
+      for (int i = 0; i < 64; ++i)
+        mx8[i & 7] = fmaxf(mx8[i & 7], (diag && kbase + i > r) ? -INFINITY : __uint_as_float(sr[i]));
+      xred[wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
     }
-    const float m_new = fmaxf(m_i, mx * scale_log2);
-    const float corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
-    float sum = 0.0f;
+    // both halves of every row's max (every thread reaches this barrier)
+    ok = __syncthreads_and(ok) != 0;
+    if (ok) {
+      const float mx = fmaxf(xred[0][r], xred[1][r]);
+      const float m_new = fmaxf(m_i, mx * scale_log2);
+      corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
+      float sum8[8];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tc::tmem_ld32(tS + c * 32, s);
-      uint32_t w[16];
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
+      // P_j: this warpgroup's keys are chunk wg of the P tile
+      uint8_t* rowp = sP[b] + wg * kChunkBytes + r * 128;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0 = (diag && c * 32 + i > r) ? 0.0f : ex2(fmaf(s[i], scale_log2, -m_new));
-        const float p1 = (diag && c * 32 + i + 1 > r) ? 0.0f : ex2(fmaf(s[i + 1], scale_log2, -m_new));
-        sum += p0 + p1;
-        w[i / 2] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int k0 = c * 32 + i;
+          const float p0 = (diag && kbase + k0 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_new));
+          const float p1 =
+              (diag && kbase + k0 + 1 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_new));
+          sum8[(i >> 1) & 7] += p0 + p1;
+          w[i / 2] = pack_bf16x2(p0, p1);
+        }
+        // keys kbase + c*32 .. +31: 16-byte units c*4 .. c*4+3 of row r, swizzled
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (c * 4 + u) ^ (r & 7);
+          *reinterpret_cast<uint4*>(rowp + unit * 16) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
       }
-      // keys c*32 .. c*32+31: chunk c/2, 16-byte units (c%2)*4 .. +3 of row r, swizzled
-      uint8_t* rowp = sP + (c / 2) * kChunkBytes + r * 128;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int unit = ((c % 2) * 4 + u) ^ (r & 7);
-        *reinterpret_cast<uint4*>(rowp + unit * 16) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-      }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      l_i = fmaf(l_i, corr, sum);
+      m_i = m_new;
     }
-    l_i = fmaf(l_i, corr, sum);
-    m_i = m_new;
-
-    // rescale O when the max grew (warp-uniform decision: tcgen05 ld/st are warp-wide)
-    if (j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+    // O += P_{j-1} V_{j-1} must be complete before O is rescaled; its V
+    // buffer then takes V_{j+1}
+    if (j > 0) {
+      ok = attn_wait(&bar_o, (j - 1) & 1) && ok;
+      if (tid == 0 && ok && j + 1 < nkv) load_v(j + 1);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+      tc::fence_after_sync();
+      uint32_t ov[D / 2];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) tc::tmem_ld32_async(tO + c * 32, ov + c * 32);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
         float v[32];
-        tc::tmem_ld32(tO + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= corr;
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ov[c * 32 + i]) * corr;
         tc::tmem_st32(tO + c * 32, v);
       }
       tc::tmem_wait_st();
     }
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok) break;
 
     // O += P_j V_j: 8 MMAs of K = 16 keys; P K-major, V MN-major (D contiguous)
     if (tid == 0) {
-      tc::fence_after_sync();
+      ok = attn_wait(&bar_v[b], (j >> 1) & 1);
+      if (ok) {
+        tc::fence_after_sync();
+        const uint32_t aP = smem_addr(sP[b]), aV = smem_addr(sV[b]);
 #pragma unroll
-      for (int ks = 0; ks < kAttnBlock / 16; ++ks) {
-        const uint32_t offp = (ks / 4) * kChunkBytes + (ks % 4) * 32;
-        tc::mma_bf16(tmem + 128, tc::smem_desc(aP + offp, 16, 1024), tc::smem_desc(aV + ks * 2048, kChunkBytes, 1024),
-                     IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kAttnBlock / 16; ++ks) {
+          const uint32_t offp = (ks / 4) * kChunkBytes + (ks % 4) * 32;
+          tc::mma_bf16(tmem + 256, tc::smem_desc(aP + offp, 16, 1024),
+                       tc::smem_desc(aV + ks * 2048, kChunkBytes, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&bar_o);
       }
-      tc::mma_commit(&bar_mma);
     }
-    ok = __syncthreads_and(attn_wait(&bar_mma, 1)) != 0;
-    tc::fence_after_sync();
   }
 
+  ok = attn_wait(&bar_o, (nkv - 1) & 1) && ok;
+  xred[wg][r] = l_i;  // the last reads of the maxima were before the loop's last barrier
+  ok = __syncthreads_and(ok) != 0;
   if (ok) {
-    // O / l, rounded to bf16, row r of the block
-    const float inv = 1.0f / l_i;
-    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + r) * D);
+    tc::fence_after_sync();
+    // O / l, rounded to bf16: row r, this warpgroup's half of the columns
+    const float inv = 1.0f / (xred[0][r] + xred[1][r]);
+    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + r) * D + wg * (D / 2));
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       float v[32];
       tc::tmem_ld32(tO + c * 32, v);
 #pragma unroll
@@ -257,11 +331,11 @@ template <int D, bool CAUSAL>
 cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, size_t bh,
                         size_t t, float scale_log2, cudaStream_t s) {
   constexpr uint32_t TILE = (D / 64) * kChunkBytes;
-  const size_t smem = 3 * TILE + 2 * kChunkBytes + 1024;
+  const size_t smem = 5 * TILE + 4 * kChunkBytes + 1024;
   auto kernel = attention_fwd_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(t / kAttnBlock), static_cast<unsigned>(bh));
+  const dim3 grid(static_cast<unsigned>(bh), static_cast<unsigned>(t / kAttnBlock));
   kernel<<<grid, kAttnThreads, smem, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(t),
                                           scale_log2);
   return cudaGetLastError();

@@ -71,6 +71,9 @@ def algorithmic_bytes(op: str, itemsize: int, shape: tuple) -> int:
     softmax (rows in blocks of T = cols queries against T keys) only the kept
     entries are read: row i of a block reads i + 1 of its T values; with
     masked stores skipped, only those are written too."""
+    if op in ("attention", "attention_full"):
+        _, bh, t, d = shape
+        return 4 * bh * t * d * itemsize  # q, k, v read, o written
     if op in ("softmax_causal", "softmax_causal_skip"):
         rows, cols = shape
         full, rem = divmod(rows, cols)
@@ -114,6 +117,11 @@ WORKLOADS = {
                  "gamma ~ 1+N(0,0.1^2), beta ~ N(0,0.1^2); eps 1e-5"),
         Workload("ln_gelu_bf16", "layernorm_gelu", "bf16", (65536, 4096), 7,
                  "bf16 65536x4096, same recipe, then tanh-GELU"),
+        # attention forward: q, k, v stacked as [3, batch*heads, t, d]
+        Workload("attn_causal_bf16", "attention", "bf16", (3, 4 * 16, 2048, 128), 8,
+                 "q, k, v: 4 x 16 heads x 2048 x 128 bf16, N(0,1); causal; scale 1/sqrt(128)"),
+        Workload("attn_bf16", "attention_full", "bf16", (3, 4 * 16, 2048, 128), 9,
+                 "as attn_causal_bf16 without the mask"),
     ]
 }
 
@@ -286,6 +294,10 @@ def make(name: str, threads: int | None = None, rows: int | None = None) -> np.n
         return _cfg2()[:rows]
     if name in ("gelu_bf16", "gelu_erf_bf16"):
         return f32_to_bf16_bits(_cfg2(16777216, seed=5))[:rows]
+    if name in ("attn_causal_bf16", "attn_bf16"):
+        w = WORKLOADS[name]
+        shape = w.shape if rows is None else (3, rows, w.shape[2], w.shape[3])
+        return f32_to_bf16_bits(np.random.default_rng(w.seed).standard_normal(shape, dtype=np.float32))
     if name in ("ln_f32", "ln_gelu_bf16"):
         w = WORKLOADS[name]
         r = rows or w.shape[0]
@@ -368,3 +380,11 @@ def layernorm_params(cols: int, seed: int = 6) -> tuple[np.ndarray, np.ndarray]:
     gamma = (1.0 + 0.1 * g.standard_normal(cols)).astype(np.float32)
     beta = (0.1 * g.standard_normal(cols)).astype(np.float32)
     return gamma, beta
+
+
+def attention_flops(bh: int, t: int, d: int, causal: bool) -> int:
+    """Algorithmic FLOPs of attention forward: 2 d per (query, key) pair for
+    q . k and 2 d for p v, over the unmasked pairs (t (t + 1) / 2 of t^2 per
+    slice when causal)."""
+    pairs = t * (t + 1) // 2 if causal else t * t
+    return 4 * d * bh * pairs
