@@ -5,11 +5,11 @@
 // sum l, rescale the output accumulator when m grows, and divide by l at the
 // end -- the online recurrence of section 7.2 -- so S and P never reach HBM.
 //
-// One CTA of 256 threads per (128-query block, batch*head): two warpgroups
-// that both serve query rows 0..127 (TMEM lanes; warp w reaches lanes
-// 32 (w % 4) ..), warpgroup g taking columns g*64 .. g*64+63 of S and its
-// half of O.  The row max is exchanged once per key block through shared
-// memory; the partial sums are added at the end.
+// One CTA of 288 threads per (128-query block, batch*head): two softmax
+// warpgroups that both serve query rows 0..127 (TMEM lanes; warp w reaches
+// lanes 32 (w % 4) ..), warpgroup g taking columns g*64 .. g*64+63 of S and
+// its half of O, plus one producer warp.  The row max is exchanged once per
+// key block through shared memory; the partial sums are added at the end.
 //   S_j (128 x 128 fp32, TMEM columns (j % 2) * 128 ..) = Q K_j^T   (tcgen05.mma)
 //   O   (128 x D   fp32, TMEM columns 256 ..)          += P_j V_j   (tcgen05.mma)
 // Q, K_j, V_j arrive by TMA in 128-byte-swizzled tiles; P_j is written by the
@@ -18,12 +18,12 @@
 // (tcgen05.commit).  Every mbarrier wait is bounded (1 s); a wait that gives
 // up is counted, the whole CTA stops, frees its TMEM and returns.
 //
-// Pipelining: S is double-buffered in TMEM, so the tensor cores compute
-// S_{j+1} while the threads run the softmax of block j; P is
-// double-buffered in shared memory; K and V each have two buffers and their
-// own barriers, and each buffer is refilled by TMA as soon as the MMA that
-// read it has completed (K after S_j, V after O_{j-1}).  Causal grids hand
-// out the longest query blocks (most key blocks) first.
+// Warp specialisation: a producer warp issues every TMA load and MMA and
+// talks to the softmax warps only through mbarriers (S_j ready, P_j ready,
+// O_j done).  S is double-buffered in TMEM, so the tensor cores compute
+// S_{j+1} while the softmax warps work on block j; K and V each have two
+// buffers, refilled as soon as the MMA that read them has completed.
+// Causal grids hand out the longest query blocks (most key blocks) first.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -40,19 +40,25 @@ __device__ unsigned int g_attn_wait_timeouts = 0;
 
 namespace {
 
-constexpr int kAttnThreads = 256;  // two warpgroups on the same 128 rows
+constexpr int kAttnSoftmaxThreads = 256;  // two warpgroups on the same 128 rows
+constexpr int kAttnThreads = kAttnSoftmaxThreads + 32;  // + the producer warp
 constexpr int kAttnBlock = 128;                // queries per CTA = keys per step
 constexpr uint32_t kChunkBytes = 128 * 128;    // 128 rows x 64 bf16 columns
 constexpr uint32_t kTmemCols = 512;            // S0, S1: 128 columns each; O: up to 128
 constexpr uint64_t kAttnWaitNs = 1000000000ull;
 
-__device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity) {
+// Bounded mbarrier wait.  A wait that gives up (1 s) is counted and raises
+// the CTA's abort flag; every other wait then returns at once, and the CTA
+// skips its remaining work (but not its barriers) and frees its TMEM.
+__device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
     if (global_ns() - t0 > kAttnWaitNs) {
       atomicAdd(&g_attn_wait_timeouts, 1u);
+      *abort = 1;
       return false;
     }
   }
@@ -63,6 +69,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -70,33 +82,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          float scale_log2) {
   constexpr int KC = D / 64;                     // 64-column chunks of a head row
   constexpr uint32_t TILE = KC * kChunkBytes;    // bytes of a 128 x D tile
-  constexpr uint32_t PTILE = 2 * kChunkBytes;    // bytes of a 128 x 128 P tile
   constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_o;
+  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_o, bar_p;
   __shared__ uint32_t tmem_slot;
-  // per-warpgroup row maxima of a key block; at the end, the row sums (the
-  // whole CTA fits the 227 KB of shared memory with ~1 KB to spare at D = 128)
-  __shared__ float xred[2][128];
+  __shared__ int abort_flag;
+  // per-warpgroup row maxima of key block j in xred[j % 2]; at the end, the
+  // row sums
+  __shared__ float xred[2][2][128];
 
-  // Q | K0 | K1 | V0 | V1 | P0 | P1, every tile 1024-byte aligned
+  // Q | K0 | K1 | V0 | V1 | P, every tile 1024-byte aligned
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   uint8_t* sQ = base;
   uint8_t* sK[2] = {base + TILE, base + 2 * TILE};
   uint8_t* sV[2] = {base + 3 * TILE, base + 4 * TILE};
-  uint8_t* sP[2] = {base + 5 * TILE, base + 5 * TILE + PTILE};
-  const uint32_t aQ = smem_addr(sQ);
+  uint8_t* sP = base + 5 * TILE;  // 2 chunks: keys 0..63, 64..127
+  const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int wg = warp >> 2;                        // warpgroup: S columns wg*64.., O columns wg*D/2..
-  const int r = ((warp & 3) << 5) | (tid & 31);    // query row = TMEM lane
   const int slice = blockIdx.x;
   const int nq = static_cast<int>(gridDim.y);
   const int qblk = CAUSAL ? nq - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
   const int row0 = slice * t + qblk * kAttnBlock;  // first query row in the [bh * t, D] view
   const int nkv = CAUSAL ? qblk + 1 : t / kAttnBlock;
+  volatile int* abort = &abort_flag;
 
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
   if (tid == 0) {
@@ -107,157 +118,70 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bar_s[i], 1);
     }
     mbar_init(&bar_o, 1);
+    mbar_init(&bar_p, kAttnSoftmaxThreads);
+    abort_flag = 0;
     fence_mbarrier_init();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = tmem_slot;                        // S0 | S1 | O
-  const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tO = tmem + lane + 256 + wg * (D / 2);
+  const uint32_t tmem = tmem_slot;  // S0 | S1 | O
 
-  // producer side, thread 0 only
-  auto load_k = [&](int j) {
-    const int b = j & 1;
-    mbar_arrive_expect_tx(&bar_k[b], TILE);
+  if (warp == kAttnSoftmaxThreads / 32) {
+    // ------------------------------------------------ producer warp: TMA and MMA issue
+    if ((tid & 31) == 0) {
+      auto load_k = [&](int j) {
+        const int b = j & 1;
+        mbar_arrive_expect_tx(&bar_k[b], TILE);
 #pragma unroll
-    for (int c = 0; c < KC; ++c) tc::tma_load_2d(sK[b] + c * kChunkBytes, &tmk, &bar_k[b], c * 64, slice * t + j * 128);
-  };
-  auto load_v = [&](int j) {
-    const int b = j & 1;
-    mbar_arrive_expect_tx(&bar_v[b], TILE);
+        for (int c = 0; c < KC; ++c)
+          tc::tma_load_2d(sK[b] + c * kChunkBytes, &tmk, &bar_k[b], c * 64, slice * t + j * 128);
+      };
+      auto load_v = [&](int j) {
+        const int b = j & 1;
+        mbar_arrive_expect_tx(&bar_v[b], TILE);
 #pragma unroll
-    for (int c = 0; c < KC; ++c) tc::tma_load_2d(sV[b] + c * kChunkBytes, &tmv, &bar_v[b], c * 64, slice * t + j * 128);
-  };
-  // S_j = Q K_j^T into TMEM columns (j & 1) * 128, once K_j has landed
-  auto issue_s = [&](int j) -> bool {
-    const int b = j & 1;
-    if (!attn_wait(&bar_k[b], (j >> 1) & 1)) return false;
-    tc::fence_after_sync();
-    const uint32_t aK = smem_addr(sK[b]);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t off = (ks / 4) * kChunkBytes + (ks % 4) * 32;
-      tc::mma_bf16(tmem + b * 128, tc::smem_desc(aQ + off, 16, 1024), tc::smem_desc(aK + off, 16, 1024), IDESC_S,
-                   ks > 0 ? 1u : 0u);
-    }
-    tc::mma_commit(&bar_s[b]);
-    return true;
-  };
-
-  bool ok = true;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar_q, TILE);
-#pragma unroll
-    for (int c = 0; c < KC; ++c) tc::tma_load_2d(sQ + c * kChunkBytes, &tmq, &bar_q, c * 64, row0);
-    load_k(0);
-    load_v(0);
-    if (nkv > 1) {
-      load_k(1);
-      load_v(1);
-    }
-    ok = attn_wait(&bar_q, 0) && issue_s(0);
-  }
-  float m_i = -INFINITY, l_i = 0.0f;
-
-  for (int j = 0; j < nkv; ++j) {
-    const int b = j & 1;
-    // the tensor cores start on S_{j+1} while the threads work on S_j (its
-    // buffer was last read by block j - 1's softmax, finished at the last
-    // barrier)
-    if (tid == 0 && ok && j + 1 < nkv) ok = issue_s(j + 1);
-    ok = attn_wait(&bar_s[b], (j >> 1) & 1) && ok;
-    // K_j is consumed: refill its buffer with K_{j+2}
-    if (tid == 0 && ok && j + 2 < nkv) load_k(j + 2);
-    ok = __all_sync(0xffffffffu, ok);  // tcgen05 loads below are warp-wide
-    const bool diag = CAUSAL && j == qblk;
-    float corr = 1.0f;
-    const uint32_t tS = tmem + lane + b * 128 + wg * 64;
-    const int kbase = wg * 64;  // key index of sr[0] within the block
-    uint32_t sr[64];
-    if (ok) {
-      tc::fence_after_sync();
-      // this warpgroup's 64 columns of the row in registers: two loads, one wait
-      tc::tmem_ld32_async(tS, sr);
-      tc::tmem_ld32_async(tS + 32, sr + 32);
-      tc::tmem_wait_ld();
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        mx8[i & 7] = fmaxf(mx8[i & 7], (diag && kbase + i > r) ? -INFINITY : __uint_as_float(sr[i]));
-      xred[wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-    }
-    // both halves of every row's max (every thread reaches this barrier)
-    ok = __syncthreads_and(ok) != 0;
-    if (ok) {
-      const float mx = fmaxf(xred[0][r], xred[1][r]);
-      const float m_new = fmaxf(m_i, mx * scale_log2);
-      corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
-      float sum8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
-      // P_j: this warpgroup's keys are chunk wg of the P tile
-      uint8_t* rowp = sP[b] + wg * kChunkBytes + r * 128;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int k0 = c * 32 + i;
-          const float p0 = (diag && kbase + k0 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_new));
-          const float p1 =
-              (diag && kbase + k0 + 1 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_new));
-          sum8[(i >> 1) & 7] += p0 + p1;
-          w[i / 2] = pack_bf16x2(p0, p1);
-        }
-        // keys kbase + c*32 .. +31: 16-byte units c*4 .. c*4+3 of row r, swizzled
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (c * 4 + u) ^ (r & 7);
-          *reinterpret_cast<uint4*>(rowp + unit * 16) =
-              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
-      }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      l_i = fmaf(l_i, corr, sum);
-      m_i = m_new;
-    }
-    // O += P_{j-1} V_{j-1} must be complete before O is rescaled; its V
-    // buffer then takes V_{j+1}
-    if (j > 0) {
-      ok = attn_wait(&bar_o, (j - 1) & 1) && ok;
-      if (tid == 0 && ok && j + 1 < nkv) load_v(j + 1);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
-      tc::fence_after_sync();
-      uint32_t ov[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) tc::tmem_ld32_async(tO + c * 32, ov + c * 32);
-      tc::tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ov[c * 32 + i]) * corr;
-        tc::tmem_st32(tO + c * 32, v);
-      }
-      tc::tmem_wait_st();
-    }
-    tc::fence_proxy_async_smem();
-    tc::fence_before_sync();
-    ok = __syncthreads_and(ok) != 0;
-    if (!ok) break;
-
-    // O += P_j V_j: 8 MMAs of K = 16 keys; P K-major, V MN-major (D contiguous)
-    if (tid == 0) {
-      ok = attn_wait(&bar_v[b], (j >> 1) & 1);
-      if (ok) {
+        for (int c = 0; c < KC; ++c)
+          tc::tma_load_2d(sV[b] + c * kChunkBytes, &tmv, &bar_v[b], c * 64, slice * t + j * 128);
+      };
+      // S_j = Q K_j^T into TMEM columns (j % 2) * 128
+      auto issue_s = [&](int j) {
+        const int b = j & 1;
+        if (!attn_wait(&bar_k[b], (j >> 1) & 1, abort)) return;
         tc::fence_after_sync();
-        const uint32_t aP = smem_addr(sP[b]), aV = smem_addr(sV[b]);
+        const uint32_t aK = smem_addr(sK[b]);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks / 4) * kChunkBytes + (ks % 4) * 32;
+          tc::mma_bf16(tmem + b * 128, tc::smem_desc(aQ + off, 16, 1024), tc::smem_desc(aK + off, 16, 1024),
+                       IDESC_S, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&bar_s[b]);
+      };
+      mbar_arrive_expect_tx(&bar_q, TILE);
+#pragma unroll
+      for (int c = 0; c < KC; ++c) tc::tma_load_2d(sQ + c * kChunkBytes, &tmq, &bar_q, c * 64, row0);
+      load_k(0);
+      load_v(0);
+      if (nkv > 1) {
+        load_k(1);
+        load_v(1);
+      }
+      if (attn_wait(&bar_q, 0, abort)) issue_s(0);
+      for (int j = 0; j < nkv && !*abort; ++j) {
+        const int b = j & 1;
+        // S_{j+1}: its TMEM buffer was last read by softmax j - 1 (bar_p below)
+        if (j + 1 < nkv) issue_s(j + 1);
+        // K_j consumed once S_j is done: refill with K_{j+2}
+        if (!attn_wait(&bar_s[b], (j >> 1) & 1, abort)) break;
+        if (j + 2 < nkv) load_k(j + 2);
+        // softmax j done: P_j written, S_j read, O rescaled (after O_{j-1}
+        // completed, so V_{j-1}'s buffer is free for V_{j+1})
+        if (!attn_wait(&bar_p, j & 1, abort)) break;
+        if (j >= 1 && j + 1 < nkv) load_v(j + 1);
+        if (!attn_wait(&bar_v[b], (j >> 1) & 1, abort)) break;
+        tc::fence_after_sync();
+        const uint32_t aV = smem_addr(sV[b]);
 #pragma unroll
         for (int ks = 0; ks < kAttnBlock / 16; ++ks) {
           const uint32_t offp = (ks / 4) * kChunkBytes + (ks % 4) * 32;
@@ -267,26 +191,116 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc::mma_commit(&bar_o);
       }
     }
-  }
-
-  ok = attn_wait(&bar_o, (nkv - 1) & 1) && ok;
-  xred[wg][r] = l_i;  // the last reads of the maxima were before the loop's last barrier
-  ok = __syncthreads_and(ok) != 0;
-  if (ok) {
-    tc::fence_after_sync();
-    // O / l, rounded to bf16: row r, this warpgroup's half of the columns
-    const float inv = 1.0f / (xred[0][r] + xred[1][r]);
-    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + r) * D + wg * (D / 2));
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ softmax warpgroups
+    // Both warpgroups serve query rows 0..127 (TMEM lanes; warp w reaches
+    // lanes 32 (w % 4) ..); warpgroup g takes S columns g*64 .. g*64+63 and
+    // O columns g*D/2 .. .  Every thread executes every named barrier and
+    // every arrival, whatever happens, so no barrier can strand a warp.
+    const int wg = warp >> 2;
+    const int r = ((warp & 3) << 5) | (tid & 31);
+    const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + lane + 256 + wg * (D / 2);
+    const int kbase = wg * 64;
+    float m_i = -INFINITY, l_i = 0.0f;
+    for (int j = 0; j < nkv; ++j) {
+      const int b = j & 1;
+      const bool diag = CAUSAL && j == qblk;
+      attn_wait(&bar_s[b], (j >> 1) & 1, abort);
+      uint32_t sr[64];
+      if (!__any_sync(0xffffffffu, *abort)) {
+        tc::fence_after_sync();
+        const uint32_t tS = tmem + lane + b * 128 + kbase;
+        tc::tmem_ld32_async(tS, sr);
+        tc::tmem_ld32_async(tS + 32, sr + 32);
+        tc::tmem_wait_ld();
+        float mx8[8];
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      float v[32];
-      tc::tmem_ld32(tO + c * 32, v);
+        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        dst[c * 4 + q] = make_uint4(pack_bf16x2(v[8 * q] * inv, v[8 * q + 1] * inv),
-                                    pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv),
-                                    pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
-                                    pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
+        for (int i = 0; i < 64; ++i)
+          mx8[i & 7] = fmaxf(mx8[i & 7], (diag && kbase + i > r) ? -INFINITY : __uint_as_float(sr[i]));
+        xred[b][wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      }
+      softmax_bar();  // both halves of every row's max of block j
+      float corr = 1.0f;
+      // O_{j-1} complete: P's buffer and O may be touched
+      if (j > 0) attn_wait(&bar_o, (j - 1) & 1, abort);
+      if (!__any_sync(0xffffffffu, *abort)) {
+        const float mx = fmaxf(xred[b][0][r], xred[b][1][r]);
+        const float m_new = fmaxf(m_i, mx * scale_log2);
+        corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
+        float sum8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
+        uint8_t* rowp = sP + wg * kChunkBytes + r * 128;  // this warpgroup's keys: chunk wg of P
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int k0 = c * 32 + i;
+            const float p0 =
+                (diag && kbase + k0 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_new));
+            const float p1 =
+                (diag && kbase + k0 + 1 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_new));
+            sum8[(i >> 1) & 7] += p0 + p1;
+            w[i / 2] = pack_bf16x2(p0, p1);
+          }
+          // keys kbase + c*32 .. +31: 16-byte units c*4 .. c*4+3 of row r, swizzled
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int unit = (c * 4 + u) ^ (r & 7);
+            *reinterpret_cast<uint4*>(rowp + unit * 16) =
+                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+        l_i = fmaf(l_i, corr, ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
+        m_i = m_new;
+        if (j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+          tc::fence_after_sync();
+          uint32_t ov[D / 2];
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tc::tmem_ld32_async(tO + c * 32, ov + c * 32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ov[c * 32 + i]) * corr;
+            tc::tmem_st32(tO + c * 32, v);
+          }
+          tc::tmem_wait_st();
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(&bar_p);
+    }
+    attn_wait(&bar_o, (nkv - 1) & 1, abort);
+    // the row sums go to the buffer the last key block did not use: its last
+    // readers finished before the previous named barrier
+    const int e = nkv & 1;
+    xred[e][wg][r] = l_i;
+    softmax_bar();
+    if (!__any_sync(0xffffffffu, *abort)) {
+      tc::fence_after_sync();
+      // O / l, rounded to bf16: row r, this warpgroup's half of the columns
+      const float inv = 1.0f / (xred[e][0][r] + xred[e][1][r]);
+      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + r) * D + wg * (D / 2));
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        float v[32];
+        tc::tmem_ld32(tO + c * 32, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[c * 4 + q] = make_uint4(pack_bf16x2(v[8 * q] * inv, v[8 * q + 1] * inv),
+                                      pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv),
+                                      pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
+                                      pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
+      }
     }
   }
   tc::fence_before_sync();
@@ -331,7 +345,7 @@ template <int D, bool CAUSAL>
 cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, size_t bh,
                         size_t t, float scale_log2, cudaStream_t s) {
   constexpr uint32_t TILE = (D / 64) * kChunkBytes;
-  const size_t smem = 5 * TILE + 4 * kChunkBytes + 1024;
+  const size_t smem = 5 * TILE + 2 * kChunkBytes + 1024;
   auto kernel = attention_fwd_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
