@@ -163,10 +163,33 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
-def csrc_digest() -> str:
+# Sources each kernel family is compiled from (its profile stays valid while
+# these are unchanged).
+_FAMILY_SOURCES = {
+    "gelu": ["fk_gelu.cu", "fk_gelu.cuh", "fk_common.cuh"],
+    "softmax": ["fk_softmax.cu", "fk_rows.cuh", "fk_common.cuh", "fk_sync.cuh", "fk_plan.cpp"],
+    "layernorm": ["fk_layernorm.cu", "fk_rows.cuh", "fk_common.cuh", "fk_gelu.cuh", "fk_plan.cpp"],
+    "attention": ["fk_attention.cu", "fk_tc.cuh", "fk_sync.cuh", "fk_common.cuh"],
+}
+
+
+def kernel_family(op: str) -> str:
+    for fam in ("gelu", "softmax", "layernorm", "attention"):
+        if op.startswith(fam):
+            return fam
+    raise KeyError(op)
+
+
+def csrc_digest(family: str | None = None) -> str:
+    """Digest of the kernel sources of one family (all of csrc/ if None),
+    with the shared internal header and the public header."""
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "memory_bound_fk_b200", "csrc", "*"))) + \
-        [os.path.join(ROOT, "include", "fk.h")]
+    csrc = os.path.join(ROOT, "memory_bound_fk_b200", "csrc")
+    if family is None:
+        files = sorted(glob.glob(os.path.join(csrc, "*")))
+    else:
+        files = [os.path.join(csrc, f) for f in _FAMILY_SOURCES[family] + ["fk_internal.h"]]
+    files.append(os.path.join(ROOT, "include", "fk.h"))
     for p in files:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
@@ -176,8 +199,9 @@ def csrc_digest() -> str:
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch recorded by an ncu capture in profiles/, if the
-    kernel sources have not changed since (else None)."""
-    digest = csrc_digest()
+    kernel family's sources have not changed since (else None)."""
+    from memory_bound_fk_b200 import synth
+    digest = csrc_digest(kernel_family(synth.WORKLOADS[workload].op))
     for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         text = open(p).read()
         for m in re.finditer(r"traffic:\s*workload=(\w+)\s+bytes_per_launch=(\d+)\s+csrc=(\w+)", text):

@@ -112,3 +112,18 @@ def test_tensor_wrapper_against_torch_sdpa(fk, torch_mod):
     o = fk.attention(q, k, v, causal=True)
     ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(), is_causal=True)
     assert torch.max(torch.abs(o.float() - ref)).item() <= 2e-2
+
+
+@pytest.mark.parametrize("name", ["attn_causal_bf16", "attn_bf16"])
+def test_bench_workloads_full_size(fk, torch_mod, name):
+    """The attention bench workloads at full size (4 x 16 heads of 2048 x 128)
+    in the launch bench.py times: sampled slices against the oracle."""
+    from memory_bound_fk_b200 import synth
+    w = synth.WORKLOADS[name]
+    causal = w.op == "attention"
+    qkv = synth.make(name)
+    _, bh, t, d = qkv.shape
+    scale = 1.0 / math.sqrt(d)
+    o = run(fk, torch_mod, qkv[0], qkv[1], qkv[2], causal, scale)
+    for sl in (0, bh - 1):
+        check(o[sl:sl + 1], qkv[0, sl:sl + 1], qkv[1, sl:sl + 1], qkv[2, sl:sl + 1], causal, scale)
