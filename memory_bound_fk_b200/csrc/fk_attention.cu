@@ -54,7 +54,7 @@ __device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;  // suspended up to 20 us per try
     if (*abort) return false;
     if (global_ns() - t0 > kAttnWaitNs) {
       atomicAdd(&g_attn_wait_timeouts, 1u);
@@ -73,6 +73,88 @@ __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" 
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// One key block of a softmax warpgroup thread (row r, columns kbase ..
+// kbase+63 of S_j in TMEM buffer b): the row max (exchanged with the other
+// warpgroup), p = 2^(s scale log2e - m) written to P as bf16, the running
+// max and sum, and O rescaled when the max grew (after O_{j-1} completed).
+// diag: the causal grid's diagonal block, whose keys after the query are
+// set to -inf in registers first (exp gives 0), so the common body carries
+// no per-element mask.  Every thread executes the named barrier whatever
+// `abort` says.
+template <int D>
+__device__ __forceinline__ void softmax_step(uint32_t tmem, uint32_t lane, uint32_t tO, int b, int kbase, int r,
+                                             int wg, int j, bool diag, uint8_t* sP, float (*xred)[2][128],
+                                             uint64_t* bar_o, float scale_log2, volatile int* abort, float& m_i,
+                                             float& l_i) {
+  uint32_t sr[64];
+  if (!__any_sync(0xffffffffu, *abort)) {
+    tc::fence_after_sync();
+    const uint32_t tS = tmem + lane + b * 128 + kbase;
+    tc::tmem_ld32_async(tS, sr);
+    tc::tmem_ld32_async(tS + 32, sr + 32);
+    tc::tmem_wait_ld();
+    if (diag) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) sr[i] = (kbase + i > r) ? 0xff800000u : sr[i];
+    }
+    float mx8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i]));
+    xred[b][wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+  }
+  softmax_bar();  // both halves of every row's max of block j
+  float corr = 1.0f;
+  if (j > 0) attn_wait(bar_o, (j - 1) & 1, abort);
+  if (!__any_sync(0xffffffffu, *abort)) {
+    const float mx = fmaxf(xred[b][0][r], xred[b][1][r]);
+    const float m_new = fmaxf(m_i, mx * scale_log2);
+    corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
+    float sum8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
+    uint8_t* rowp = sP + wg * kChunkBytes + r * 128;  // this warpgroup's keys: chunk wg of P
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const int k0 = c * 32 + i;
+        const float p0 = ex2(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_new));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_new));
+        sum8[(i >> 1) & 7] += p0 + p1;
+        w[i / 2] = pack_bf16x2(p0, p1);
+      }
+      // keys kbase + c*32 .. +31: 16-byte units c*4 .. c*4+3 of row r, swizzled
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int unit = (c * 4 + u) ^ (r & 7);
+        *reinterpret_cast<uint4*>(rowp + unit * 16) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+    }
+    l_i = fmaf(l_i, corr, ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
+    m_i = m_new;
+    if (j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+      tc::fence_after_sync();
+      uint32_t ov[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tc::tmem_ld32_async(tO + c * 32, ov + c * 32);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ov[c * 32 + i]) * corr;
+        tc::tmem_st32(tO + c * 32, v);
+      }
+      tc::tmem_wait_st();
+    }
+  }
 }
 
 template <int D, bool CAUSAL>
@@ -208,73 +290,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int b = j & 1;
       const bool diag = CAUSAL && j == qblk;
       attn_wait(&bar_s[b], (j >> 1) & 1, abort);
-      uint32_t sr[64];
-      if (!__any_sync(0xffffffffu, *abort)) {
-        tc::fence_after_sync();
-        const uint32_t tS = tmem + lane + b * 128 + kbase;
-        tc::tmem_ld32_async(tS, sr);
-        tc::tmem_ld32_async(tS + 32, sr + 32);
-        tc::tmem_wait_ld();
-        float mx8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          mx8[i & 7] = fmaxf(mx8[i & 7], (diag && kbase + i > r) ? -INFINITY : __uint_as_float(sr[i]));
-        xred[b][wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      }
-      softmax_bar();  // both halves of every row's max of block j
-      float corr = 1.0f;
-      // O_{j-1} complete: P's buffer and O may be touched
-      if (j > 0) attn_wait(&bar_o, (j - 1) & 1, abort);
-      if (!__any_sync(0xffffffffu, *abort)) {
-        const float mx = fmaxf(xred[b][0][r], xred[b][1][r]);
-        const float m_new = fmaxf(m_i, mx * scale_log2);
-        corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
-        float sum8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
-        uint8_t* rowp = sP + wg * kChunkBytes + r * 128;  // this warpgroup's keys: chunk wg of P
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int k0 = c * 32 + i;
-            const float p0 =
-                (diag && kbase + k0 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0]), scale_log2, -m_new));
-            const float p1 =
-                (diag && kbase + k0 + 1 > r) ? 0.0f : ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale_log2, -m_new));
-            sum8[(i >> 1) & 7] += p0 + p1;
-            w[i / 2] = pack_bf16x2(p0, p1);
-          }
-          // keys kbase + c*32 .. +31: 16-byte units c*4 .. c*4+3 of row r, swizzled
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int unit = (c * 4 + u) ^ (r & 7);
-            *reinterpret_cast<uint4*>(rowp + unit * 16) =
-                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-          }
-        }
-        l_i = fmaf(l_i, corr, ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
-        m_i = m_new;
-        if (j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
-          tc::fence_after_sync();
-          uint32_t ov[D / 2];
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) tc::tmem_ld32_async(tO + c * 32, ov + c * 32);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ov[c * 32 + i]) * corr;
-            tc::tmem_st32(tO + c * 32, v);
-          }
-          tc::tmem_wait_st();
-        }
-      }
+      // the causal mask only touches the diagonal block: the other blocks
+      // take the unmasked body (no per-element tests)
+      softmax_step<D>(tmem, lane, tO, b, kbase, r, wg, j, diag, sP, xred, &bar_o, scale_log2, abort, m_i, l_i);
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(&bar_p);
