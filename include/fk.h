@@ -341,7 +341,8 @@ FK_API fk_status fk_layernorm_rows_ex(const void *x, void *y, const float *gamma
  * memory and shared memory), with the running max / sum of section 7.2.
  *   q, k, v  [bh, t, d] bf16, contiguous, device memory, 16-byte aligned.
  *   o        [bh, t, d] bf16 output; must not overlap q, k or v.
- *   t        a multiple of 128 (queries and keys per slice); d = 64 or 128.
+ *   t        a multiple of 128, at most 128 * 65535 (queries and keys per
+ *            slice); d = 64 or 128.
  *   causal   0 or 1.
  *   scale    finite, > 0 (e.g. 1 / sqrt(d)).
  * Arithmetic: S and the O accumulator in fp32 (tcgen05, TMEM), P rounded to

@@ -75,17 +75,23 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Growth of a row's max (log2 units) that the running reference may lag
+// behind: the exponentials are then at most 2^8, and O is rescaled only
+// when the max outgrows the reference by more than that.
+constexpr float kLazyRescale = 8.0f;
+
 // One key block of a softmax warpgroup thread (row r, columns kbase ..
 // kbase+63 of S_j in TMEM buffer b): the row max (exchanged with the other
-// warpgroup), p = 2^(s scale log2e - m) written to P as bf16, the running
-// max and sum, and O rescaled when the max grew (after O_{j-1} completed).
-// diag: the causal grid's diagonal block, whose keys after the query are
-// set to -inf in registers first (exp gives 0), so the common body carries
-// no per-element mask.  Every thread executes the named barrier whatever
-// `abort` says.
+// warpgroup), the reference max m (moved only when the block's max exceeds
+// it by more than kLazyRescale, the same decision in both warpgroups),
+// p = 2^(s scale log2e - m) written to P_j as bf16, the running sum, and O
+// rescaled when m moved (after O_{j-1} completed).  diag: the causal grid's
+// diagonal block, whose keys after the query are set to -inf in registers
+// first (exp gives 0), so the common body carries no per-element mask.
+// Every thread executes both named barriers whatever `abort` says.
 template <int D>
 __device__ __forceinline__ void softmax_step(uint32_t tmem, uint32_t lane, uint32_t tO, int b, int kbase, int r,
-                                             int wg, int j, bool diag, uint8_t* sP, float (*xred)[2][128],
+                                             int wg, int j, bool diag, uint8_t* sPb, float (*xred)[128],
                                              uint64_t* bar_o, float scale_log2, volatile int* abort, float& m_i,
                                              float& l_i) {
   uint32_t sr[64];
@@ -103,22 +109,23 @@ __device__ __forceinline__ void softmax_step(uint32_t tmem, uint32_t lane, uint3
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
-      mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i]));
-    xred[b][wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i]));
+    xred[wg][r] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
   }
   softmax_bar();  // both halves of every row's max of block j
-  float corr = 1.0f;
-  if (j > 0) attn_wait(bar_o, (j - 1) & 1, abort);
+  const float mx = fmaxf(xred[0][r], xred[1][r]) * scale_log2;
+  softmax_bar();  // every read is done before the next block's writes
+  const bool upd = mx > m_i + kLazyRescale;  // always for the first block (m_i = -inf)
+  const float m_new = upd ? mx : m_i;
+  const float corr = upd ? ex2(m_i - m_new) : 1.0f;
+  // P_j's buffer was last read by O_{j-2}
+  if (j >= 2) attn_wait(&bar_o[b], ((j - 2) >> 1) & 1, abort);
   if (!__any_sync(0xffffffffu, *abort)) {
-    const float mx = fmaxf(xred[b][0][r], xred[b][1][r]);
-    const float m_new = fmaxf(m_i, mx * scale_log2);
-    corr = ex2(m_i - m_new);  // 0 for the first block (m_i = -inf)
     float sum8[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
-    uint8_t* rowp = sP + wg * kChunkBytes + r * 128;  // this warpgroup's keys: chunk wg of P
+    uint8_t* rowp = sPb + wg * kChunkBytes + r * 128;  // this warpgroup's keys: chunk wg of P_j
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       uint32_t w[16];
@@ -139,7 +146,11 @@ __device__ __forceinline__ void softmax_step(uint32_t tmem, uint32_t lane, uint3
     }
     l_i = fmaf(l_i, corr, ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
     m_i = m_new;
-    if (j > 0 && __any_sync(0xffffffffu, corr != 1.0f)) {
+  }
+  // O rescale (rare): O_{j-1} must be complete first
+  if (j > 0 && __any_sync(0xffffffffu, upd)) {
+    attn_wait(&bar_o[(j - 1) & 1], ((j - 1) >> 1) & 1, abort);
+    if (!__any_sync(0xffffffffu, *abort)) {
       tc::fence_after_sync();
       uint32_t ov[D / 2];
 #pragma unroll
@@ -168,20 +179,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_o, bar_p;
+  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_o[2], bar_p[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  // per-warpgroup row maxima of key block j in xred[j % 2]; at the end, the
-  // row sums
-  __shared__ float xred[2][2][128];
+  // per-warpgroup row maxima of a key block; at the end, the row sums (the
+  // CTA fits the 227 KB of shared memory with ~0.9 KB to spare at D = 128)
+  __shared__ float xred[2][128];
 
-  // Q | K0 | K1 | V0 | V1 | P, every tile 1024-byte aligned
+  // Q | K0 | K1 | V0 | V1 | P0 | P1, every tile 1024-byte aligned
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   uint8_t* sQ = base;
   uint8_t* sK[2] = {base + TILE, base + 2 * TILE};
   uint8_t* sV[2] = {base + 3 * TILE, base + 4 * TILE};
-  uint8_t* sP = base + 5 * TILE;  // 2 chunks: keys 0..63, 64..127
-  const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP);
+  uint8_t* sP[2] = {base + 5 * TILE, base + 5 * TILE + 2 * kChunkBytes};  // 2 chunks each: keys 0..63, 64..127
+  const uint32_t aQ = smem_addr(sQ);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int slice = blockIdx.x;
@@ -198,9 +209,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
       mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_o[i], 1);
+      mbar_init(&bar_p[i], kAttnSoftmaxThreads);
     }
-    mbar_init(&bar_o, 1);
-    mbar_init(&bar_p, kAttnSoftmaxThreads);
     abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -257,20 +268,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // K_j consumed once S_j is done: refill with K_{j+2}
         if (!attn_wait(&bar_s[b], (j >> 1) & 1, abort)) break;
         if (j + 2 < nkv) load_k(j + 2);
-        // softmax j done: P_j written, S_j read, O rescaled (after O_{j-1}
-        // completed, so V_{j-1}'s buffer is free for V_{j+1})
-        if (!attn_wait(&bar_p, j & 1, abort)) break;
-        if (j >= 1 && j + 1 < nkv) load_v(j + 1);
+        // softmax j done: P_j written, S_j read, O rescaled if needed (two
+        // barriers: without a rescale, softmax j+1 may finish before this
+        // wait, but softmax j+2 needs S_{j+2}, issued after it)
+        if (!attn_wait(&bar_p[b], (j >> 1) & 1, abort)) break;
         if (!attn_wait(&bar_v[b], (j >> 1) & 1, abort)) break;
         tc::fence_after_sync();
-        const uint32_t aV = smem_addr(sV[b]);
+        const uint32_t aV = smem_addr(sV[b]), aP = smem_addr(sP[b]);
 #pragma unroll
         for (int ks = 0; ks < kAttnBlock / 16; ++ks) {
           const uint32_t offp = (ks / 4) * kChunkBytes + (ks % 4) * 32;
           tc::mma_bf16(tmem + 256, tc::smem_desc(aP + offp, 16, 1024),
                        tc::smem_desc(aV + ks * 2048, kChunkBytes, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
         }
-        tc::mma_commit(&bar_o);
+        tc::mma_commit(&bar_o[b]);
+        // V_{j+1} goes to the buffer of V_{j-1}, free once O_{j-1} is done
+        if (j >= 1 && j + 1 < nkv) {
+          if (!attn_wait(&bar_o[(j - 1) & 1], ((j - 1) >> 1) & 1, abort)) break;
+          load_v(j + 1);
+        }
       }
     }
     __syncwarp();
@@ -292,21 +308,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       attn_wait(&bar_s[b], (j >> 1) & 1, abort);
       // the causal mask only touches the diagonal block: the other blocks
       // take the unmasked body (no per-element tests)
-      softmax_step<D>(tmem, lane, tO, b, kbase, r, wg, j, diag, sP, xred, &bar_o, scale_log2, abort, m_i, l_i);
+      softmax_step<D>(tmem, lane, tO, b, kbase, r, wg, j, diag, sP[b], xred, bar_o, scale_log2, abort, m_i, l_i);
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
-      mbar_arrive(&bar_p);
+      mbar_arrive(&bar_p[b]);
     }
-    attn_wait(&bar_o, (nkv - 1) & 1, abort);
-    // the row sums go to the buffer the last key block did not use: its last
-    // readers finished before the previous named barrier
-    const int e = nkv & 1;
-    xred[e][wg][r] = l_i;
+    attn_wait(&bar_o[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort);
+    xred[wg][r] = l_i;  // the last reads of the maxima were before the last named barrier
     softmax_bar();
     if (!__any_sync(0xffffffffu, *abort)) {
       tc::fence_after_sync();
       // O / l, rounded to bf16: row r, this warpgroup's half of the columns
-      const float inv = 1.0f / (xred[e][0][r] + xred[e][1][r]);
+      const float inv = 1.0f / (xred[0][r] + xred[1][r]);
       uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + r) * D + wg * (D / 2));
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
@@ -363,7 +376,7 @@ template <int D, bool CAUSAL>
 cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, size_t bh,
                         size_t t, float scale_log2, cudaStream_t s) {
   constexpr uint32_t TILE = (D / 64) * kChunkBytes;
-  const size_t smem = 5 * TILE + 2 * kChunkBytes + 1024;
+  const size_t smem = 5 * TILE + 4 * kChunkBytes + 1024;
   auto kernel = attention_fwd_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;

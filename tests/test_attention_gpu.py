@@ -76,6 +76,27 @@ def test_score_ranges(fk, torch_mod, sigma, scale):
     check(run(fk, torch_mod, q, k, v, True, scale), q, k, v, True, scale)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("delta", [-4.0, 3.0, 7.9, 12.0])
+def test_running_max_ramps(fk, torch_mod, delta, causal):
+    """Scores that rise (or fall) along the keys by `delta` log2 units per
+    128-key block: the running max grows a little every block (the output
+    is rescaled only once it has outgrown the last rescale by more than
+    2^8), by more than that every block, or never after the first."""
+    bh, t, d = 2, 1024, 64
+    scale = 0.125
+    g = np.random.default_rng(int(delta * 10) + 100 + 7 * causal)
+    q = np.zeros((bh, t, d))
+    q[..., 0] = 1.0
+    q[..., 1:] = 0.05 * g.standard_normal((bh, t, d - 1))
+    k = 0.05 * g.standard_normal((bh, t, d))
+    k[..., 0] = delta / (scale * math.log2(math.e)) * (np.arange(t) / 128.0) + 0.3 * g.standard_normal((bh, t))
+    v = g.standard_normal((bh, t, d))
+    q, k, v = (oracle.round_to_bf16(a) for a in (q, k, v))
+    check(run(fk, torch_mod, q, k, v, causal, scale), q, k, v, causal, scale)
+    assert fk.fk_wait_timeouts(reset=True) == 0
+
+
 def test_constant_values_and_first_row(fk, torch_mod):
     """With every value row equal, every output row is that row; causal row
     0 sees key 0 only."""
