@@ -60,7 +60,8 @@ def inputs(bh, t, d, seed, sigma=1.0):
 
 @pytest.mark.parametrize("bh,t,d,causal", [(1, 128, 64, False), (1, 128, 64, True), (2, 256, 64, True),
                                             (2, 256, 128, False), (3, 384, 128, True), (2, 512, 64, False),
-                                            (1, 1024, 128, True), (4, 256, 128, True)])
+                                            (1, 1024, 128, True), (4, 256, 128, True), (2, 384, 64, False),
+                                            (1, 640, 128, True), (3, 128, 128, True)])
 def test_parity(fk, torch_mod, bh, t, d, causal):
     q, k, v = inputs(bh, t, d, seed=bh * 1000 + t + d)
     scale = 1.0 / math.sqrt(d)
