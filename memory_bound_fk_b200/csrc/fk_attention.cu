@@ -5,22 +5,27 @@
 // sum l, rescale the output accumulator when m grows, and divide by l at the
 // end -- the online recurrence of section 7.2 -- so S and P never reach HBM.
 //
-// One CTA of 288 threads per (pair of 128-query blocks, batch*head): one
+// One CTA of 384 threads per (pair of 128-query blocks, batch*head): one
 // softmax warpgroup per query tile (thread r owns row r of its tile: TMEM
 // lane r, the whole 128-key row of S in registers, so the row max needs no
-// exchange), plus one producer warp.  Each K_j, V_j tile brought into
-// shared memory serves both query tiles.
+// exchange), and a producer warpgroup whose first warp issues every MMA and
+// whose second issues every TMA load (the other two idle).  setmaxnreg moves
+// registers from the producer warpgroup to the softmax warpgroups.  Each
+// K_j, V_j tile brought into shared memory serves both query tiles.
 //   S_i   (128 x 128 fp32, TMEM columns 256 i ..)        = Q_i K_j^T   (tcgen05.mma, A and B in smem)
 //   P_i   (128 x 128 bf16, over the first 64 columns of S_i)            (written by the softmax threads)
 //   O_i   (128 x D   fp32, TMEM columns 256 i + 128 ..) += P_i V_j     (tcgen05.mma, A in TMEM)
-// Q, K_j, V_j arrive by TMA in 128-byte-swizzled tiles.  One thread issues
-// every MMA, in the order S_0,0 S_1,0 | O_0,j S_0,j+1 | O_1,j S_1,j+1 | ...,
-// so the tensor cores work on one tile while the other tile's warpgroup
-// computes its exponentials.  The MMAs of one thread complete in issue order
-// (tcgen05.commit reports everything issued before it), so "S_i,j+1 done"
-// also means "O_i,j done and P_i,j read".  Every mbarrier wait is bounded
-// (1 s); a wait that gives up is counted, the whole CTA stops, waits (again
-// bounded) for its copies and MMAs in flight, frees its TMEM and returns.
+// Q, K_j, V_j arrive by TMA in 128-byte-swizzled tiles, two buffers each for
+// K and V.  The MMA thread issues in the order S_0,0 S_1,0 | O_0,j S_0,j+1 |
+// O_1,j S_1,j+1 | ..., so the tensor cores work on one tile while the other
+// tile's warpgroup computes its exponentials; after the last MMA that reads
+// K_j (or V_j) it commits to that buffer's "free" barrier, on which the load
+// thread waits before it refills the buffer.  The MMAs of one thread complete
+// in issue order (tcgen05.commit reports everything issued before it), so
+// "S_i,j+1 done" also means "O_i,j done and P_i,j read".  Every mbarrier
+// wait is bounded (1 s); a wait that gives up is counted, the whole CTA
+// stops, waits (again bounded) for its copies and MMAs in flight, frees its
+// TMEM and returns.
 //
 // The running max is lazy (the rescaling rule of the online softmax holds
 // for any reference value, not only the true max): a row's reference moves
@@ -44,7 +49,11 @@ __device__ unsigned int g_attn_wait_timeouts = 0;
 namespace {
 
 constexpr int kAttnTileThreads = 128;                   // one softmax warpgroup per query tile
-constexpr int kAttnThreads = 2 * kAttnTileThreads + 32;  // + the producer warp
+constexpr int kAttnThreads = 3 * kAttnTileThreads;       // + the producer warpgroup
+constexpr int kMmaWarp = 8, kLoadWarp = 9;               // producer warps (10, 11 idle)
+constexpr int kSoftmaxRegs = 208, kProducerRegs = 72;    // setmaxnreg split of the launch's registers
+constexpr int kSplitRegs = kAttnTileThreads * (2 * kSoftmaxRegs + kProducerRegs);
+static_assert(kSplitRegs <= 65536, "register split above the register file");
 constexpr int kAttnBlock = 128;                         // queries per tile = keys per step
 constexpr uint32_t kChunkBytes = 128 * 128;             // 128 rows x 64 bf16 columns
 constexpr uint32_t kTmemCols = 512;                     // tile i: S_i at 256 i, O_i at 256 i + 128
@@ -57,7 +66,7 @@ constexpr float kLazyRescale = 8.0f;
 // the CTA's abort flag; every other wait then returns at once, and the CTA
 // skips its remaining work (but not its arrivals) and frees its TMEM.
 __device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;  // suspended up to 20 us per try
@@ -91,21 +100,42 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Two fp32 lanes per instruction (sm_100 packed arithmetic), each rounded as
+// the scalar operation would be.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // One key block j of a softmax thread (row r of its tile; S in TMEM at tS,
 // O at tO): the row max, the lazy reference m (moved only when the block's
 // max exceeds it by more than kLazyRescale), p = 2^(s scale log2e - m)
 // written as bf16 over the first 64 columns of S, the running sum, and O
-// rescaled when m moved.  diag: the causal grid's diagonal block, whose keys
+// rescaled when m moved.  DIAG: the causal grid's diagonal block, whose keys
 // after the query are set to -inf in registers first (exp gives 0), so the
-// common body carries no per-element mask.
-__device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_cols, int r, int j, bool diag,
-                                              float scale_log2, float& m_i, float& l_i) {
+// other blocks carry no per-element mask.
+template <bool DIAG>
+__device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_cols, int r, int j, float scale_log2,
+                                              float& m_i, float& l_i) {
   tc::fence_after_sync();
   uint32_t sr[128];
 #pragma unroll
   for (int c = 0; c < 4; ++c) tc::tmem_ld32_async(tS + c * 32, sr + c * 32);
   tc::tmem_wait_ld();
-  if (diag) {
+  if (DIAG) {
 #pragma unroll
     for (int i = 0; i < 128; ++i) sr[i] = (i > r) ? 0xff800000u : sr[i];
   }
@@ -120,18 +150,20 @@ __device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_co
   const bool upd = mx > m_i + kLazyRescale;  // always for the first block (m_i = -inf)
   const float m_new = upd ? mx : m_i;
   const float corr = upd ? ex2_ftz(m_i - m_new) : 1.0f;
-  float sum8[8];
+  const float2 k2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_new, -m_new);
+  float2 sum4[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
+  for (int i = 0; i < 4; ++i) sum4[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-      const float p0 = ex2_ftz(fmaf(__uint_as_float(sr[c * 16 + i]), scale_log2, -m_new));
-      const float p1 = ex2_ftz(fmaf(__uint_as_float(sr[c * 16 + i + 1]), scale_log2, -m_new));
-      sum8[i >> 1] += p0 + p1;
-      w[i >> 1] = pack_bf16x2(p0, p1);
+      const float2 x =
+          ffma2(make_float2(__uint_as_float(sr[c * 16 + i]), __uint_as_float(sr[c * 16 + i + 1])), k2, nm2);
+      const float2 p = make_float2(ex2_ftz(x.x), ex2_ftz(x.y));
+      sum4[(i >> 1) & 3] = fadd2(sum4[(i >> 1) & 3], p);
+      w[i >> 1] = pack_bf16x2(p.x, p.y);
     }
     // keys 16c .. 16c+15 -> P columns 8c .. 8c+7 (x16 stores take two chunks)
     if (c & 1) {
@@ -148,7 +180,8 @@ __device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_co
     }
   }
   tc::tmem_wait_st();
-  l_i = fmaf(l_i, corr, ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
+  const float2 s2 = fadd2(fadd2(sum4[0], sum4[1]), fadd2(sum4[2], sum4[3]));
+  l_i = fmaf(l_i, corr, s2.x + s2.y);
   m_i = m_new;
   // O rescale (rare): O_j-1 is complete, since S_j (issued after it) is
   if (j > 0 && __any_sync(0xffffffffu, upd)) {
@@ -174,15 +207,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_p[2], bar_o[2], bar_drain;
+  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_kfree[2], bar_vfree[2], bar_s[2], bar_p[2], bar_o[2],
+      bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
-  // Q0 | Q1 | K0 | K1 | V0 | V1, every tile 1024-byte aligned
+  // Q0 | Q1 | K0 | K1 | V0 | V1, every tile 1024-byte aligned (addressed by
+  // offset: arrays of pointers indexed at run time would live in local memory)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
-  uint8_t* sQ[2] = {base, base + TILE};
-  uint8_t* sK[2] = {base + 2 * TILE, base + 3 * TILE};
-  uint8_t* sV[2] = {base + 4 * TILE, base + 5 * TILE};
+  auto sQ = [&](int i) { return base + i * TILE; };
+  auto sK = [&](int b) { return base + (2 + b) * TILE; };
+  auto sV = [&](int b) { return base + (4 + b) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int slice = blockIdx.x;
@@ -191,12 +226,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int pair = CAUSAL ? npair - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
   // query tiles 2 pair and 2 pair + 1 (the second absent when nq is odd and
   // this is the last pair); key blocks per tile (0: absent)
-  int nkv[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
+  auto nkv_of = [&](int i) {
     const int qb = 2 * pair + i;
-    nkv[i] = qb < nq ? (CAUSAL ? qb + 1 : nq) : 0;
-  }
+    return qb < nq ? (CAUSAL ? qb + 1 : nq) : 0;
+  };
+  const int nkv0 = nkv_of(0), nkv1 = nkv_of(1);
+  const int nmax = nkv0 > nkv1 ? nkv0 : nkv1;
+  const int ntiles = nkv1 > 0 ? 2 : 1;
   volatile int* abort = &abort_flag;
 
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
@@ -205,6 +241,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
+      mbar_init(&bar_kfree[i], 1);
+      mbar_init(&bar_vfree[i], 1);
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_o[i], 1);
       mbar_init(&bar_p[i], kAttnTileThreads);
@@ -218,27 +256,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 2 * kAttnTileThreads / 32) {
-    // ------------------------------------------------ producer warp: TMA and MMA issue
-    if ((tid & 31) == 0) {
-      const int nmax = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
-      const int ntiles = nkv[1] > 0 ? 2 : 1;
-      const int row0 = slice * t;  // first row of this slice in the [bh * t, D] view
-      int k_ld = 0, k_wt = 0, v_ld = 0, v_wt = 0;  // K_0 .. K_{k_ld-1} issued, K_0 .. K_{k_wt-1} seen
-      auto load_k = [&](int j) {
+  if (warp >= 2 * kAttnTileThreads / 32) {
+    // ------------------------------------------------ producer warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs) : "memory");
+    const int row0 = slice * t;  // first row of this slice in the [bh * t, D] view
+    if (warp == kLoadWarp && (tid & 31) == 0) {
+      // ---- TMA loads: Q, then K_j and V_j into buffer j % 2 once the MMAs
+      // that read K_j-2 / V_j-2 have completed
+      mbar_arrive_expect_tx(&bar_q, ntiles * TILE);
+      for (int i = 0; i < ntiles; ++i) {
+#pragma unroll
+        for (int c = 0; c < KC; ++c)
+          tc::tma_load_2d(sQ(i) + c * kChunkBytes, &tmq, &bar_q, c * 64, row0 + (2 * pair + i) * kAttnBlock);
+      }
+      int nk = 0, nv = 0;  // K_0 .. K_nk-1, V_0 .. V_nv-1 issued
+      for (int j = 0; j < nmax; ++j) {
         const int b = j & 1;
+        if (j >= 2 && !attn_wait(&bar_kfree[b], ((j - 2) >> 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bar_k[b], TILE);
 #pragma unroll
-        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sK[b] + c * kChunkBytes, &tmk, &bar_k[b], c * 64, row0 + j * 128);
-        k_ld = j + 1;
-      };
-      auto load_v = [&](int j) {
-        const int b = j & 1;
+        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sK(b) + c * kChunkBytes, &tmk, &bar_k[b], c * 64, row0 + j * 128);
+        nk = j + 1;
+        if (j >= 2 && !attn_wait(&bar_vfree[b], ((j - 2) >> 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bar_v[b], TILE);
 #pragma unroll
-        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sV[b] + c * kChunkBytes, &tmv, &bar_v[b], c * 64, row0 + j * 128);
-        v_ld = j + 1;
-      };
+        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sV(b) + c * kChunkBytes, &tmv, &bar_v[b], c * 64, row0 + j * 128);
+        nv = j + 1;
+      }
+      // copies in flight land before the CTA exits.  A buffer is refilled only
+      // after the MMA warp has seen its previous load land, so only the last
+      // load into each buffer can be pending.
+      drain_wait(&bar_q, 0);
+      for (int j = nk > 2 ? nk - 2 : 0; j < nk; ++j) drain_wait(&bar_k[j & 1], (j >> 1) & 1);
+      for (int j = nv > 2 ? nv - 2 : 0; j < nv; ++j) drain_wait(&bar_v[j & 1], (j >> 1) & 1);
+    } else if (warp == kMmaWarp && (tid & 31) == 0) {
+      // ---- MMA issue
+      int k_wt = 0, v_wt = 0;  // K_0 .. K_k_wt-1, V_0 .. V_v_wt-1 seen in shared memory
       auto wait_k = [&](int j) {
         if (j < k_wt) return true;
         if (!attn_wait(&bar_k[j & 1], (j >> 1) & 1, abort)) return false;
@@ -251,95 +304,87 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         v_wt = j + 1;
         return true;
       };
+      auto last = [&](int j) { return j < nkv1 ? 1 : 0; };  // the tile that reads K_j and V_j last
+      // shared-memory descriptors, low words (the high words are constants):
+      // one per buffer, stepped through a tile by constant offsets
+      constexpr uint32_t HI = tc::smem_desc_hi(1024);
+      const uint32_t dq0 = tc::smem_desc_lo(smem_addr(sQ(0)), 16);
+      const uint32_t dk0 = tc::smem_desc_lo(smem_addr(sK(0)), 16);
+      const uint32_t dv0 = tc::smem_desc_lo(smem_addr(sV(0)), kChunkBytes);
       // S_i = Q_i K_j^T into TMEM columns 256 i ..
       auto issue_s = [&](int i, int j) {
-        const uint32_t aQ = smem_addr(sQ[i]), aK = smem_addr(sK[j & 1]);
+        const uint32_t dq = dq0 + i * (TILE >> 4), dk = dk0 + (j & 1) * (TILE >> 4);
+        const uint32_t ts = tmem + i * 256;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks / 4) * kChunkBytes + (ks % 4) * 32;
-          tc::mma_bf16(tmem + i * 256, tc::smem_desc(aQ + off, 16, 1024), tc::smem_desc(aK + off, 16, 1024),
-                       IDESC_S, ks > 0 ? 1u : 0u);
+          const uint32_t off = ((ks / 4) * kChunkBytes + (ks % 4) * 32) >> 4;
+          tc::mma_bf16(ts, tc::desc_join(dq + off, HI), tc::desc_join(dk + off, HI), IDESC_S, ks > 0 ? 1u : 0u);
         }
         tc::mma_commit(&bar_s[i]);
+        if (i == last(j)) tc::mma_commit(&bar_kfree[j & 1]);
       };
       // O_i += P_i V_j: P_i (TMEM, 8 columns per 16 keys), V_j MN-major in smem
       auto issue_o = [&](int i, int j) {
-        const uint32_t aV = smem_addr(sV[j & 1]);
+        const uint32_t dv = dv0 + (j & 1) * (TILE >> 4);
+        const uint32_t to = tmem + i * 256 + 128, tp = tmem + i * 256;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < kAttnBlock / 16; ++ks)
-          tc::mma_bf16_ts(tmem + i * 256 + 128, tmem + i * 256 + ks * 8,
-                          tc::smem_desc(aV + ks * 2048, kChunkBytes, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(to, tp + ks * 8, tc::desc_join(dv + ((ks * 2048) >> 4), HI), IDESC_O, ks > 0 ? 1u : acc0);
+        if (i == last(j)) tc::mma_commit(&bar_vfree[j & 1]);
       };
 
-      mbar_arrive_expect_tx(&bar_q, ntiles * TILE);
-      for (int i = 0; i < ntiles; ++i) {
-#pragma unroll
-        for (int c = 0; c < KC; ++c)
-          tc::tma_load_2d(sQ[i] + c * kChunkBytes, &tmq, &bar_q, c * 64, row0 + (2 * pair + i) * kAttnBlock);
-      }
-      load_k(0);
-      load_v(0);
-      if (nmax > 1) {
-        load_k(1);
-        load_v(1);
-      }
-      const bool q_ok = attn_wait(&bar_q, 0, abort);
-      bool ok = q_ok && wait_k(0);
+      bool ok = attn_wait(&bar_q, 0, abort) && wait_k(0);
       if (ok) {
         tc::fence_after_sync();
         for (int i = 0; i < ntiles; ++i) issue_s(i, 0);
       }
       for (int j = 0; ok && j < nmax; ++j) {
-        const int last = j < nkv[1] ? 1 : 0;  // the tile that reads K_j last
-        for (int i = 0; ok && i < 2; ++i) {
-          if (i == last && (j + 2 < nmax || (j >= 1 && j + 1 < nmax))) {
-            // refills: K_j was last read by S_last,j and V_j-1 by O_last,j-1,
-            // both complete once S_last,j is.  This runs before S_last,j+1 is
-            // issued, so bar_s[last] cannot be a phase further on.
-            ok = attn_wait(&bar_s[last], j & 1, abort);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int nkv_i = i == 0 ? nkv0 : nkv1;
+          if (!ok || j >= nkv_i) continue;
+          // softmax i is done with block j: P_i,j written, O_i rescaled
+          ok = attn_wait(&bar_p[i], j & 1, abort) && wait_v(j);
+          if (!ok) break;
+          tc::fence_after_sync();
+          issue_o(i, j);
+          if (j + 1 < nkv_i) {
+            ok = wait_k(j + 1);
             if (!ok) break;
-            if (j + 2 < nmax) load_k(j + 2);
-            if (j >= 1 && j + 1 < nmax) load_v(j + 1);
-          }
-          if (j < nkv[i]) {
-            // softmax i is done with block j: P_i,j written, O_i rescaled
-            ok = attn_wait(&bar_p[i], j & 1, abort) && wait_v(j);
-            if (!ok) break;
-            tc::fence_after_sync();
-            issue_o(i, j);
-            if (j + 1 < nkv[i]) {
-              ok = wait_k(j + 1);
-              if (!ok) break;
-              issue_s(i, j + 1);
-            } else {
-              tc::mma_commit(&bar_o[i]);
-            }
+            issue_s(i, j + 1);
+          } else {
+            tc::mma_commit(&bar_o[i]);
           }
         }
       }
-      // everything in flight lands before the CTA exits
+      // every MMA completes before the CTA exits
       tc::mma_commit(&bar_drain);
       drain_wait(&bar_drain, 0);
-      if (!q_ok) drain_wait(&bar_q, 0);
-      for (int j = k_wt; j < k_ld; ++j) drain_wait(&bar_k[j & 1], (j >> 1) & 1);
-      for (int j = v_wt; j < v_ld; ++j) drain_wait(&bar_v[j & 1], (j >> 1) & 1);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------ softmax warpgroup i: query tile 2 pair + i
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs) : "memory");
     const int i = warp >> 2;
     const int r = ((warp & 3) << 5) | (tid & 31);
     const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane + i * 256, tO = tS + 128;
     const int qb = 2 * pair + i;
+    const int nkv_i = i == 0 ? nkv0 : nkv1;
     float m_i = -INFINITY, l_i = 0.0f;
-    for (int j = 0; j < nkv[i]; ++j) {
+    for (int j = 0; j < nkv_i; ++j) {
       attn_wait(&bar_s[i], j & 1, abort);
-      if (!__any_sync(0xffffffffu, *abort)) softmax_block(tS, tO, D, r, j, CAUSAL && j == qb, scale_log2, m_i, l_i);
+      if (!__any_sync(0xffffffffu, *abort)) {
+        if (CAUSAL && j == qb)
+          softmax_block<true>(tS, tO, D, r, j, scale_log2, m_i, l_i);
+        else
+          softmax_block<false>(tS, tO, D, r, j, scale_log2, m_i, l_i);
+      }
       tc::fence_before_sync();
       mbar_arrive(&bar_p[i]);
     }
-    if (nkv[i] > 0) {
+    if (nkv_i > 0) {
       attn_wait(&bar_o[i], 0, abort);
       if (!__any_sync(0xffffffffu, *abort)) {
         tc::fence_after_sync();
@@ -404,6 +449,13 @@ cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   constexpr uint32_t TILE = (D / 64) * kChunkBytes;
   const size_t smem = 6 * TILE + 1024;
   auto kernel = attention_fwd_kernel<D, CAUSAL>;
+  // setmaxnreg.inc waits until the registers it asks for are free in the
+  // block's pool (its threads x the registers each was launched with): the
+  // split must fit that pool, or the softmax warpgroups would wait forever
+  cudaFuncAttributes fa;
+  cudaError_t e0 = cudaFuncGetAttributes(&fa, kernel);
+  if (e0 != cudaSuccess) return e0;
+  if (fa.numRegs * kAttnThreads < kSplitRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(bh), static_cast<unsigned>((t / kAttnBlock + 1) / 2));

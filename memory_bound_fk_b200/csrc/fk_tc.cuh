@@ -33,6 +33,24 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
   return d;
 }
 
+// The same descriptor split into its 32-bit halves, for issue loops that
+// step through a tile: the low word holds the start address (bits 0..13,
+// address / 16) and the leading offset, the high word the stride offset, the
+// version bit and the swizzle mode.  A shared-memory address is below 256 KB,
+// so advancing the start by `bytes` is a 32-bit add of bytes / 16 to the low
+// word, with no carry out of the address field.
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t addr, uint32_t lbo_bytes) {
+  return ((addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+
 // Instruction descriptor of a dense kind::f16 MMA with bf16 A and B and an
 // fp32 accumulator, M x N, A K-major, B K-major (b_mn = false) or MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn) {

@@ -1,7 +1,8 @@
 """A CPU model of the attention kernel's synchronisation (fk_attention.cu):
-the producer thread's schedule of TMA loads, MMA issues, commits and
-mbarrier waits, the two softmax warpgroups, an in-order tensor-core queue
-and TMA loads that land in any order, all interleaved at random.
+the load warp's TMA loads and buffer-free waits, the MMA warp's schedule of
+MMA issues, commits and mbarrier waits, the two softmax warpgroups, an
+in-order tensor-core queue and TMA loads that land in any order, all
+interleaved at random.
 
 The mbarrier is modelled by its phase count; a parity wait succeeds when
 the current phase's parity differs from the one asked for, as on the GPU.
@@ -12,10 +13,10 @@ region, O holding blocks 0..j-1), and no schedule may stall.  Every tile
 count a grid can hand a CTA (one or two query tiles, causal or not, up to
 eight key blocks) is run under many random interleavings.
 
-The model follows the kernel's producer loop step by step; a change there
-must be made here too.  A variant with the refill wait in the wrong place
-(after tile 0's MMAs, whatever tile reads K_j last) is shown to stall, so
-the model can catch that class of mistake.
+The model follows the kernel's load and MMA loops step by step; a change
+there must be made here too.  A variant that frees K_j too early (after
+tile 0's S_j, whatever tile reads K_j last) is shown to overwrite a tile
+an MMA still needs, so the model can catch that class of mistake.
 """
 import random
 
@@ -38,11 +39,16 @@ class Bar:
 
 
 class Model:
-    def __init__(self, nkv, rng, refill_before_last=True):
+    """kfree_after_last=False plants a mistake: K_j is reported free once
+    tile 0's S_j is issued, whatever tile reads K_j last."""
+
+    def __init__(self, nkv, rng, kfree_after_last=True):
         self.nkv = nkv
         self.rng = rng
-        self.refill_before_last = refill_before_last
-        self.bars = {n: Bar(1) for n in ("q", "k0", "k1", "v0", "v1", "s0", "s1", "o0", "o1", "p0", "p1", "drain")}
+        self.kfree_after_last = kfree_after_last
+        names = ("q", "k0", "k1", "v0", "v1", "kfree0", "kfree1", "vfree0", "vfree1", "s0", "s1", "o0", "o1",
+                 "p0", "p1", "drain")
+        self.bars = {n: Bar(1) for n in names}
         self.tensor = []  # in issue order: ("mma", op) or ("commit", bar)
         self.tma = []     # (buffer, tile)
         self.smem = {}
@@ -59,14 +65,28 @@ class Model:
         if b.phase != k + 1:
             self.errors.append(f"wait on {bar} for phase {k} passed with {b.phase} phases complete")
 
-    def producer(self):
+    def loader(self):
+        """The load warp: Q, then K_j and V_j into buffer j % 2 once the
+        MMAs that read K_j-2 / V_j-2 are done."""
+        nmax = max(self.nkv)
+        self.tma.append(("q", ("q", 0)))
+        for j in range(nmax):
+            if j >= 2:
+                yield from self.wait(f"kfree{j & 1}", (j - 2) >> 1)
+            self.tma.append((f"k{j & 1}", ("k", j)))
+            if j >= 2:
+                yield from self.wait(f"vfree{j & 1}", (j - 2) >> 1)
+            self.tma.append((f"v{j & 1}", ("v", j)))
+
+    def mma(self):
+        """The MMA warp."""
         nkv = self.nkv
         nmax = max(nkv)
         ntiles = 2 if nkv[1] > 0 else 1
         seen = {"k": 0, "v": 0}
 
-        def load(kind, j):
-            self.tma.append((f"{kind}{j & 1}", (kind, j)))
+        def last(j):  # the tile that reads K_j and V_j last
+            return 1 if j < nkv[1] else 0
 
         def wait_tile(kind, j):
             if j < seen[kind]:
@@ -77,41 +97,26 @@ class Model:
         def issue_s(i, j):
             self.tensor.append(("mma", ("S", i, j, f"k{j & 1}", ("k", j))))
             self.tensor.append(("commit", f"s{i}"))
+            if i == (last(j) if self.kfree_after_last else 0):
+                self.tensor.append(("commit", f"kfree{j & 1}"))
 
-        def refill(j, last):
-            yield from self.wait(f"s{last}", j)
-            if j + 2 < nmax:
-                load("k", j + 2)
-            if j >= 1 and j + 1 < nmax:
-                load("v", j + 1)
-
-        self.tma.append(("q", ("q", 0)))
-        load("k", 0)
-        load("v", 0)
-        if nmax > 1:
-            load("k", 1)
-            load("v", 1)
         yield from self.wait("q", 0)
         yield from wait_tile("k", 0)
         for i in range(ntiles):
             issue_s(i, 0)
         for j in range(nmax):
-            last = 1 if j < nkv[1] else 0
-            needs_refill = j + 2 < nmax or (j >= 1 and j + 1 < nmax)
             for i in range(2):
-                if self.refill_before_last and i == last and needs_refill:
-                    yield from refill(j, last)
                 if j < nkv[i]:
                     yield from self.wait(f"p{i}", j)
                     yield from wait_tile("v", j)
                     self.tensor.append(("mma", ("O", i, j, f"v{j & 1}", ("v", j))))
+                    if i == last(j):
+                        self.tensor.append(("commit", f"vfree{j & 1}"))
                     if j + 1 < nkv[i]:
                         yield from wait_tile("k", j + 1)
                         issue_s(i, j + 1)
                     else:
                         self.tensor.append(("commit", f"o{i}"))
-                if not self.refill_before_last and i == 0 and needs_refill:
-                    yield from refill(j, last)
         self.tensor.append(("commit", "drain"))
         yield from self.wait("drain", 0)
 
@@ -163,7 +168,8 @@ class Model:
         return True
 
     def run(self):
-        live = {"producer": self.producer(), "softmax0": self.softmax(0), "softmax1": self.softmax(1)}
+        live = {"loader": self.loader(), "mma": self.mma(), "softmax0": self.softmax(0),
+                "softmax1": self.softmax(1)}
         idle = 0
         while live or self.tensor or self.tma:
             c = self.rng.choice(list(live) + ["tensor", "tma"])
@@ -203,13 +209,12 @@ def test_schedule_is_race_and_stall_free(nkv):
         assert not errors, (seed, errors[:3])
 
 
-def test_model_catches_a_misplaced_refill():
-    """With the refill wait after tile 0's MMAs, a CTA with one query tile
-    waits on bar_s[0] after issuing S_0,j+1: once that MMA is done the
-    barrier is two phases on and the wait never succeeds."""
+def test_model_catches_an_early_kfree():
+    """With K_j reported free after tile 0's S_j, the load of K_j+2 can
+    land while S_1,j still waits in the tensor queue for K_j."""
     found = False
-    for seed in range(50):
-        if Model((3, 0), random.Random(seed), refill_before_last=False).run():
+    for seed in range(200):
+        if Model((4, 4), random.Random(seed), kfree_after_last=False).run():
             found = True
             break
     assert found
