@@ -180,9 +180,23 @@ def kernel_family(op: str) -> str:
     raise KeyError(op)
 
 
+def code_text(src: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed:
+    what the compiler sees, so that a comment edit does not count as a kernel
+    change.  String literals (inline PTX) are kept as written."""
+    out, pos = [], 0
+    for m in re.finditer(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', src, re.S):
+        out.append(src[pos:m.start()])
+        out.append(m.group(0) if m.group(0).startswith('"') else " ")
+        pos = m.end()
+    out.append(src[pos:])
+    return " ".join("".join(out).split())
+
+
 def csrc_digest(family: str | None = None) -> str:
-    """Digest of the kernel sources of one family (all of csrc/ if None),
-    with the shared internal header and the public header."""
+    """Digest of the code (comments and layout excluded) of the kernel
+    sources of one family (all of csrc/ if None), with the shared internal
+    header and the public header."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "memory_bound_fk_b200", "csrc")
     if family is None:
@@ -191,9 +205,9 @@ def csrc_digest(family: str | None = None) -> str:
         files = [os.path.join(csrc, f) for f in _FAMILY_SOURCES[family] + ["fk_internal.h"]]
     files.append(os.path.join(ROOT, "include", "fk.h"))
     for p in files:
-        with open(p, "rb") as f:
+        with open(p, encoding="utf-8") as f:
             h.update(os.path.basename(p).encode())
-            h.update(f.read())
+            h.update(code_text(f.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -587,6 +601,10 @@ def run_attention(args) -> dict | None:
     peak = float(d_all.get("bf16_tflops", 1590.0))
     ms = max_ms / args.steps
     kname = f"attention_fwd_kernel<d={d},causal={int(causal)}>"
+    # DRAM bytes of one launch from the ncu capture in profiles/ (q, k, v
+    # read, o written: 4 bh t d bf16 values algorithmically; K/V tiles that
+    # miss L2 are read again)
+    traffic, traffic_src = profiled_traffic(n)
     return {
         "metric": "attention forward TFLOP/s (bf16 in, fp32 accumulate) at 1 B200", "value": round(tflops, 2),
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -600,7 +618,8 @@ def run_attention(args) -> dict | None:
         "roofline": {"bound": "tensor", "kernel": kname, "workload": n, "achieved": round(flops / ms / 1e9, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(flops / ms / 1e9 / peak, 4),
                      "peak_source": "measured (cuBLAS bf16 burst)" if d_all else "fallback",
-                     "traffic": None},
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_bytes_per_launch": 4 * bh * t * d * 2},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
     }
 

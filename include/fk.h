@@ -338,7 +338,7 @@ FK_API fk_status fk_layernorm_rows_ex(const void *x, void *y, const float *gamma
  * and 8):
  *     O = softmax(scale * Q K^T  [+ causal mask: key j > query i is -inf]) V
  * for bh independent (batch, head) slices; S and P stay on chip (tensor
- * memory and shared memory), with the running max / sum of section 7.2.
+ * memory), with the running max / sum of section 7.2.
  *   q, k, v  [bh, t, d] bf16, contiguous, device memory, 16-byte aligned.
  *   o        [bh, t, d] bf16 output; must not overlap q, k or v.
  *   t        a multiple of 128, at most 128 * 65535 (queries and keys per
@@ -348,8 +348,11 @@ FK_API fk_status fk_layernorm_rows_ex(const void *x, void *y, const float *gamma
  * Arithmetic: S and the O accumulator in fp32 (tcgen05, TMEM), P rounded to
  * bf16 for the second product, O rounded to bf16 at the end.
  * Errors: FK_ERR_INVALID_ARG for a shape or argument outside the above,
- * bh * t >= 2^31, bad pointers or overlap.  A wait that gives up (see
- * fk_wait_timeouts) leaves that block of O unwritten.
+ * bh * t >= 2^31, bad pointers or overlap; FK_ERR_CUDA if the kernel cannot
+ * be launched (including a build whose register allocation cannot fund the
+ * kernel's warp-specialised register split, which it checks before
+ * launching).  A wait that gives up (see fk_wait_timeouts) leaves that
+ * block of O unwritten.
  */
 FK_API fk_status fk_attention_fwd(const void *q, const void *k, const void *v, void *o, size_t bh, size_t t,
                                   size_t d, int causal, float scale, void *stream);
