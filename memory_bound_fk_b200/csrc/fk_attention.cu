@@ -31,7 +31,8 @@
 // for any reference value, not only the true max): a row's reference moves
 // only when the block max exceeds it by more than 2^8, so the weights stay
 // at most 256 and the O rescale -- a TMEM round trip -- is rare.
-// Causal grids hand out the longest query blocks (most key blocks) first.
+// Causal grids hand out the longest query-tile pairs first; other grids keep
+// the pairs of a slice together in launch order, for L2 reuse of K and V.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -220,10 +221,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto sV = [&](int b) { return base + (4 + b) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int slice = blockIdx.x;
   const int nq = t / kAttnBlock;
-  const int npair = static_cast<int>(gridDim.y);
-  const int pair = CAUSAL ? npair - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
+  const int npair = (nq + 1) / 2;
+  // launch order: causal grids hand out the longest pairs (most key blocks)
+  // first, across all slices; other grids keep the pairs of a slice
+  // together, so its K/V tiles are read from HBM once and then hit L2
+  const int bh = static_cast<int>(gridDim.x) / npair;
+  const int lin = static_cast<int>(blockIdx.x);
+  const int slice = CAUSAL ? lin % bh : lin / npair;
+  const int pair = CAUSAL ? npair - 1 - lin / bh : lin % npair;
   // query tiles 2 pair and 2 pair + 1 (the second absent when nq is odd and
   // this is the last pair); key blocks per tile (0: absent)
   auto nkv_of = [&](int i) {
@@ -344,14 +350,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < 2; ++i) {
           const int nkv_i = i == 0 ? nkv0 : nkv1;
           if (!ok || j >= nkv_i) continue;
-          // softmax i is done with block j: P_i,j written, O_i rescaled
-          ok = attn_wait(&bar_p[i], j & 1, abort) && wait_v(j);
+          // the tiles first (long since loaded: their loads wait only on
+          // MMAs already issued), then softmax i's block j: P_i,j written,
+          // O_i rescaled.  The two MMA groups then go out back to back.
+          ok = wait_v(j) && (j + 1 >= nkv_i || wait_k(j + 1)) && attn_wait(&bar_p[i], j & 1, abort);
           if (!ok) break;
           tc::fence_after_sync();
           issue_o(i, j);
           if (j + 1 < nkv_i) {
-            ok = wait_k(j + 1);
-            if (!ok) break;
             issue_s(i, j + 1);
           } else {
             tc::mma_commit(&bar_o[i]);
@@ -458,7 +464,7 @@ cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (fa.numRegs * kAttnThreads < kSplitRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(bh), static_cast<unsigned>((t / kAttnBlock + 1) / 2));
+  const dim3 grid(static_cast<unsigned>(bh * ((t / kAttnBlock + 1) / 2)));
   kernel<<<grid, kAttnThreads, smem, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(t),
                                           scale_log2);
   return cudaGetLastError();

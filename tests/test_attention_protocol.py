@@ -107,13 +107,15 @@ class Model:
         for j in range(nmax):
             for i in range(2):
                 if j < nkv[i]:
-                    yield from self.wait(f"p{i}", j)
+                    # the tiles first (long since loaded), then the softmax
                     yield from wait_tile("v", j)
+                    if j + 1 < nkv[i]:
+                        yield from wait_tile("k", j + 1)
+                    yield from self.wait(f"p{i}", j)
                     self.tensor.append(("mma", ("O", i, j, f"v{j & 1}", ("v", j))))
                     if i == last(j):
                         self.tensor.append(("commit", f"vfree{j & 1}"))
                     if j + 1 < nkv[i]:
-                        yield from wait_tile("k", j + 1)
                         issue_s(i, j + 1)
                     else:
                         self.tensor.append(("commit", f"o{i}"))
