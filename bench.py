@@ -166,9 +166,9 @@ def measured_peaks() -> dict:
 # Sources each kernel family is compiled from (its profile stays valid while
 # these are unchanged).
 _FAMILY_SOURCES = {
-    "gelu": ["fk_gelu.cu", "fk_gelu.cuh", "fk_common.cuh"],
+    "gelu": ["fk_gelu.cu", "fk_gelu.cuh", "fk_f32x2.cuh", "fk_common.cuh"],
     "softmax": ["fk_softmax.cu", "fk_rows.cuh", "fk_common.cuh", "fk_sync.cuh", "fk_plan.cpp"],
-    "layernorm": ["fk_layernorm.cu", "fk_rows.cuh", "fk_common.cuh", "fk_gelu.cuh", "fk_plan.cpp"],
+    "layernorm": ["fk_layernorm.cu", "fk_rows.cuh", "fk_common.cuh", "fk_gelu.cuh", "fk_f32x2.cuh", "fk_plan.cpp"],
     "attention": ["fk_attention.cu", "fk_tc.cuh", "fk_sync.cuh", "fk_common.cuh"],
 }
 

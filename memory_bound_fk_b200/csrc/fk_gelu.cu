@@ -42,7 +42,11 @@ __device__ __forceinline__ uint4 gelu_vec(uint4 v) {
   float f[VEC];
   Elem<T>::unpack(v, f);
 #pragma unroll
-  for (int k = 0; k < VEC; ++k) f[k] = gelu_f<T, KIND>(f[k]);
+  for (int k = 0; k < VEC; k += 2) {
+    const float2 g = gelu_f2<T, KIND>(make_float2(f[k], f[k + 1]));
+    f[k] = g.x;
+    f[k + 1] = g.y;
+  }
   return Elem<T>::pack(f);
 }
 

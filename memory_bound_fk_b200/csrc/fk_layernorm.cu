@@ -140,14 +140,15 @@ __device__ __forceinline__ void load_affine(const float* p, float dflt, Idx vfir
   }
 }
 
-// The epilogue.  GELU takes the flush-to-zero exponential for either output
-// type: a GELU output below 2^-126 is within the LayerNorm error bound of 0.
+// The epilogue, on a pair of values.  GELU takes the flush-to-zero
+// exponential for either output type: a GELU output below 2^-126 is within
+// the LayerNorm error bound of 0.
 template <int EPI>
-__device__ __forceinline__ float epilogue(float z) {
+__device__ __forceinline__ float2 epilogue2(float2 z) {
   if constexpr (EPI == FK_EPILOGUE_GELU_TANH) {
-    return gelu_tanh_f<float>(z);
+    return gelu_tanh_f2<float>(z);
   } else if constexpr (EPI == FK_EPILOGUE_GELU_ERF) {
-    return gelu_erf_f<float>(z);
+    return gelu_erf_f2<float>(z);
   } else {
     return z;
   }
@@ -164,9 +165,15 @@ __device__ __forceinline__ void normalise_store(T* yr, const uint4* raw, float m
     float g[VEC], b[VEC];
     load_affine<T, TEAM, ALIGNED, Idx>(gamma, 1.0f, vfirst, c, cols, t, g);
     load_affine<T, TEAM, ALIGNED, Idx>(beta, 0.0f, vfirst, c, cols, t, b);
+    // pairs of columns, each lane as ((x - m1) - d) * rstd * gamma + beta
 #pragma unroll
-    for (int k = 0; k < VEC; ++k)
-      o[k] = epilogue<EPI>(fmaf(((val<T>(raw[c], k) - m1) - d) * rstd, g[k], b[k]));
+    for (int k = 0; k < VEC; k += 2) {
+      float2 z = add2(make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1)), splat2(-m1));
+      z = mul2(add2(z, splat2(-d)), splat2(rstd));
+      z = epilogue2<EPI>(fma2(z, make_float2(g[k], g[k + 1]), make_float2(b[k], b[k + 1])));
+      o[k] = z.x;
+      o[k + 1] = z.y;
+    }
   });
 }
 
@@ -174,12 +181,19 @@ __device__ __forceinline__ void normalise_store(T* yr, const uint4* raw, float m
 template <typename T, int VPT>
 __device__ __forceinline__ float sum_raw(const uint4* raw) {
   constexpr int VEC = Elem<T>::VEC;
-  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // four accumulators (column k into k % 4), two per packed pair
+  float2 s01 = make_float2(0.0f, 0.0f), s23 = make_float2(0.0f, 0.0f);
 #pragma unroll
   for (int c = 0; c < VPT; ++c)
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) s[k & 3] += val<T>(raw[c], k);
-  return (s[0] + s[1]) + (s[2] + s[3]);
+    for (int k = 0; k < VEC; k += 2) {
+      const float2 v = make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1));
+      if (k & 2)
+        s23 = add2(s23, v);
+      else
+        s01 = add2(s01, v);
+    }
+  return (s01.x + s01.y) + (s23.x + s23.y);
 }
 
 // Pass-2 partial sums of one thread: sum (x - m1) and sum (x - m1)^2 over
@@ -187,17 +201,20 @@ __device__ __forceinline__ float sum_raw(const uint4* raw) {
 template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
 __device__ __forceinline__ float2 centred_sums(const uint4* raw, float m1, Idx vfirst, Idx cols, int t) {
   constexpr int VEC = Elem<T>::VEC;
-  float a[2] = {0.0f, 0.0f}, b[2] = {0.0f, 0.0f};
+  // two accumulators each (even and odd columns), one packed pair
+  float2 a = make_float2(0.0f, 0.0f), b = make_float2(0.0f, 0.0f);
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) {
-      const float z = in_row<T, TEAM, ALIGNED>(vfirst, c, k, t, cols) ? val<T>(raw[c], k) - m1 : 0.0f;
-      a[k & 1] += z;
-      b[k & 1] = fmaf(z, z, b[k & 1]);
+    for (int k = 0; k < VEC; k += 2) {
+      float2 z = add2(make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1)), splat2(-m1));
+      z.x = in_row<T, TEAM, ALIGNED>(vfirst, c, k, t, cols) ? z.x : 0.0f;
+      z.y = in_row<T, TEAM, ALIGNED>(vfirst, c, k + 1, t, cols) ? z.y : 0.0f;
+      a = add2(a, z);
+      b = fma2(z, z, b);
     }
   }
-  return make_float2(a[0] + a[1], b[0] + b[1]);
+  return make_float2(a.x + a.y, b.x + b.y);
 }
 
 // ---------------------------------------------------------------- warp path

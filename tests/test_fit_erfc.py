@@ -15,9 +15,10 @@ def test_kernel_constants_are_the_fitted_ones():
     coeffs, err = fit_erfc.fit(9)
     assert err <= 1.2e-7
     text = open(HEADER).read()
-    body = text[text.index("gelu_erf_f(float x)"):]
-    lits = [np.float32(float(v)) for v in re.findall(r"fmaf\(p, t, ([-+0-9.e]+)f\)", body)]
-    first = np.float32(float(re.search(r"float p = ([-+0-9.e]+)f;", body).group(1)))
+    body = text[text.index("erfc_poly(V t)"):]
+    body = body[:body.index("return p;")]
+    lits = [np.float32(float(v)) for v in re.findall(r"fma_v\(p, t, ([-+0-9.e]+)f\)", body)]
+    first = np.float32(float(re.search(r"V p = splat_v<V>\(([-+0-9.e]+)f\);", body).group(1)))
     got = np.array([first] + lits, np.float32)[::-1]   # c0 .. c9
     assert got.shape == (10,)
     assert np.array_equal(got, coeffs)
