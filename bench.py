@@ -183,7 +183,9 @@ def kernel_family(op: str) -> str:
 def code_text(src: str) -> str:
     """C/C++/CUDA source with comments removed and whitespace collapsed:
     what the compiler sees, so that a comment edit does not count as a kernel
-    change.  String literals (inline PTX) are kept as written."""
+    change.  String literals (inline PTX) are kept, so a `//` inside one is
+    not taken for a comment; runs of whitespace are collapsed there too,
+    which changes nothing ptxas reads."""
     out, pos = [], 0
     for m in re.finditer(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', src, re.S):
         out.append(src[pos:m.start()])

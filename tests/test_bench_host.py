@@ -128,3 +128,15 @@ def test_traffic_model_of_the_unfused_sequences():
     t = 32 << 20
     assert bench.unfused_traffic_bytes("gelu", t) == 18 * t
     assert bench.unfused_traffic_bytes("softmax", t) == 8 * t
+
+
+def test_source_digest_ignores_comments_and_layout_but_not_code():
+    """The digest that ties a profile's DRAM traffic to the kernel sources
+    hashes the code only: comments and whitespace may change, code and the
+    contents of string literals (inline PTX) may not."""
+    src = 'int a = 1; // note\n/* block\n comment */ asm("add.f32 %0, %1; // inside");\n'
+    code = bench.code_text(src)
+    assert code == 'int a = 1; asm("add.f32 %0, %1; // inside");'
+    assert bench.code_text('int  a =\n 1;  /* x */') == bench.code_text('int a = 1; // y')
+    assert bench.code_text('int a = 1;') != bench.code_text('int a = 2;')
+    assert bench.code_text('asm("mov.u32 %0, 1;")') != bench.code_text('asm("mov.u32 %0, 2;")')
