@@ -151,8 +151,10 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 // ---------------------------------------------------------------- MMA
 
-// D[tmem] (+)= A[smem] * B[smem]^T-ish per the descriptors; issued by one
-// thread.  accumulate = 0 overwrites D.
+// D (M x N, fp32, tensor memory) = A B (+ D when accumulate != 0), with A
+// (M x K) and B (K x N) in shared memory as the descriptors and the
+// instruction descriptor's major-ness bits lay them out (K-major A and B
+// give D = A B^T of the stored row-major tiles).  Issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
