@@ -1,9 +1,9 @@
 /*
  * fk.h -- C ABI of libfk: fused memory-bound operators for NVIDIA B200 (sm_100a).
  *
- * Two operators, each one kernel that reads every input element once from
- * HBM and writes every output element once (the fusion argument of
- * "Lecture 6: GPU Kernels and Triton", cs336.sjfarmltd.com, section 1.1:
+ * The two core operators are each one kernel that reads every input element
+ * once from HBM and writes every output element once (the fusion argument
+ * of "Lecture 6: GPU Kernels and Triton", cs336.sjfarmltd.com, section 1.1:
  * one read plus one write instead of a read and a write per separate op):
  *
  *   fk_gelu_tanh     y = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
@@ -15,6 +15,13 @@
  *                    used where one row is split across thread blocks), and
  *                    the lecture-6 notes, section 5.2 (row max, exponentials
  *                    and sum, normalise).
+ *
+ * Around them, the same one-pass design for the neighbouring steps the
+ * lecture builds on: fk_gelu (both GELU forms, fp32 or bf16),
+ * fk_softmax_rows_causal (scaled, causally masked softmax with the mask made
+ * in the kernel), fk_layernorm_rows (LayerNorm, optional affine and GELU
+ * epilogue), and fk_attention_fwd (attention forward on the tensor cores,
+ * the Flash-Attention computation of lecture 6, sections 7.3 and 8).
  *
  * Conventions common to every entry point
  * ---------------------------------------
