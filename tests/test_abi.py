@@ -160,3 +160,56 @@ def test_split_plan_and_workspace(fk):
         P.fk_softmax_rows_ws(A, B, 1, 1 << 22, 0, None, 0x30000000, 8, 0) in REJECT_NO_LAUNCH
     with pytest.raises(P.FkError):
         P.fk_softmax_rows_workspace(1, 10, 9)
+
+
+def _layernorm_rule(cols, dtype):
+    """The documented LayerNorm plan: one warp per row up to 1024 columns;
+    one block per row up to 32768 (16 values per thread up to 2048 columns,
+    else 32; the fewest threads from 128 up that hold the row); a 512-thread
+    streaming block above.  vpt counts 16-byte vectors (4 fp32 or 8 bf16)."""
+    vec = 4 if dtype == 0 else 8
+    if cols <= 1024:
+        return "warp"
+    if cols <= 32768:
+        ept = 16 if cols <= 128 * 16 else 32
+        threads = 128
+        while threads * ept < cols:
+            threads *= 2
+        return ("cta", threads, ept // vec)
+    return ("twophase", 512, 16 // vec)
+
+
+@pytest.mark.parametrize("cols", [1, 1024, 1025, 2048, 2049, 4096, 4097, 8193, 16384, 16385, 32768, 32769, 1 << 20])
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_layernorm_auto_plans_follow_the_rule(fk, cols, dtype):
+    p = fk.fk_layernorm_rows_plan(64, cols, dtype).as_dict()
+    want = _layernorm_rule(cols, dtype)
+    if want == "warp":
+        vec = 4 if dtype == 0 else 8
+        assert p["path"] == "warp" and p["cluster"] == 1
+        assert p["vpt"] * vec * 32 >= cols  # the warp's 32 lanes hold the row
+    else:
+        assert (p["path"], p["threads"], p["vpt"]) == want and p["cluster"] == 1
+
+
+def test_layernorm_plans_of_the_bench_workloads(fk):
+    # 16384 x 4096 fp32 and 65536 x 4096 bf16: 128 threads, 32 values each
+    assert fk.fk_layernorm_rows_plan(16384, 4096, 0).as_dict()["threads"] == 128
+    assert fk.fk_layernorm_rows_plan(65536, 4096, 1).as_dict()["vpt"] * 8 == 32
+
+
+def test_layernorm_forced_plans_and_errors(fk):
+    P = fk
+    assert P.fk_layernorm_rows_plan(2, 100, 0, P.FK_PATH_CTA).as_dict()["path"] == "cta"
+    assert P.fk_layernorm_rows_plan(2, 100, 0, P.FK_PATH_TWOPHASE).as_dict()["threads"] == 512
+    with pytest.raises(P.FkError):
+        P.fk_layernorm_rows_plan(2, 32769, 0, P.FK_PATH_CTA)     # more than a block holds
+    with pytest.raises(P.FkError):
+        P.fk_layernorm_rows_plan(2, 1025, 0, P.FK_PATH_WARP)     # more than a warp holds
+    with pytest.raises(P.FkError):
+        P.fk_layernorm_rows_plan(2, 4096, 0, P.FK_PATH_CLUSTER)  # no cluster path for LayerNorm
+    with pytest.raises(P.FkError) as e:
+        P.fk_layernorm_rows_plan(2, 10, 7)
+    assert e.value.status == P.FK_ERR_UNSUPPORTED_DTYPE
+    with pytest.raises(P.FkError):
+        P.fk_layernorm_rows_plan(2, 0, 0)
