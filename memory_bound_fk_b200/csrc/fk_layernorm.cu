@@ -25,7 +25,8 @@
 // make it.
 //
 // Three shapes, chosen by row length as for softmax: one warp per row (up to
-// 1024 fp32 / 2048 bf16 columns), one block per row (up to 32768 columns),
+// 1024 columns; a forced warp plan holds up to 1024 fp32 / 2048 bf16), one
+// block per row (up to 32768 columns),
 // and for longer rows one 512-thread block per row that streams the row
 // twice: a statistics pass that keeps a running (count, mean, M2) of x - p
 // per thread (p: the mean of the row's first chunk), merging each
