@@ -239,11 +239,16 @@ FK_API fk_status fk_softmax_rows_ws(const void *x, void *y, size_t rows, size_t 
  *   (few or very long rows) needs scratch; here it is a fixed 1 MiB device
  *   array inside the library (131072 (max, sum) pairs), which every GPU that
  *   loads the library holds until the process exits.  Rows are processed in
- *   batches whose partials fit it; a shape whose single row needs more than
- *   131072 chunks (rows far beyond 2^33 elements) returns FK_ERR_INVALID_ARG.
+ *   batches whose partials fit it; a row of more than 2^35 elements (which
+ *   would need more than 131072 chunks; a chunk holds at most 262144
+ *   elements) returns FK_ERR_INVALID_ARG.  Every check,
+ *   including that x and y lie wholly inside device allocations, runs before
+ *   the first batch is enqueued, so a call that returns an error has written
+ *   nothing.
  *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, once per device, with that device current); make
- *   that first call before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and keeps it; a lookup
+ *   that fails is retried by the next call.  Make that first call before any
+ *   stream capture.
  *   All calls on a device share the array and it keeps the last call's
  *   contents (nothing in it needs clearing: each call writes every partial
  *   it reads before reading it).  Calls whose kernels overlap on the GPU --
@@ -373,7 +378,10 @@ FK_API fk_status fk_attention_fwd(const void *q, const void *k, const void *v, v
  *          since the library was loaded or last reset.
  *   reset  nonzero: set the count back to 0 after reading it.
  * Synchronous; call after the work of interest has completed.  A nonzero
- * count in normal operation means a partner block never arrived.
+ * count in normal operation means a partner block never arrived.  A call
+ * whose wait gave up still returns FK_OK (the give-up happens on the GPU,
+ * after the call has returned), so callers that must detect it read this
+ * count after synchronising.
  */
 FK_API fk_status fk_wait_timeouts(unsigned int *count, int reset);
 

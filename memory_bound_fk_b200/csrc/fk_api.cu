@@ -158,6 +158,11 @@ fk_status check_call(const void* x, const void* y, size_t count, size_t esize,
 
 }  // namespace
 
+fk_status validate_call(const void* x, const void* y, size_t count, size_t esize) {
+  const DeviceInfo* dev = nullptr;
+  return check_call(x, y, count, esize, &dev);
+}
+
 const DeviceInfo* current_device_info(int* device_out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -22,6 +22,11 @@ struct DeviceInfo {
 // Properties of the current device; nullptr if there is none.
 const DeviceInfo* current_device_info(int* device_out);
 
+// The checks every (x, y) entry point runs for `count` elements of `esize`
+// bytes: non-null, element-aligned, no partial overlap, an sm_100 current
+// device, and both spans inside device-accessible allocations.
+fk_status validate_call(const void* x, const void* y, size_t count, size_t esize);
+
 // ---- GELU --------------------------------------------------------------
 // y[i] = GELU(x[i]) for i < n, dtype FK_F32 / FK_BF16, kind FK_GELU_TANH /
 // FK_GELU_ERF.  Arguments already validated.

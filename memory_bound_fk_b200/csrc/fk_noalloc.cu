@@ -30,23 +30,27 @@ static_assert(kNoAllocPartials * sizeof(float2) == (size_t{1} << 20), "1 MiB of 
 static __device__ __align__(256) float2 g_noalloc_scratch[kNoAllocPartials];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_setup_once[kMaxDevices];
+std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
-cudaError_t g_setup_error[kMaxDevices] = {};
 
 // Device address of the scratch array on device `dev`, which must be the
 // current device.  (In host code the array's name is only a host-side
 // stand-in; a kernel given it would read the wrong memory or fault.)
-// Looked up once per device.
+// A successful lookup is kept for the life of the process; a failed one
+// (for example inside a stream capture) is not, and the next call retries.
 void* scratch_address(int dev, cudaError_t* err) {
-  std::call_once(g_setup_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  *err = cudaSuccess;
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_setup_error[dev] = e;
-    g_scratch_ptr[dev] = (e == cudaSuccess) ? p : nullptr;
-    if (e != cudaSuccess) (void)cudaGetLastError();
-  });
-  *err = g_setup_error[dev];
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      *err = e;
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
   return g_scratch_ptr[dev];
 }
 
@@ -65,11 +69,15 @@ extern "C" fk_status fk_softmax_rows_noalloc(const void* x, void* y, size_t rows
     // every other path keeps its state on chip: nothing to allocate
     return fk_softmax_rows_ws(x, y, rows, cols, dtype, &plan, nullptr, 0, stream);
   }
-  // The split path in batches of rows whose partials fit the scratch array
-  // (each batch is checked against the array's size before anything runs);
-  // a single row with more chunks than the array holds is refused.
+  // The split path in batches of rows whose partials fit the scratch array;
+  // a single row with more chunks than the array holds (more than 2^35
+  // elements) is refused.  The whole of x and y is checked before the first
+  // batch is enqueued, so a rejected call writes nothing.
   const fk::SplitGeometry g = fk::split_geometry(rows, cols, dtype);
   if (g.nchunks > fk::kNoAllocPartials) return FK_ERR_INVALID_ARG;
+  const size_t esize = dtype == FK_F32 ? 4 : 2;
+  st = fk::validate_call(x, y, rows * cols, esize);
+  if (st != FK_OK) return st;
   const size_t rows_per_batch = fk::kNoAllocPartials / g.nchunks;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= fk::kMaxDevices) {
@@ -78,18 +86,18 @@ extern "C" fk_status fk_softmax_rows_noalloc(const void* x, void* y, size_t rows
   }
   cudaError_t err = cudaSuccess;
   void* scratch = fk::scratch_address(dev, &err);
-  if (scratch == nullptr || err != cudaSuccess) return FK_ERR_CUDA;
-  const size_t esize = dtype == FK_F32 ? 4 : 2;
+  if (scratch == nullptr) return FK_ERR_CUDA;
   const char* xb = static_cast<const char*>(x);
   char* yb = static_cast<char*>(y);
   for (size_t r0 = 0; r0 < rows; r0 += rows_per_batch) {
     const size_t n = (rows - r0 < rows_per_batch) ? rows - r0 : rows_per_batch;
-    // each batch plans its own chunking for its rows
+    // each batch plans its own chunking for its rows; its partials fit the
+    // array (n * chunks(n) <= 131072 for every n up to rows_per_batch)
     fk_softmax_plan p = plan;
     p.chunks = 0;
     const size_t off = r0 * cols * esize;
-    st = fk_softmax_rows_ws(xb == nullptr ? nullptr : xb + off, yb == nullptr ? nullptr : yb + off, n, cols,
-                            dtype, &p, scratch, fk::kNoAllocPartials * sizeof(float2), stream);
+    st = fk_softmax_rows_ws(xb + off, yb + off, n, cols, dtype, &p, scratch, fk::kNoAllocPartials * sizeof(float2),
+                            stream);
     if (st != FK_OK) return st;
   }
   return FK_OK;

@@ -251,9 +251,13 @@ __device__ __forceinline__ void exchange_init(ClusterExchange& ex) {
 // barrier (so every receiver's mbarrier is initialised), pushes this
 // block's (m, l) into every other block's inbox with st.async, waits
 // (bounded) for the other blocks' pushes, and returns the merged (M, L) of
-// the row.  A block exits only after all pushes addressed to it have
-// landed, and it pushes only to blocks that are waiting for it, so no block
-// touches the shared memory of a block that has exited.
+// the row.  When every partner arrives within the wait's limit, a block
+// exits only after all pushes addressed to it have landed, and it pushes
+// only to blocks that are waiting for it, so no block touches the shared
+// memory of a block that has exited.  A wait that gives up (a partner did
+// not arrive within 1 s) is counted in g_wait_timeouts and the block goes on
+// with the partials it has; the call still returns FK_OK, so the count
+// (fk_wait_timeouts) is how a caller learns that a row may be wrong.
 __device__ __forceinline__ float2 exchange_merge(ClusterExchange& ex, float m, float l, int csize, int crank,
                                                  float k) {
   const int t = threadIdx.x, lane = t & 31;

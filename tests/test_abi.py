@@ -162,6 +162,38 @@ def test_split_plan_and_workspace(fk):
         P.fk_softmax_rows_workspace(1, 10, 9)
 
 
+NOALLOC_PAIRS = 131072  # the allocation-free entry point's scratch: 1 MiB of (max, sum) pairs
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_noalloc_batches_fit_its_scratch_array(fk, dtype):
+    """fk_softmax_rows_noalloc runs split-path shapes in batches of
+    floor(131072 / chunks) rows, each batch planned for its own row count.
+    Every batch size it can form -- the full batch and every shorter last
+    batch -- must need at most the array's 1 MiB of workspace (host-only
+    planning through the C ABI).  The multi-batch loop engages only when
+    rows * chunks exceeds 131072, e.g. more than 8192 rows of 4M columns
+    (64 GiB of bf16 input), so this planning check is how it is tested."""
+    P = fk
+    split = P.make_plan(P.FK_PATH_SPLIT)
+    for cols in (524289, 1 << 20, 3_000_001, 1 << 22, 5_000_001, 1 << 24, 1 << 28, 1 << 35):
+        for rows in (1, 2, 3, 4, 7, 64, 1183, 1184, 1185, 5000, 8192, 8193, 20000, 100_000, 1_000_003):
+            plan = P.fk_softmax_rows_plan(rows, cols, dtype).as_dict()
+            if plan["path"] != "split":
+                continue
+            per_batch = NOALLOC_PAIRS // plan["chunks"]
+            assert per_batch >= 1
+            last = rows % per_batch
+            sizes = {min(per_batch, rows), last or per_batch, 1}
+            sizes |= {n for n in (2, 3, 4, 100, 1183, 1184, 1185) if n <= min(per_batch, rows)}
+            for n in sizes:
+                need = P.fk_softmax_rows_workspace(n, cols, dtype, split)
+                assert 0 < need <= NOALLOC_PAIRS * 8, (rows, cols, n, need)
+    # the longest row the array serves: 2^35 elements in 131072 chunks
+    assert P.fk_softmax_rows_plan(1, 1 << 35, dtype, P.FK_PATH_SPLIT).as_dict()["chunks"] == NOALLOC_PAIRS
+    assert P.fk_softmax_rows_plan(1, (1 << 35) + 1, dtype, P.FK_PATH_SPLIT).as_dict()["chunks"] > NOALLOC_PAIRS
+
+
 def _layernorm_rule(cols, dtype):
     """The documented LayerNorm plan: one warp per row up to 1024 columns;
     one block per row up to 32768 (16 values per thread up to 2048 columns,
