@@ -293,10 +293,13 @@ def _slice(name, arr, frac):
     return arr[:r]
 
 
-def oracle_run(names, inputs, frac, threads):
+def oracle_run(names, inputs, frac, threads, keep=False):
+    """The oracle over the leading fraction `frac` of every workload, timed;
+    with keep=True its outputs (fp32 values or bf16 bit patterns, rounded
+    once from double) are returned too, for the max-error check."""
     import oracle
     from memory_bound_fk_b200 import synth
-    total_bytes, elems = 0, 0
+    total_bytes, elems, outputs = 0, 0, {}
     t0 = time.perf_counter()
     for n in names:
         w = synth.WORKLOADS[n]
@@ -304,23 +307,54 @@ def oracle_run(names, inputs, frac, threads):
         if w.op in ("gelu", "gelu_erf"):
             f64 = oracle.gelu_tanh_f64 if w.op == "gelu" else oracle.gelu_erf_f64
             if w.dtype == "f32":
-                oracle.round_to_f32(f64(x.astype(np.float64), nthreads=threads))
+                y = oracle.round_to_f32(f64(x.astype(np.float64), nthreads=threads))
             else:
-                oracle.round_to_bf16(f64(oracle.bf16_to_f64(x), nthreads=threads))
+                y = oracle.round_to_bf16(f64(oracle.bf16_to_f64(x), nthreads=threads))
         elif w.op.startswith("softmax_causal"):
-            oracle.softmax_rows_causal(x, 1.0, x.shape[1], 0, nthreads=threads)
+            y = oracle.softmax_rows_causal(x, 1.0, x.shape[1], 0, nthreads=threads)
         elif w.op.startswith("layernorm"):
             g, b = synth.layernorm_params(x.shape[1], w.seed)
-            oracle.layernorm_rows(x, LN_EPS, g, b, "tanh" if w.op == "layernorm_gelu" else None,
-                                  nthreads=threads)
+            y = oracle.layernorm_rows(x, LN_EPS, g, b, "tanh" if w.op == "layernorm_gelu" else None,
+                                      nthreads=threads)
         elif w.dtype == "f32":
-            oracle.softmax_rows_f32(x, nthreads=threads)
+            y = oracle.softmax_rows_f32(x, nthreads=threads)
         else:
-            oracle.softmax_rows_bf16(x, nthreads=threads)
+            y = oracle.softmax_rows_bf16(x, nthreads=threads)
+        if keep:
+            outputs[n] = y
         total_bytes += workload_bytes(w, x.shape)
         elems += x.size
     dt = time.perf_counter() - t0
-    return {"seconds": dt, "bytes": total_bytes, "elements": elems}
+    return {"seconds": dt, "bytes": total_bytes, "elements": elems, "outputs": outputs}
+
+
+def bf16_ordinal(bits: np.ndarray) -> np.ndarray:
+    """Monotone integer encoding of bf16 bit patterns (adjacent values differ by 1)."""
+    b = bits.astype(np.int32)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def max_error(gpu: np.ndarray, ref: np.ndarray, dtype: str, chunk: int = 1 << 24) -> dict:
+    """Largest deviation of GPU outputs from the oracle's correctly rounded
+    outputs: absolute error for fp32, distance in bf16 ulps for bf16.  NaN
+    must sit at the same places on both sides.  Works through the arrays in
+    pieces of `chunk` elements to bound host memory."""
+    g_all, r_all = gpu.reshape(-1), ref.reshape(-1)
+    worst, nan_mismatch = 0, 0
+    for i in range(0, g_all.size, chunk):
+        if dtype == "bf16":
+            g, r = g_all[i:i + chunk].view(np.uint16), r_all[i:i + chunk].view(np.uint16)
+            gn, rn = (g & 0x7FFF) > 0x7F80, (r & 0x7FFF) > 0x7F80
+            d = np.where(gn | rn, 0, np.abs(bf16_ordinal(g) - bf16_ordinal(r)))
+            worst = max(worst, int(d.max(initial=0)))
+        else:
+            g, r = g_all[i:i + chunk].astype(np.float64), r_all[i:i + chunk].astype(np.float64)
+            gn, rn = np.isnan(g), np.isnan(r)
+            d = np.where(gn | rn, 0.0, np.abs(g - r))
+            worst = max(worst, float(d.max(initial=0.0)))
+        nan_mismatch += int(np.count_nonzero(gn != rn))
+    key = "max_ulp_bf16" if dtype == "bf16" else "max_abs"
+    return {key: worst, "nan_mismatch": nan_mismatch}
 
 
 def host_threads() -> int:
@@ -342,6 +376,44 @@ def make_inputs(names, rows=None):
 
 # ---------------------------------------------------------------- our arm
 
+class L2Cleaner:
+    """Leaves the L2 holding nothing of the timed work: a read-only pass (a
+    sum) over a buffer of 4x the L2 size, so that every dirty line left by
+    earlier kernels is written back and evicted before the timed launch,
+    whose own time then excludes other kernels' write-backs."""
+
+    def __init__(self, device, l2_bytes: int):
+        import torch
+        self.buf = torch.ones(max(4 * l2_bytes, 256 << 20) // 4, dtype=torch.float32, device=device)
+        self.out = torch.empty((), dtype=torch.float32, device=device)
+
+    def __call__(self):
+        import torch
+        torch.sum(self.buf, dim=0, out=self.out)
+
+
+def time_alone(call, stream, device, reps: int, cleaner) -> list[float]:
+    """reps launches of `call`, each after an L2 clean, each timed alone by
+    CUDA events on the launching stream (ms)."""
+    import torch
+    call()
+    ts = []
+    for _ in range(reps):
+        cleaner()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ts.append(a.elapsed_time(b))
+    return ts
+
+
+# Workloads timed one by one with the L2 cleaned before each launch: every
+# configuration of the pages' workloads, the small report-only ones too.
+ALONE = ["cfg1_gelu", "cfg1_softmax"] + SUITE
+
+
 def run_ours(args) -> dict | None:
     import numpy as np
     import torch
@@ -360,14 +432,16 @@ def run_ours(args) -> dict | None:
                                 device_id=device)
     fk.lib()  # fail loudly if libfk.so is missing
     names = workload_list(args.workload)
-    host = make_inputs(names, args.rows)
-    shapes = {n: host[n].shape for n in names}
+    alone_names = [n for n in (ALONE if args.workload == "suite" else names)] if not args.no_alone else []
+    all_names = names + [n for n in alone_names if n not in names]
+    host = make_inputs(all_names, args.rows)
+    shapes = {n: host[n].shape for n in all_names}
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
 
     # device buffers, inputs resident in HBM before the timed region
-    dev_in, dev_out, calls, params, keep = {}, {}, [], {}, []
-    for n in names:
+    dev_in, dev_out, call_of, params, keep = {}, {}, {}, {}, []
+    for n in all_names:
         w = synth.WORKLOADS[n]
         if w.dtype == "bf16":
             t = torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16)
@@ -380,20 +454,30 @@ def run_ours(args) -> dict | None:
             gb = [torch.from_numpy(a).to(device) for a in synth.layernorm_params(shapes[n][1], w.seed)]
             keep += gb
             params[n] = (gb[0].data_ptr(), gb[1].data_ptr())
-        calls.append((n, lambda w=w, xp=xp, yp=yp, shape=shapes[n], pr=params.get(n):
-                      launch_workload(fk, w, xp, yp, shape, sh, pr)))
+        call_of[n] = (lambda w=w, xp=xp, yp=yp, shape=shapes[n], pr=params.get(n):
+                      launch_workload(fk, w, xp, yp, shape, sh, pr))
+    calls = [(n, call_of[n]) for n in names]
+    # bytes of each input (rounded down to fk_copy's 16-byte granule; every
+    # full-size workload is a multiple of 16 already)
+    in_bytes = {n: dev_in[n].numel() * dev_in[n].element_size() // 16 * 16 for n in all_names}
+
+    def copy_call(n):
+        """fk_copy of a workload's input into its output buffer: the same
+        bytes read and written as the fused kernel, nothing computed."""
+        return lambda: fk.fk_copy(dev_in[n].data_ptr(), dev_out[n].data_ptr(), in_bytes[n], sh)
+
     bytes_step = sum(workload_bytes(synth.WORKLOADS[n], shapes[n]) for n in names)
     elems_step = sum(host[n].size for n in names)
 
-    def step(evs=None):
-        for i, (n, call) in enumerate(calls):
+    def step(seq, evs=None):
+        for i, (n, call) in enumerate(seq):
             if evs is not None:
                 evs[i].record(stream)
             st = call()
             if st != fk.FK_OK:
                 raise fk.FkError(st, n)
         if evs is not None:
-            evs[len(calls)].record(stream)
+            evs[len(seq)].record(stream)
 
     def barrier():
         if world > 1:
@@ -401,33 +485,65 @@ def run_ours(args) -> dict | None:
             dist.barrier()
         torch.cuda.synchronize(device)
 
+    def timed_steps(seq, steps):
+        """`steps` passes over seq between barriers; the total (ms) and, per
+        entry, the event time of every pass (the stretch from its launch to
+        the next entry's launch on the stream)."""
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)] for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        start.record(stream)
+        for k in range(steps):
+            step(seq, events[k])
+        stop.record(stream)
+        barrier()
+        per = [[evs[i].elapsed_time(evs[i + 1]) for evs in events] for i in range(len(seq))]
+        return start.elapsed_time(stop), per
+
     for _ in range(args.warmup):
-        step()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-              for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step(calls)
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     barrier()
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     time.sleep(0.25 if sampler else 0)  # let the sampler take its first reading
-    barrier()
-    start.record(stream)
-    for k in range(args.steps):
-        step(events[k])
-    stop.record(stream)
-    barrier()
+    total_ms, per_kernel = timed_steps(calls, args.steps)
     clocks = sampler.stop() if sampler else None
-    total_ms = start.elapsed_time(stop)
-    per_kernel_ms = [0.0] * len(calls)
-    for evs in events:
-        for i in range(len(calls)):
-            per_kernel_ms[i] += evs[i].elapsed_time(evs[i + 1])
-    reduced = max_over_ranks([total_ms] + per_kernel_ms, world, device)
-    max_ms, kernel_ms = reduced[0], reduced[1:]
+    # slowest rank: the total, then per kernel the sum, median and minimum
+    red = max_over_ranks([total_ms] + [sum(t) for t in per_kernel] + [statistics.median(t) for t in per_kernel]
+                         + [min(t) for t in per_kernel], world, device)
+    nk = len(calls)
+    max_ms, kernel_sum, kernel_med, kernel_min = red[0], red[1:1 + nk], red[1 + nk:1 + 2 * nk], red[1 + 2 * nk:]
+
+    # the copy floor of every slot: the same sequence with each kernel
+    # replaced by fk_copy of its bytes, so each copy follows the same
+    # predecessor traffic as the kernel it stands for
+    copy_seq = [(n, copy_call(n)) for n in names]
+    for _ in range(max(1, args.warmup)):
+        step(copy_seq)
+    copy_total, copy_per = timed_steps(copy_seq, args.steps)
+    red = max_over_ranks([copy_total] + [statistics.median(t) for t in copy_per], world, device)
+    copy_total, copy_med = red[0], red[1:]
+
+    # each workload alone, L2 cleaned before every launch
+    alone = {}
+    if alone_names:
+        cleaner = L2Cleaner(device, torch.cuda.get_device_properties(device).L2_cache_size)
+        reps = max(5, min(args.alone_reps, 200))
+        for n in alone_names:
+            def checked(c=call_of[n], n=n):
+                st = c()
+                if st != fk.FK_OK:
+                    raise fk.FkError(st, n)
+            tk = time_alone(checked, stream, device, reps, cleaner)
+            tc = time_alone(copy_call(n), stream, device, reps, cleaner)
+            red = max_over_ranks([statistics.median(tk), min(tk), statistics.median(tc), min(tc),
+                                  statistics.fmean(tk), statistics.fmean(tc)], world, device)
+            alone[n] = red
+        del cleaner
 
     # copy ceiling for the dominant kernel's bytes: cudaMemcpy D2D and
     # libfk's plain 16-byte copy, same buffers, timed the same way
-    dom_i = max(range(len(names)), key=lambda i: kernel_ms[i])
+    dom_i = max(range(len(names)), key=lambda i: kernel_sum[i])
     copy_ceiling = copy_reference(fk, dev_in[names[dom_i]], dev_out[names[dom_i]], stream, device, world)
 
     # end to end: pinned host buffers, copies inside the timed region
@@ -435,41 +551,85 @@ def run_ours(args) -> dict | None:
     if not args.no_e2e:
         e2e = run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_step, params)
 
-    cpu = None
+    # outputs of every workload as the timed kernels write them (the copy
+    # floor overwrote them), for the max-error check below
+    for n in all_names:
+        st = call_of[n]()
+        if st != fk.FK_OK:
+            raise fk.FkError(st, n)
+    torch.cuda.synchronize(device)
+
+    cpu, errors = None, {}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = host_threads()
-        f = oracle_sample_plan(names, host, args.cpu_budget, threads)
-        res = oracle_run(names, host, f, threads)
-        one = oracle_run(names, host, f / max(1, threads), 1)
+        f = oracle_sample_plan(all_names, host, args.cpu_budget, threads)
+        res = oracle_run(all_names, host, f, threads, keep=True)
+        one = oracle_run(all_names, host, f / max(1, threads), 1)
         cpu = {"value": res["bytes"] / res["seconds"] / 1e9, "unit": UNIT, "cores": threads,
                "value_1_thread": one["bytes"] / one["seconds"] / 1e9,
                "kind": "oracle",
                "sample": f"leading {100 * f:.3f}% of every workload ({res['elements']} elements, "
                          f"{res['bytes'] / 1e9:.3f} GB algorithmic, {res['seconds']:.1f} s)"}
+        # the GPU outputs of the same leading rows against the oracle's
+        for n, ref in res["outputs"].items():
+            w = synth.WORKLOADS[n]
+            got = dev_out[n][:ref.shape[0]]
+            got = got.view(torch.int16).cpu().numpy().view(np.uint16) if w.dtype == "bf16" else got.cpu().numpy()
+            errors[n] = dict(max_error(got, ref, w.dtype), elements_checked=int(ref.size))
 
     if rank != 0:
         return None
     peaks = measured_peaks()
+
+    def gbs_of(nbytes, ms):
+        return nbytes / (ms * 1e-3) / 1e9
+
+    def plan_of(n):
+        w = synth.WORKLOADS[n]
+        code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
+        if w.op.startswith("softmax"):
+            return fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
+        if w.op.startswith("layernorm"):
+            return fk.fk_layernorm_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
+        return {"path": "gelu"}
+
     kernels = []
     for i, n in enumerate(names):
         w = synth.WORKLOADS[n]
-        ms = kernel_ms[i] / args.steps
+        ms = kernel_sum[i] / args.steps
         nbytes = workload_bytes(w, shapes[n])
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        code = fk.FK_BF16 if w.dtype == "bf16" else fk.FK_F32
-        if w.op.startswith("softmax"):
-            plan = fk.fk_softmax_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
-        elif w.op.startswith("layernorm"):
-            plan = fk.fk_layernorm_rows_plan(shapes[n][0], shapes[n][1], code).as_dict()
-        else:
-            plan = {"path": "gelu"}
+        gbs = gbs_of(nbytes, ms)
+        plan = plan_of(n)
         kernels.append({"workload": n, "kernel": kernel_name(w, plan), "plan": plan,
                         "shape": list(shapes[n]), "ms": round(ms, 5), "GB_s": round(gbs, 1),
+                        "ms_median": round(kernel_med[i], 5), "ms_min": round(kernel_min[i], 5),
+                        "GB_s_median": round(gbs_of(nbytes, kernel_med[i]), 1),
                         "elements_per_s": round(host[n].size / (ms * 1e-3), 1),
                         "pct_of_8TBs": round(100 * gbs / SPEC_HBM_GBS, 2),
                         "frac_of_measured_copy": round(gbs / peaks["hbm_gbs"], 4),
+                        "copy_floor_same_slot_ms_median": round(copy_med[i], 5),
+                        "copy_floor_same_slot_GB_s": round(gbs_of(nbytes, copy_med[i]), 1),
+                        "frac_of_copy_floor_same_slot": round(copy_med[i] / kernel_med[i], 4),
                         "bytes_per_launch": nbytes})
-    dom = max(range(len(names)), key=lambda i: kernel_ms[i])
+    alone_rows = []
+    for n in alone_names:
+        w = synth.WORKLOADS[n]
+        nbytes = workload_bytes(w, shapes[n])
+        kmed, kmin, cmed, cmin, kmean, cmean = alone[n]
+        alone_rows.append({"workload": n, "kernel": kernel_name(w, plan_of(n)), "shape": list(shapes[n]),
+                           "bytes_per_launch": nbytes, "ms_median": round(kmed, 5), "ms_min": round(kmin, 5),
+                           "ms_mean": round(kmean, 5), "GB_s_mean": round(gbs_of(nbytes, kmean), 1),
+                           "fk_copy_ms_mean": round(cmean, 5), "frac_of_fk_copy_mean": round(cmean / kmean, 4),
+                           "GB_s_median": round(gbs_of(nbytes, kmed), 1), "GB_s_best": round(gbs_of(nbytes, kmin), 1),
+                           "pct_of_8TBs_median": round(100 * gbs_of(nbytes, kmed) / SPEC_HBM_GBS, 2),
+                           "frac_of_measured_peak": round(gbs_of(nbytes, kmed) / peaks["hbm_gbs"], 4),
+                           "fk_copy_ms_median": round(cmed, 5), "fk_copy_GB_s_median": round(gbs_of(nbytes, cmed), 1),
+                           "frac_of_fk_copy": round(cmed / kmed, 4),
+                           "elements_per_s": round(host[n].size / (kmed * 1e-3), 1),
+                           "max_error": errors.get(n)})
+    for k in kernels:
+        k["max_error"] = errors.get(k["workload"])
+    dom = max(range(len(names)), key=lambda i: kernel_sum[i])
     dk = kernels[dom]
     traffic, traffic_src = profiled_traffic(names[dom])
     value = aggregate_value(bytes_step, args.steps, world, max_ms)
@@ -487,6 +647,13 @@ def run_ours(args) -> dict | None:
         "pct_of_8TBs": round(100 * value / world / SPEC_HBM_GBS, 2),
         "elements_per_s": round(elems_step * args.steps * world / (max_ms * 1e-3), 1),
         "kernels": kernels,
+        "copy_floor_step": {"ms_per_step": round(copy_total / args.steps, 5),
+                            "GB_s": round(aggregate_value(bytes_step, args.steps, world, copy_total), 1),
+                            "what": "the same sequence with every kernel replaced by fk_copy of its bytes"},
+        "alone": {"l2": "L2 written back and evicted (read-only pass over 4x L2) before every launch",
+                  "timer": "CUDA events tick in steps of about 2 us on this GPU: for launches of tens of us "
+                           "the mean over the launches resolves finer than the median",
+                  "reps": max(5, min(args.alone_reps, 200)) if alone_names else 0, "workloads": alone_rows},
         "roofline": {"bound": "hbm", "kernel": dk["kernel"], "workload": names[dom],
                      "achieved": dk["GB_s"], "peak": peaks["hbm_gbs"], "unit": UNIT,
                      "frac": round(dk["GB_s"] / peaks["hbm_gbs"], 4),
@@ -889,6 +1056,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-chunk-mb", type=int, default=64,
                    help="input bytes per pipelined host<->device chunk in the e2e leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-alone", action="store_true", help="skip the per-workload L2-clean leg")
+    p.add_argument("--alone-reps", type=int, default=30, help="launches per workload in the L2-clean leg")
     p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     p.add_argument("--reference-budget", type=float, default=120.0,
                    help="seconds for the whole --impl reference run")

@@ -140,3 +140,21 @@ def test_source_digest_ignores_comments_and_layout_but_not_code():
     assert bench.code_text('int  a =\n 1;  /* x */') == bench.code_text('int a = 1; // y')
     assert bench.code_text('int a = 1;') != bench.code_text('int a = 2;')
     assert bench.code_text('asm("mov.u32 %0, 1;")') != bench.code_text('asm("mov.u32 %0, 2;")')
+
+
+def test_max_error_reports_abs_error_ulps_and_nan_placement():
+    import numpy as np
+    # fp32: absolute error, NaN compared by position only
+    g = np.array([1.0, 2.0, np.nan, 0.0], dtype=np.float32)
+    r = np.array([1.0, 2.25, np.nan, 0.0], dtype=np.float32)
+    assert bench.max_error(g, r, "f32", chunk=3) == {"max_abs": 0.25, "nan_mismatch": 0}
+    r2 = r.copy()
+    r2[3] = np.nan
+    assert bench.max_error(g, r2, "f32")["nan_mismatch"] == 1
+    # bf16: distance in the monotone encoding; -0 and +0 coincide, the
+    # smallest subnormals of either sign are 2 apart
+    gb = np.array([0x3F80, 0x8000, 0x8001, 0x7FC0], dtype=np.uint16)
+    rb = np.array([0x3F81, 0x0000, 0x0001, 0x7FC0], dtype=np.uint16)
+    assert bench.max_error(gb, rb, "bf16", chunk=2) == {"max_ulp_bf16": 2, "nan_mismatch": 0}
+    assert list(bench.bf16_ordinal(np.array([0xFF80, 0x8000, 0x0000, 0x7F80], dtype=np.uint16))) == \
+        [-0x7F80, 0, 0, 0x7F80]
