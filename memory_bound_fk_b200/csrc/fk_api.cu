@@ -186,7 +186,7 @@ fk_status fk_gelu(const void* x, void* y, size_t n, int dtype, int kind, void* s
   const fk::DeviceInfo* dev = nullptr;
   const fk_status st = fk::check_call(x, y, n, dtype == FK_F32 ? 4 : 2, &dev);
   if (st != FK_OK) return st;
-  const cudaError_t e = fk::launch_gelu(x, y, n, dtype, kind, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = fk::launch_gelu(x, y, n, dtype, kind, *dev, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 
@@ -198,7 +198,7 @@ fk_status fk_copy(const void* src, void* dst, size_t bytes, void* stream) {
   const fk::DeviceInfo* dev = nullptr;
   const fk_status st = fk::check_call(src, dst, bytes / 16, 16, &dev);
   if (st != FK_OK) return st;
-  const cudaError_t e = fk::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = fk::launch_copy(src, dst, bytes, *dev, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 
@@ -376,10 +376,11 @@ fk_status fk_wait_timeouts(unsigned int* count, int reset) {
   const fk::DeviceInfo* info = fk::current_device_info(&dev);
   if (info == nullptr || !info->ok) return FK_ERR_UNSUPPORTED_DEVICE;
   if (info->major != 10 || info->minor != 0) return FK_ERR_UNSUPPORTED_DEVICE;
-  unsigned a = 0, b = 0;
+  unsigned a = 0, b = 0, c = 0;
   cudaError_t e = fk::read_wait_timeouts(&a, reset != 0);
   if (e == cudaSuccess) e = fk::read_attention_wait_timeouts(&b, reset != 0);
-  *count = a + b;
+  if (e == cudaSuccess) e = fk::read_gelu_wait_timeouts(&c, reset != 0);
+  *count = a + b + c;
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 
@@ -409,7 +410,7 @@ fk_status fk_attention_fwd(const void* q, const void* k, const void* v, void* o,
     if (st != FK_OK) return st;
   }
   const cudaError_t e = fk::launch_attention(q, k, v, o, bh, t, static_cast<int>(d), causal != 0, scale,
-                                             static_cast<cudaStream_t>(stream));
+                                             dev->sm_count, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FK_OK : fk::cuda_fail(e);
 }
 

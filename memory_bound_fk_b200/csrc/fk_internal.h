@@ -29,11 +29,17 @@ fk_status validate_call(const void* x, const void* y, size_t count, size_t esize
 
 // ---- GELU --------------------------------------------------------------
 // y[i] = GELU(x[i]) for i < n, dtype FK_F32 / FK_BF16, kind FK_GELU_TANH /
-// FK_GELU_ERF.  Arguments already validated.
-cudaError_t launch_gelu(const void* x, void* y, size_t n, int dtype, int kind, cudaStream_t stream);
+// FK_GELU_ERF.  Arguments already validated; the device's L2 size and SM
+// count choose the path and size the grid.
+cudaError_t launch_gelu(const void* x, void* y, size_t n, int dtype, int kind, const DeviceInfo& dev,
+                        cudaStream_t stream);
 
 // dst <- src, bytes a multiple of 16 and both 16-byte aligned (validated).
-cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t stream);
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, const DeviceInfo& dev, cudaStream_t stream);
+
+// Threads whose bounded wait in the GELU / copy kernels gave up (see
+// read_wait_timeouts).
+cudaError_t read_gelu_wait_timeouts(unsigned* out, bool reset);
 
 // ---- softmax -----------------------------------------------------------
 constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
@@ -119,7 +125,7 @@ size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_pla
 // O = softmax(scale Q K^T, causal) V over bh slices of [t, d] bf16 rows
 // (validated: t % 128 == 0, d in {64, 128}, 16-byte aligned, bh * t < 2^31).
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* o, size_t bh, size_t t, int d,
-                             bool causal, float scale, cudaStream_t stream);
+                             bool causal, float scale, int sm_count, cudaStream_t stream);
 cudaError_t read_attention_wait_timeouts(unsigned* out, bool reset);
 
 // Number of threads whose bounded mbarrier wait gave up, on the current

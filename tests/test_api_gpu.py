@@ -89,6 +89,16 @@ def test_fk_copy_reference(fk, cuda_device):
     assert fk.fk_copy(x.data_ptr(), y.data_ptr(), nb, 0) == fk.FK_OK
     torch.cuda.synchronize()
     assert torch.equal(x, y)
+    # both data paths (through shared memory while source and destination fit
+    # in L2, through registers beyond), ragged last chunk, exact bytes only
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    for nbytes in (l2 // 2 - 48, l2 // 2 + 4096 + 16, 16, 16400):
+        a = torch.randint(0, 1 << 30, (nbytes // 4 + 64,), dtype=torch.int32, device="cuda")
+        b = torch.full_like(a, -1)
+        assert fk.fk_copy(a.data_ptr(), b.data_ptr(), nbytes, 0) == fk.FK_OK
+        torch.cuda.synchronize()
+        k = nbytes // 4
+        assert torch.equal(a[:k], b[:k]) and bool((b[k:] == -1).all()), nbytes
     assert fk.fk_copy(x.data_ptr(), y.data_ptr(), 0, 0) == fk.FK_OK
     assert fk.fk_copy(x.data_ptr(), y.data_ptr(), 24, 0) == fk.FK_ERR_INVALID_ARG      # not a multiple of 16
     assert fk.fk_copy(x.data_ptr() + 4, y.data_ptr(), 32, 0) == fk.FK_ERR_INVALID_ARG  # misaligned
