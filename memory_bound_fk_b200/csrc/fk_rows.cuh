@@ -30,19 +30,35 @@ __device__ __forceinline__ void load_chunks(const T* row, Idx vfirst, Idx ve, Id
   constexpr int VEC = Elem<T>::VEC;
   constexpr uint32_t kFill = ZERO ? 0u : Elem<T>::kNegInfWord;
   const float fill = ZERO ? 0.0f : -INFINITY;
+  if constexpr (ALIGNED) {
 #pragma unroll
-  for (int c = 0; c < VPT; ++c) {
-    if constexpr (ALIGNED) {
+    for (int c = 0; c < VPT; ++c) {
       const Idx vi = vfirst + static_cast<Idx>(c) * TEAM + t;
-      const Idx e = vi * VEC;
-      const bool live = MASK ? (vi < ve && e < lim) : (vi < ve);
+      const bool live = MASK ? (vi < ve && vi * VEC < lim) : (vi < ve);
       raw[c] = ld_stream_v4_if(row + static_cast<size_t>(vi) * VEC, live, kFill);
-      // vectors wholly past lim were not loaded (all -inf); only the one
-      // that straddles lim needs its tail masked
-      if constexpr (MASK) {
-        if (e < lim && lim - e < static_cast<Idx>(VEC)) raw[c] = Elem<T>::keep_first(raw[c], static_cast<int>(lim - e));
+    }
+    // Vectors wholly past lim were not loaded (all -inf); only the one that
+    // straddles lim needs its tail masked.  One thread of the team holds it,
+    // so the masking sits behind a warp vote: masking every vector in the
+    // unrolled loop (the selects run for all of them) added 40% to the
+    // instructions of causal 2048-column rows and made them issue-bound.
+    // Every caller runs this with all lanes of the warp converged.
+    if constexpr (MASK) {
+      const Idx vs = lim / VEC;  // the straddling vector, if lim % VEC != 0
+      const Idx off = vs - vfirst;
+      const bool mine = (lim % VEC != 0) && vs >= vfirst && vs < ve && off / TEAM < static_cast<Idx>(VPT) &&
+                        off % TEAM == static_cast<Idx>(t);
+      if (__any_sync(0xffffffffu, mine) && mine) {
+        const int cs = static_cast<int>(off / TEAM);
+        const int keep = static_cast<int>(lim % VEC);
+#pragma unroll
+        for (int c = 0; c < VPT; ++c)
+          if (c == cs) raw[c] = Elem<T>::keep_first(raw[c], keep);
       }
-    } else {
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < VPT; ++c) {
       const Idx e0 = (vfirst + static_cast<Idx>(c) * TEAM) * VEC + t;
       Idx eend = (ve * VEC < cols) ? ve * VEC : cols;
       if constexpr (MASK) eend = imin(eend, lim);
