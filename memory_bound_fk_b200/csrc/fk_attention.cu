@@ -52,7 +52,7 @@ namespace {
 constexpr int kAttnTileThreads = 128;                   // one softmax warpgroup per query tile
 constexpr int kAttnThreads = 3 * kAttnTileThreads;       // + the producer warpgroup
 constexpr int kMmaWarp = 8, kLoadWarp = 9;               // producer warps (10, 11 idle)
-constexpr int kSoftmaxRegs = 208, kProducerRegs = 72;    // setmaxnreg split of the launch's registers
+constexpr int kSoftmaxRegs = 208, kProducerRegs = 88;    // setmaxnreg split of the launch's registers
 constexpr int kSplitRegs = kAttnTileThreads * (2 * kSoftmaxRegs + kProducerRegs);
 static_assert(kSplitRegs <= 65536, "register split above the register file");
 constexpr int kAttnBlock = 128;                         // queries per tile = keys per step
@@ -197,10 +197,38 @@ __device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_co
   }
 }
 
+// The units of work, a pair of 128-query tiles of one slice, in the order
+// they are handed out: causal grids take the longest pairs (most key
+// blocks) first, across all slices; other grids keep the pairs of a slice
+// together, so that its K/V tiles are read from HBM once and then hit L2.
+// Each block is persistent and takes the units blockIdx.x, then
+// 2 G - 1 - blockIdx.x, then 2 G + blockIdx.x, ... (G blocks): a serpentine
+// that balances the decreasing causal unit lengths across blocks, and lets
+// a block start its next unit's loads while the current one finishes.
+struct AttnUnits {
+  int t, bh;  // keys (and queries) per slice, slices
+  bool causal;
+  __device__ __forceinline__ int nq() const { return t / 128; }
+  __device__ __forceinline__ int npair() const { return (nq() + 1) / 2; }
+  __device__ __forceinline__ int unit(int round) const {  // -1: no more units for this block
+    const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    const int u = round * g + ((round & 1) ? g - 1 - b : b);
+    return u < bh * npair() ? u : -1;
+  }
+  __device__ __forceinline__ int slice(int u) const { return causal ? u % bh : u / npair(); }
+  __device__ __forceinline__ int pair(int u) const { return causal ? npair() - 1 - u / bh : u % npair(); }
+  // key blocks of query tile i of unit u (0: the tile is absent, when nq is
+  // odd and this is the last pair)
+  __device__ __forceinline__ int nkv(int u, int i) const {
+    const int qb = 2 * pair(u) + i;
+    return qb < nq() ? (causal ? qb + 1 : nq()) : 0;
+  }
+};
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                         const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out, int t,
+                         const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out, int t, int bh,
                          float scale_log2) {
   constexpr int KC = D / 64;                     // 64-column chunks of a head row
   constexpr uint32_t TILE = KC * kChunkBytes;    // bytes of a 128 x D tile
@@ -208,8 +236,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_k[2], bar_v[2], bar_kfree[2], bar_vfree[2], bar_s[2], bar_p[2], bar_o[2],
-      bar_drain;
+  __shared__ uint64_t bar_q, bar_qfree, bar_k[2], bar_v[2], bar_kfree[2], bar_vfree[2], bar_s[2], bar_p[2],
+      bar_o[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -221,29 +249,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto sV = [&](int b) { return base + (4 + b) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int nq = t / kAttnBlock;
-  const int npair = (nq + 1) / 2;
-  // launch order: causal grids hand out the longest pairs (most key blocks)
-  // first, across all slices; other grids keep the pairs of a slice
-  // together, so its K/V tiles are read from HBM once and then hit L2
-  const int bh = static_cast<int>(gridDim.x) / npair;
-  const int lin = static_cast<int>(blockIdx.x);
-  const int slice = CAUSAL ? lin % bh : lin / npair;
-  const int pair = CAUSAL ? npair - 1 - lin / bh : lin % npair;
-  // query tiles 2 pair and 2 pair + 1 (the second absent when nq is odd and
-  // this is the last pair); key blocks per tile (0: absent)
-  auto nkv_of = [&](int i) {
-    const int qb = 2 * pair + i;
-    return qb < nq ? (CAUSAL ? qb + 1 : nq) : 0;
-  };
-  const int nkv0 = nkv_of(0), nkv1 = nkv_of(1);
-  const int nmax = nkv0 > nkv1 ? nkv0 : nkv1;
-  const int ntiles = nkv1 > 0 ? 2 : 1;
+  const AttnUnits units{t, bh, CAUSAL};
   volatile int* abort = &abort_flag;
 
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
   if (tid == 0) {
     mbar_init(&bar_q, 1);
+    mbar_init(&bar_qfree, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
@@ -262,107 +274,148 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
 
+  // Barrier phases run on from one unit to the next: Q and its "free"
+  // barrier complete once per unit, the K and V buffers are filled by one
+  // tile counter g across units (tile g in buffer g % 2), and S, P and O of
+  // each query tile count their phases across units.
   if (warp >= 2 * kAttnTileThreads / 32) {
     // ------------------------------------------------ producer warpgroup
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs) : "memory");
-    const int row0 = slice * t;  // first row of this slice in the [bh * t, D] view
     if (warp == kLoadWarp && (tid & 31) == 0) {
-      // ---- TMA loads: Q, then K_j and V_j into buffer j % 2 once the MMAs
-      // that read K_j-2 / V_j-2 have completed
-      mbar_arrive_expect_tx(&bar_q, ntiles * TILE);
-      for (int i = 0; i < ntiles; ++i) {
+      // ---- TMA loads: per unit, Q once the tensor cores are done with the
+      // previous unit's S products, then K_g and V_g into buffer g % 2 once
+      // the MMAs that read tile g - 2 have completed
+      int g = 0, nk = 0, nv = 0;  // K/V tiles issued (counted across units)
+      int nql = 0;                // Q loads issued
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int u = units.unit(round);
+        if (u < 0) break;
+        const int nkv0 = units.nkv(u, 0), nkv1 = units.nkv(u, 1);
+        const int nmax = nkv0 > nkv1 ? nkv0 : nkv1, ntiles = nkv1 > 0 ? 2 : 1;
+        const int row0 = units.slice(u) * t;  // first row of the slice in the [bh * t, D] view
+        const int pair = units.pair(u);
+        if (round > 0 && !attn_wait(&bar_qfree, (round - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bar_q, ntiles * TILE);
+        for (int i = 0; i < ntiles; ++i) {
 #pragma unroll
-        for (int c = 0; c < KC; ++c)
-          tc::tma_load_2d(sQ(i) + c * kChunkBytes, &tmq, &bar_q, c * 64, row0 + (2 * pair + i) * kAttnBlock);
+          for (int c = 0; c < KC; ++c)
+            tc::tma_load_2d(sQ(i) + c * kChunkBytes, &tmq, &bar_q, c * 64, row0 + (2 * pair + i) * kAttnBlock);
+        }
+        nql = round + 1;
+        for (int j = 0; j < nmax; ++j, ++g) {
+          const int b = g & 1;
+          if (g >= 2 && !attn_wait(&bar_kfree[b], ((g - 2) >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_k[b], TILE);
+#pragma unroll
+          for (int c = 0; c < KC; ++c)
+            tc::tma_load_2d(sK(b) + c * kChunkBytes, &tmk, &bar_k[b], c * 64, row0 + j * 128);
+          nk = g + 1;
+          if (g >= 2 && !attn_wait(&bar_vfree[b], ((g - 2) >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_v[b], TILE);
+#pragma unroll
+          for (int c = 0; c < KC; ++c)
+            tc::tma_load_2d(sV(b) + c * kChunkBytes, &tmv, &bar_v[b], c * 64, row0 + j * 128);
+          nv = g + 1;
+        }
       }
-      int nk = 0, nv = 0;  // K_0 .. K_nk-1, V_0 .. V_nv-1 issued
-      for (int j = 0; j < nmax; ++j) {
-        const int b = j & 1;
-        if (j >= 2 && !attn_wait(&bar_kfree[b], ((j - 2) >> 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bar_k[b], TILE);
-#pragma unroll
-        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sK(b) + c * kChunkBytes, &tmk, &bar_k[b], c * 64, row0 + j * 128);
-        nk = j + 1;
-        if (j >= 2 && !attn_wait(&bar_vfree[b], ((j - 2) >> 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bar_v[b], TILE);
-#pragma unroll
-        for (int c = 0; c < KC; ++c) tc::tma_load_2d(sV(b) + c * kChunkBytes, &tmv, &bar_v[b], c * 64, row0 + j * 128);
-        nv = j + 1;
-      }
-      // copies in flight land before the CTA exits.  A buffer is refilled only
-      // after the MMA warp has seen its previous load land, so only the last
-      // load into each buffer can be pending.
-      drain_wait(&bar_q, 0);
+      // copies in flight land before the CTA exits.  Q is reloaded only after
+      // the MMA warp has seen the previous Q land, and a K/V buffer is refilled
+      // only after it has seen that buffer's previous load land, so only the
+      // last Q load and the last load into each buffer can be pending.
+      if (nql > 0) drain_wait(&bar_q, (nql - 1) & 1);
       for (int j = nk > 2 ? nk - 2 : 0; j < nk; ++j) drain_wait(&bar_k[j & 1], (j >> 1) & 1);
       for (int j = nv > 2 ? nv - 2 : 0; j < nv; ++j) drain_wait(&bar_v[j & 1], (j >> 1) & 1);
     } else if (warp == kMmaWarp && (tid & 31) == 0) {
       // ---- MMA issue
-      int k_wt = 0, v_wt = 0;  // K_0 .. K_k_wt-1, V_0 .. V_v_wt-1 seen in shared memory
-      auto wait_k = [&](int j) {
-        if (j < k_wt) return true;
-        if (!attn_wait(&bar_k[j & 1], (j >> 1) & 1, abort)) return false;
-        k_wt = j + 1;
+      int k_wt = 0, v_wt = 0;  // K_0 .. K_k_wt-1, V_0 .. V_v_wt-1 (across units) seen in shared memory
+      auto wait_k = [&](int g) {
+        if (g < k_wt) return true;
+        if (!attn_wait(&bar_k[g & 1], (g >> 1) & 1, abort)) return false;
+        k_wt = g + 1;
         return true;
       };
-      auto wait_v = [&](int j) {
-        if (j < v_wt) return true;
-        if (!attn_wait(&bar_v[j & 1], (j >> 1) & 1, abort)) return false;
-        v_wt = j + 1;
+      auto wait_v = [&](int g) {
+        if (g < v_wt) return true;
+        if (!attn_wait(&bar_v[g & 1], (g >> 1) & 1, abort)) return false;
+        v_wt = g + 1;
         return true;
       };
-      auto last = [&](int j) { return j < nkv1 ? 1 : 0; };  // the tile that reads K_j and V_j last
       // shared-memory descriptors, low words (the high words are constants):
       // one per buffer, stepped through a tile by constant offsets
       constexpr uint32_t HI = tc::smem_desc_hi(1024);
       const uint32_t dq0 = tc::smem_desc_lo(smem_addr(sQ(0)), 16);
       const uint32_t dk0 = tc::smem_desc_lo(smem_addr(sK(0)), 16);
       const uint32_t dv0 = tc::smem_desc_lo(smem_addr(sV(0)), kChunkBytes);
-      // S_i = Q_i K_j^T into TMEM columns 256 i ..
-      auto issue_s = [&](int i, int j) {
-        const uint32_t dq = dq0 + i * (TILE >> 4), dk = dk0 + (j & 1) * (TILE >> 4);
-        const uint32_t ts = tmem + i * 256;
+      int np[2] = {0, 0};  // P arrivals waited for, per query tile (across units)
+      int g0 = 0;          // tile counter of the unit's first K/V tile
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int u = units.unit(round);
+        if (u < 0) break;
+        const int nkv0 = units.nkv(u, 0), nkv1 = units.nkv(u, 1);
+        const int nmax = nkv0 > nkv1 ? nkv0 : nkv1, ntiles = nkv1 > 0 ? 2 : 1;
+        int s_left = nkv0 + nkv1;  // S products of the unit still to issue
+        auto last = [&](int j) { return j < nkv1 ? 1 : 0; };  // the tile that reads K_j and V_j last
+        // S_i = Q_i K_j^T into TMEM columns 256 i ..; after the unit's last
+        // one, Q may be reloaded once it completes
+        auto issue_s = [&](int i, int j) {
+          const uint32_t dq = dq0 + i * (TILE >> 4), dk = dk0 + ((g0 + j) & 1) * (TILE >> 4);
+          const uint32_t ts = tmem + i * 256;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = ((ks / 4) * kChunkBytes + (ks % 4) * 32) >> 4;
-          tc::mma_bf16(ts, tc::desc_join(dq + off, HI), tc::desc_join(dk + off, HI), IDESC_S, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&bar_s[i]);
-        if (i == last(j)) tc::mma_commit(&bar_kfree[j & 1]);
-      };
-      // O_i += P_i V_j: P_i (TMEM, 8 columns per 16 keys), V_j MN-major in smem
-      auto issue_o = [&](int i, int j) {
-        const uint32_t dv = dv0 + (j & 1) * (TILE >> 4);
-        const uint32_t to = tmem + i * 256 + 128, tp = tmem + i * 256;
-        const uint32_t acc0 = j > 0 ? 1u : 0u;
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = ((ks / 4) * kChunkBytes + (ks % 4) * 32) >> 4;
+            tc::mma_bf16(ts, tc::desc_join(dq + off, HI), tc::desc_join(dk + off, HI), IDESC_S, ks > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bar_s[i]);
+          if (i == last(j)) tc::mma_commit(&bar_kfree[(g0 + j) & 1]);
+          if (--s_left == 0) tc::mma_commit(&bar_qfree);
+        };
+        // O_i += P_i V_j: P_i (TMEM, 8 columns per 16 keys), V_j MN-major in smem.
+        // The unit's first one overwrites O_i, which the previous unit's
+        // epilogue has read by then: its softmax warpgroup arrives on P_i only
+        // after that epilogue.
+        auto issue_o = [&](int i, int j) {
+          const uint32_t dv = dv0 + ((g0 + j) & 1) * (TILE >> 4);
+          const uint32_t to = tmem + i * 256 + 128, tp = tmem + i * 256;
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-        for (int ks = 0; ks < kAttnBlock / 16; ++ks)
-          tc::mma_bf16_ts(to, tp + ks * 8, tc::desc_join(dv + ((ks * 2048) >> 4), HI), IDESC_O, ks > 0 ? 1u : acc0);
-        if (i == last(j)) tc::mma_commit(&bar_vfree[j & 1]);
-      };
+          for (int ks = 0; ks < kAttnBlock / 16; ++ks)
+            tc::mma_bf16_ts(to, tp + ks * 8, tc::desc_join(dv + ((ks * 2048) >> 4), HI), IDESC_O, ks > 0 ? 1u : acc0);
+          if (i == last(j)) tc::mma_commit(&bar_vfree[(g0 + j) & 1]);
+        };
 
-      bool ok = attn_wait(&bar_q, 0, abort) && wait_k(0);
-      if (ok) {
+        ok = attn_wait(&bar_q, round & 1, abort) && wait_k(g0);
+        if (!ok) break;
         tc::fence_after_sync();
         for (int i = 0; i < ntiles; ++i) issue_s(i, 0);
-      }
-      for (int j = 0; ok && j < nmax; ++j) {
+        for (int j = 0; ok && j < nmax; ++j) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int nkv_i = i == 0 ? nkv0 : nkv1;
-          if (!ok || j >= nkv_i) continue;
-          // the tiles first (long since loaded: their loads wait only on
-          // MMAs already issued), then softmax i's block j: P_i,j written,
-          // O_i rescaled.  The two MMA groups then go out back to back.
-          ok = wait_v(j) && (j + 1 >= nkv_i || wait_k(j + 1)) && attn_wait(&bar_p[i], j & 1, abort);
-          if (!ok) break;
-          tc::fence_after_sync();
-          issue_o(i, j);
-          if (j + 1 < nkv_i) {
-            issue_s(i, j + 1);
-          } else {
-            tc::mma_commit(&bar_o[i]);
+          for (int i = 0; i < 2; ++i) {
+            const int nkv_i = i == 0 ? nkv0 : nkv1;
+            if (!ok || j >= nkv_i) continue;
+            // the tiles first (long since loaded: their loads wait only on
+            // MMAs already issued), then softmax i's block j: P_i,j written,
+            // O_i rescaled.  The two MMA groups then go out back to back.
+            ok = wait_v(g0 + j) && (j + 1 >= nkv_i || wait_k(g0 + j + 1)) && attn_wait(&bar_p[i], np[i] & 1, abort);
+            if (!ok) break;
+            ++np[i];
+            tc::fence_after_sync();
+            issue_o(i, j);
+            if (j + 1 < nkv_i) {
+              issue_s(i, j + 1);
+            } else {
+              tc::mma_commit(&bar_o[i]);
+            }
           }
         }
+        g0 += nmax;
       }
       // every MMA completes before the CTA exits
       tc::mma_commit(&bar_drain);
@@ -370,43 +423,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ softmax warpgroup i: query tile 2 pair + i
+    // ------------------------------------------------ softmax warpgroup i: query tile 2 pair + i of each unit
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs) : "memory");
     const int i = warp >> 2;
     const int r = ((warp & 3) << 5) | (tid & 31);
     const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane + i * 256, tO = tS + 128;
-    const int qb = 2 * pair + i;
-    const int nkv_i = i == 0 ? nkv0 : nkv1;
-    float m_i = -INFINITY, l_i = 0.0f;
-    for (int j = 0; j < nkv_i; ++j) {
-      attn_wait(&bar_s[i], j & 1, abort);
-      if (!__any_sync(0xffffffffu, *abort)) {
-        if (CAUSAL && j == qb)
-          softmax_block<true>(tS, tO, D, r, j, scale_log2, m_i, l_i);
-        else
-          softmax_block<false>(tS, tO, D, r, j, scale_log2, m_i, l_i);
+    int ns = 0, no = 0;  // S and O phases waited for (across units)
+    for (int round = 0;; ++round) {
+      const int u = units.unit(round);
+      if (u < 0) break;
+      const int qb = 2 * units.pair(u) + i;
+      const int nkv_i = units.nkv(u, i);
+      float m_i = -INFINITY, l_i = 0.0f;
+      for (int j = 0; j < nkv_i; ++j, ++ns) {
+        attn_wait(&bar_s[i], ns & 1, abort);
+        if (!__any_sync(0xffffffffu, *abort)) {
+          if (CAUSAL && j == qb)
+            softmax_block<true>(tS, tO, D, r, j, scale_log2, m_i, l_i);
+          else
+            softmax_block<false>(tS, tO, D, r, j, scale_log2, m_i, l_i);
+        }
+        tc::fence_before_sync();
+        mbar_arrive(&bar_p[i]);
       }
-      tc::fence_before_sync();
-      mbar_arrive(&bar_p[i]);
-    }
-    if (nkv_i > 0) {
-      attn_wait(&bar_o[i], 0, abort);
-      if (!__any_sync(0xffffffffu, *abort)) {
-        tc::fence_after_sync();
-        // O / l, rounded to bf16: row r of the tile
-        const float inv = 1.0f / l_i;
-        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(slice) * t + qb * kAttnBlock + r) * D);
+      if (nkv_i > 0) {
+        attn_wait(&bar_o[i], no & 1, abort);
+        ++no;
+        if (!__any_sync(0xffffffffu, *abort)) {
+          tc::fence_after_sync();
+          // O / l, rounded to bf16: row r of the tile
+          const float inv = 1.0f / l_i;
+          uint4* dst =
+              reinterpret_cast<uint4*>(out + (static_cast<size_t>(units.slice(u)) * t + qb * kAttnBlock + r) * D);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(tO + c * 32, v);
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tc::tmem_ld32(tO + c * 32, v);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[c * 4 + q] = make_uint4(pack_bf16x2(v[8 * q] * inv, v[8 * q + 1] * inv),
-                                        pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv),
-                                        pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
-                                        pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
+            for (int q = 0; q < 4; ++q)
+              dst[c * 4 + q] = make_uint4(pack_bf16x2(v[8 * q] * inv, v[8 * q + 1] * inv),
+                                          pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv),
+                                          pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
+                                          pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
+          }
+          // the next unit's first O product overwrites O: its tcgen05.ld
+          // reads have completed (tmem_ld32 waits for them) before this
+          // warpgroup's next arrival on P
+          tc::fence_before_sync();
         }
       }
     }
@@ -451,7 +515,7 @@ bool make_map(CUtensorMap* m, const void* ptr, size_t rows, int d) {
 
 template <int D, bool CAUSAL>
 cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, size_t bh,
-                        size_t t, float scale_log2, cudaStream_t s) {
+                        size_t t, float scale_log2, int sm_count, cudaStream_t s) {
   constexpr uint32_t TILE = (D / 64) * kChunkBytes;
   const size_t smem = 6 * TILE + 1024;
   auto kernel = attention_fwd_kernel<D, CAUSAL>;
@@ -464,26 +528,31 @@ cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (fa.numRegs * kAttnThreads < kSplitRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(bh * ((t / kAttnBlock + 1) / 2)));
-  kernel<<<grid, kAttnThreads, smem, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(t),
-                                          scale_log2);
+  // persistent blocks, one per SM (the kernel holds all of an SM's tensor
+  // memory), each walking its units
+  const size_t nunits = bh * ((t / kAttnBlock + 1) / 2);
+  const size_t grid = nunits < static_cast<size_t>(sm_count) ? nunits : static_cast<size_t>(sm_count);
+  kernel<<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
+                                                                 static_cast<int>(t), static_cast<int>(bh),
+                                                                 scale_log2);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* o, size_t bh, size_t t, int d,
-                             bool causal, float scale, cudaStream_t stream) {
+                             bool causal, float scale, int sm_count, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, bh * t, d) || !make_map(&mk, k, bh * t, d) || !make_map(&mv, v, bh * t, d))
     return cudaErrorInvalidValue;
   const float sl2 = static_cast<float>(static_cast<double>(scale) * 1.44269504088896340736);
+  const int sms = sm_count > 0 ? sm_count : 1;
   if (d == 64) {
-    return causal ? launch_attn<64, true>(mq, mk, mv, o, bh, t, sl2, stream)
-                  : launch_attn<64, false>(mq, mk, mv, o, bh, t, sl2, stream);
+    return causal ? launch_attn<64, true>(mq, mk, mv, o, bh, t, sl2, sms, stream)
+                  : launch_attn<64, false>(mq, mk, mv, o, bh, t, sl2, sms, stream);
   }
-  return causal ? launch_attn<128, true>(mq, mk, mv, o, bh, t, sl2, stream)
-                : launch_attn<128, false>(mq, mk, mv, o, bh, t, sl2, stream);
+  return causal ? launch_attn<128, true>(mq, mk, mv, o, bh, t, sl2, sms, stream)
+                : launch_attn<128, false>(mq, mk, mv, o, bh, t, sl2, sms, stream);
 }
 
 cudaError_t read_attention_wait_timeouts(unsigned* out, bool reset) {
