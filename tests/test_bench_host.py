@@ -158,3 +158,12 @@ def test_max_error_reports_abs_error_ulps_and_nan_placement():
     assert bench.max_error(gb, rb, "bf16", chunk=2) == {"max_ulp_bf16": 2, "nan_mismatch": 0}
     assert list(bench.bf16_ordinal(np.array([0xFF80, 0x8000, 0x0000, 0x7F80], dtype=np.uint16))) == \
         [-0x7F80, 0, 0, 0x7F80]
+
+
+def test_rotation_sets_cover_four_times_the_l2():
+    l2 = 126 << 20
+    assert bench.rotation_sets(9462349824, l2) == 1          # the suite: one step is 9.5 GB
+    assert bench.rotation_sets(4 * l2, l2) == 1
+    k = bench.rotation_sets(64 << 20, l2)                     # 32 MiB in + 32 MiB out
+    assert k * (64 << 20) >= 4 * l2 and (k - 1) * (64 << 20) < 4 * l2
+    assert bench.rotation_sets(1, l2) == 64                   # capped
