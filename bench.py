@@ -512,12 +512,16 @@ def run_ours(args) -> dict | None:
             dist.barrier()
         torch.cuda.synchronize(device)
 
-    def timed_steps(seqs, steps):
+    def timed_steps(seqs, steps, per_kernel=True):
         """`steps` passes, pass k over seqs[k % len(seqs)], between barriers;
-        the total (ms) and, per entry, the event time of every pass (the
-        stretch from its launch to the next entry's launch on the stream)."""
+        the total (ms) and, with per_kernel, per entry the event time of
+        every pass (the stretch from its launch to the next entry's launch
+        on the stream).  Every event recorded between two kernels holds the
+        stream for ~2.6 us on this GPU, so the pass that gives the total of
+        a measurement has none (per_kernel=False)."""
         n = len(seqs[0])
-        events = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)] \
+            if per_kernel else [None] * steps
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         start.record(stream)
@@ -525,7 +529,7 @@ def run_ours(args) -> dict | None:
             step(seqs[k % len(seqs)], events[k])
         stop.record(stream)
         barrier()
-        per = [[evs[i].elapsed_time(evs[i + 1]) for evs in events] for i in range(n)]
+        per = [[evs[i].elapsed_time(evs[i + 1]) for evs in events] for i in range(n)] if per_kernel else None
         return start.elapsed_time(stop), per
 
     for k in range(max(args.warmup, min(len(calls), 64))):
@@ -534,28 +538,36 @@ def run_ours(args) -> dict | None:
     barrier()
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     time.sleep(0.25 if sampler else 0)  # let the sampler take its first reading
-    total_ms, per_kernel = timed_steps(calls, args.steps)
+    # the timed region: K steps, events only at its ends
+    total_ms, _ = timed_steps(calls, args.steps, per_kernel=False)
+    # per-kernel breakdown: K more steps with an event between every two kernels
+    ev_total_ms, per_kernel = timed_steps(calls, args.steps)
     clocks = sampler.stop() if sampler else None
-    # slowest rank: the total, then per kernel the sum, median and minimum
-    red = max_over_ranks([total_ms] + [sum(t) for t in per_kernel] + [statistics.median(t) for t in per_kernel]
-                         + [min(t) for t in per_kernel], world, device)
+    # slowest rank: the totals, then per kernel the sum, median and minimum
+    red = max_over_ranks([total_ms, ev_total_ms] + [sum(t) for t in per_kernel]
+                         + [statistics.median(t) for t in per_kernel] + [min(t) for t in per_kernel], world, device)
     nk = len(names)
-    max_ms, kernel_sum, kernel_med, kernel_min = red[0], red[1:1 + nk], red[1 + nk:1 + 2 * nk], red[1 + 2 * nk:]
+    max_ms, ev_max_ms = red[0], red[1]
+    kernel_sum, kernel_med, kernel_min = red[2:2 + nk], red[2 + nk:2 + 2 * nk], red[2 + 2 * nk:]
 
     # the copy floor of every slot: the same sequence with each kernel
     # replaced by fk_copy of its bytes, so each copy follows the same
     # predecessor traffic as the kernel it stands for
     for k in range(max(1, args.warmup, min(len(copy_seqs), 64))):
         step(copy_seqs[k % len(copy_seqs)])
-    copy_total, copy_per = timed_steps(copy_seqs, args.steps)
+    copy_total, _ = timed_steps(copy_seqs, args.steps, per_kernel=False)
+    _, copy_per = timed_steps(copy_seqs, args.steps)
     red = max_over_ranks([copy_total] + [statistics.median(t) for t in copy_per], world, device)
     copy_total, copy_med = red[0], red[1:]
 
     # each workload alone, L2 cleaned before every launch
-    alone = {}
+    alone, event_floor = {}, None
     if alone_names:
         cleaner = L2Cleaner(device, torch.cuda.get_device_properties(device).L2_cache_size)
         reps = max(5, min(args.alone_reps, 200))
+        # two events around nothing, after the same clean: the floor of an event-timed interval
+        event_floor = max_over_ranks([statistics.fmean(time_alone(lambda: None, stream, device, reps, cleaner))],
+                                     world, device)[0]
         for n in alone_names:
             def checked(c=call_of[n], n=n):
                 st = c()
@@ -684,7 +696,12 @@ def run_ours(args) -> dict | None:
         "copy_floor_step": {"ms_per_step": round(copy_total / args.steps, 5),
                             "GB_s": round(aggregate_value(bytes_step, args.steps, world, copy_total), 1),
                             "what": "the same sequence with every kernel replaced by fk_copy of its bytes"},
+        "per_kernel_timing": {"how": "a second pass of the same K steps with a CUDA event between every two "
+                                     "kernels (the timed region above has events only at its ends)",
+                              "ms_per_step_with_events": round(ev_max_ms / args.steps, 5),
+                              "event_cost_us": round(1e3 * (ev_max_ms - max_ms) / (args.steps * len(names)), 3)},
         "alone": {"l2": "L2 written back and evicted (read-only pass over 4x L2) before every launch",
+                  "event_floor_ms": round(event_floor, 5) if event_floor is not None else None,
                   "timer": "CUDA events tick in steps of about 2 us on this GPU: for launches of tens of us "
                            "the mean over the launches resolves finer than the median",
                   "reps": max(5, min(args.alone_reps, 200)) if alone_names else 0, "workloads": alone_rows},

@@ -111,14 +111,22 @@ size_t reg_blocks(size_t nvec) {
 // in registers and stores them with 16-byte streaming stores (a warp's store
 // covers 512 contiguous bytes); after a block barrier the stage is refilled
 // with the block's chunk kStages further on.
-constexpr int kBulkThreads = 128;
 constexpr uint32_t kChunkBytes = 16384;
 constexpr int kStages = 3;
 constexpr int kBulkBlocksPerSm = 4;
 constexpr uint32_t kChunkVecs = kChunkBytes / 16;
 constexpr size_t kStageSmem = static_cast<size_t>(kStages) * kChunkBytes;
-static_assert(kChunkVecs % kBulkThreads == 0, "whole vectors per thread in a chunk");
 constexpr uint64_t kBulkWaitNs = 1000000000ull;  // 1 s
+// Threads per pipeline block, measured on B200 (32 MiB, mean of 60 launches,
+// L2 cleaned / left dirty before each): fp32 streams best with 128 (tanh
+// 12.3 / 14.3 us, exact 14.4 / 15.1); bf16, with twice the arithmetic per
+// byte, with 256 (tanh 18.5 / 19.8 us against 18.5 / 20.4 with 128; exact
+// 22.6 / 23.0 against 23.3 / 24.5).  512 was slower in every case.
+constexpr int kCopyBulkThreads = 128;
+template <typename T, int KIND>
+struct GeluBulkThreads {
+  static constexpr int value = sizeof(T) == 2 ? 256 : 128;
+};
 
 __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -141,9 +149,10 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // y = op(x) over `bytes` bytes (a multiple of 16) from 16-byte aligned x and
-// y, chunk by chunk as described above.
-template <typename Op>
+// y, chunk by chunk as described above, by blocks of THREADS threads.
+template <int THREADS, typename Op>
 __device__ __forceinline__ void stream_bulk(const char* x, char* y, size_t bytes, Op op) {
+  static_assert(kChunkVecs % THREADS == 0, "whole vectors per thread in a chunk");
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ int abort_flag;
@@ -182,8 +191,8 @@ __device__ __forceinline__ void stream_bulk(const char* x, char* y, size_t bytes
     const uint4* sv = reinterpret_cast<const uint4*>(stage_mem + s * kChunkBytes);
     uint4* yv = reinterpret_cast<uint4*>(y + c * kChunkBytes);
 #pragma unroll
-    for (int j = 0; j < static_cast<int>(kChunkVecs / kBulkThreads); ++j) {
-      const uint32_t vi = static_cast<uint32_t>(j * kBulkThreads + t);
+    for (int j = 0; j < static_cast<int>(kChunkVecs / THREADS); ++j) {
+      const uint32_t vi = static_cast<uint32_t>(j * THREADS + t);
       if (vi < nv) st_stream_v4(yv + vi, op.vec(sv[vi]));
     }
     __syncthreads();  // every thread is done with stage s, and abort_flag is settled
@@ -197,11 +206,11 @@ __device__ __forceinline__ void stream_bulk(const char* x, char* y, size_t bytes
   }
 }
 
-size_t bulk_blocks(size_t bytes, size_t scalar, int sm_count) {
+size_t bulk_blocks(size_t bytes, size_t scalar, int threads, int sm_count) {
   const size_t nchunks = (bytes + kChunkBytes - 1) / kChunkBytes;
   size_t blocks = static_cast<size_t>(sm_count > 0 ? sm_count : 1) * kBulkBlocksPerSm;
   if (blocks > nchunks) blocks = nchunks;
-  const size_t scalar_blocks = (scalar + kBulkThreads - 1) / kBulkThreads;
+  const size_t scalar_blocks = (scalar + threads - 1) / threads;
   if (blocks < scalar_blocks) blocks = scalar_blocks;
   if (blocks > kMaxGrid) blocks = kMaxGrid;
   return blocks < 1 ? 1 : blocks;
@@ -221,19 +230,19 @@ bool use_bulk(size_t bytes, size_t l2_bytes) { return bytes > 0 && 2 * bytes <= 
 
 // x, y: the arrays.  Elements [0, head) and [tail_begin, n) are done with
 // scalar accesses; [head, tail_begin) is nvec 16-byte vectors starting at a
-// 16-byte boundary of both x and y.  BULK: through shared memory (above).
-template <typename T, int KIND, bool BULK>
-__global__ void __launch_bounds__(BULK ? kBulkThreads : kRegThreads)
+// 16-byte boundary of both x and y.  BULK: through shared memory (above),
+// by blocks of THREADS threads; otherwise through registers (kRegThreads).
+template <typename T, int KIND, bool BULK, int THREADS>
+__global__ void __launch_bounds__(THREADS)
     gelu_kernel(const T* x, T* y, size_t head, size_t nvec, size_t tail_begin, size_t n) {
-  constexpr int THREADS = BULK ? kBulkThreads : kRegThreads;
   const size_t tid = static_cast<size_t>(blockIdx.x) * THREADS + threadIdx.x;
   const size_t nthr = static_cast<size_t>(gridDim.x) * THREADS;
   for (size_t i = tid; i < head; i += nthr) Elem<T>::store1(y + i, gelu_f<T, KIND>(Elem<T>::load1(x + i)));
   for (size_t i = tail_begin + tid; i < n; i += nthr)
     Elem<T>::store1(y + i, gelu_f<T, KIND>(Elem<T>::load1(x + i)));
   if constexpr (BULK) {
-    stream_bulk(reinterpret_cast<const char*>(x + head), reinterpret_cast<char*>(y + head), nvec * 16,
-                GeluOp<T, KIND>{});
+    stream_bulk<THREADS>(reinterpret_cast<const char*>(x + head), reinterpret_cast<char*>(y + head), nvec * 16,
+                         GeluOp<T, KIND>{});
   } else {
     stream_regs(reinterpret_cast<const char*>(x + head), reinterpret_cast<char*>(y + head), nvec,
                 GeluOp<T, KIND>{});
@@ -243,9 +252,11 @@ __global__ void __launch_bounds__(BULK ? kBulkThreads : kRegThreads)
 // A plain copy through the same two paths: the achievable-bandwidth
 // reference the fused kernels are measured against (fk_copy).
 template <bool BULK>
-__global__ void __launch_bounds__(BULK ? kBulkThreads : kRegThreads) copy_kernel(const uint4* src, uint4* dst, size_t nvec) {
+__global__ void __launch_bounds__(BULK ? kCopyBulkThreads : kRegThreads)
+    copy_kernel(const uint4* src, uint4* dst, size_t nvec) {
   if constexpr (BULK) {
-    stream_bulk(reinterpret_cast<const char*>(src), reinterpret_cast<char*>(dst), nvec * 16, CopyOp{});
+    stream_bulk<kCopyBulkThreads>(reinterpret_cast<const char*>(src), reinterpret_cast<char*>(dst), nvec * 16,
+                                  CopyOp{});
   } else {
     stream_regs(reinterpret_cast<const char*>(src), reinterpret_cast<char*>(dst), nvec, CopyOp{});
   }
@@ -266,17 +277,18 @@ cudaError_t launch_gelu_typed(const void* xp, void* yp, size_t n, const DeviceIn
   const size_t tail_begin = head + nvec * VEC;
   const size_t scalar = head > (n - tail_begin) ? head : (n - tail_begin);
   if (use_bulk(nvec * 16, dev.l2_bytes)) {
-    const cudaError_t e = allow_stage_smem(gelu_kernel<T, KIND, true>);
+    constexpr int TB = GeluBulkThreads<T, KIND>::value;
+    const cudaError_t e = allow_stage_smem(gelu_kernel<T, KIND, true, TB>);
     if (e != cudaSuccess) return e;
-    gelu_kernel<T, KIND, true><<<static_cast<unsigned>(bulk_blocks(nvec * 16, scalar, dev.sm_count)), kBulkThreads,
-                                 kStageSmem, stream>>>(x, y, head, nvec, tail_begin, n);
+    gelu_kernel<T, KIND, true, TB><<<static_cast<unsigned>(bulk_blocks(nvec * 16, scalar, TB, dev.sm_count)), TB,
+                                     kStageSmem, stream>>>(x, y, head, nvec, tail_begin, n);
   } else {
     size_t blocks = reg_blocks(nvec);
     const size_t scalar_blocks = (scalar + kRegThreads - 1) / kRegThreads;
     if (blocks < scalar_blocks) blocks = scalar_blocks;
     if (blocks < 1) blocks = 1;
-    gelu_kernel<T, KIND, false><<<static_cast<unsigned>(blocks), kRegThreads, 0, stream>>>(x, y, head, nvec,
-                                                                                           tail_begin, n);
+    gelu_kernel<T, KIND, false, kRegThreads><<<static_cast<unsigned>(blocks), kRegThreads, 0, stream>>>(
+        x, y, head, nvec, tail_begin, n);
   }
   return cudaGetLastError();
 }
@@ -301,8 +313,8 @@ cudaError_t launch_copy(const void* src, void* dst, size_t bytes, const DeviceIn
   if (use_bulk(bytes, dev.l2_bytes)) {
     const cudaError_t e = allow_stage_smem(copy_kernel<true>);
     if (e != cudaSuccess) return e;
-    copy_kernel<true><<<static_cast<unsigned>(bulk_blocks(bytes, 0, dev.sm_count)), kBulkThreads, kStageSmem,
-                        stream>>>(s, d, nvec);
+    copy_kernel<true><<<static_cast<unsigned>(bulk_blocks(bytes, 0, kCopyBulkThreads, dev.sm_count)),
+                        kCopyBulkThreads, kStageSmem, stream>>>(s, d, nvec);
   } else {
     copy_kernel<false><<<static_cast<unsigned>(reg_blocks(nvec)), kRegThreads, 0, stream>>>(s, d, nvec);
   }
