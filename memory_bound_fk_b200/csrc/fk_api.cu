@@ -55,6 +55,20 @@ cudaMemPool_t workspace_pool(int dev) {
   return g_pool[dev];
 }
 
+}  // namespace
+
+// Stream-ordered workspace from the private pool of the current device (the
+// default pool if the private one could not be made).
+cudaError_t workspace_alloc(void** p, size_t bytes, cudaStream_t s) {
+  int d = -1;
+  const cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return e;
+  const cudaMemPool_t pool = (d >= 0 && d < kMaxDevices) ? workspace_pool(d) : nullptr;
+  return pool ? cudaMallocFromPoolAsync(p, bytes, pool, s) : cudaMallocAsync(p, bytes, s);
+}
+
+namespace {
+
 fk_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return FK_ERR_CUDA;

@@ -205,15 +205,35 @@ __device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_co
 // 2 G - 1 - blockIdx.x, then 2 G + blockIdx.x, ... (G blocks): a serpentine
 // that balances the decreasing causal unit lengths across blocks, and lets
 // a block start its next unit's loads while the current one finishes.
+//
+// Equal units (the non-causal grid) leave the last round part-empty: 512
+// units on 148 blocks make 3.46 rounds, and the blocks with a fourth unit set
+// the time.  When the last round's units are at most half the blocks, each
+// of them is split into two halves of its key blocks, run by two blocks;
+// the online recurrence of section 7.2 merges the halves exactly (the same
+// rule that merges key blocks), see merge_halves.
+struct AttnWork {
+  int u;     // the unit; -1: no more work for this block
+  int half;  // -1: the whole unit; 0 / 1: the first / second half of its key blocks
+};
+
 struct AttnUnits {
-  int t, bh;  // keys (and queries) per slice, slices
+  int t, bh;       // keys (and queries) per slice, slices
+  int nfull;       // units handed out whole; the rest (nsplit) are split in halves
+  int nsplit;
   bool causal;
   __device__ __forceinline__ int nq() const { return t / 128; }
   __device__ __forceinline__ int npair() const { return (nq() + 1) / 2; }
-  __device__ __forceinline__ int unit(int round) const {  // -1: no more units for this block
+  __device__ __forceinline__ AttnWork work(int round) const {
     const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-    const int u = round * g + ((round & 1) ? g - 1 - b : b);
-    return u < bh * npair() ? u : -1;
+    const int w = (round & 1) ? g - 1 - b : b;
+    const int base = round * g;
+    if (nsplit > 0 && base >= nfull) {  // the last round: half units
+      if (base > nfull || w >= 2 * nsplit) return AttnWork{-1, -1};
+      return AttnWork{nfull + w / 2, w & 1};
+    }
+    const int u = base + w;
+    return AttnWork{u < bh * npair() ? u : -1, -1};
   }
   __device__ __forceinline__ int slice(int u) const { return causal ? u % bh : u / npair(); }
   __device__ __forceinline__ int pair(int u) const { return causal ? npair() - 1 - u / bh : u % npair(); }
@@ -223,13 +243,39 @@ struct AttnUnits {
     const int qb = 2 * pair(u) + i;
     return qb < nq() ? (causal ? qb + 1 : nq()) : 0;
   }
+  // first key block and key blocks of query tile i for a piece of work
+  // (halves are made only of non-causal units, whose tiles see every key)
+  __device__ __forceinline__ int key0(const AttnWork& wk) const { return wk.half == 1 ? nq() / 2 : 0; }
+  __device__ __forceinline__ int nkv(const AttnWork& wk, int i) const {
+    const int n = nkv(wk.u, i);
+    if (wk.half < 0 || n == 0) return n;
+    return wk.half == 0 ? nq() / 2 : nq() - nq() / 2;
+  }
 };
+
+// Scratch of the split units (global memory): per split unit, half and
+// query tile, every row's unnormalised O (fp32) and its (reference max m,
+// sum l), and per split unit and tile a counter of the halves that finished.
+struct AttnSplitScratch {
+  float* o;        // [nsplit][2 halves][2 tiles][128 rows][D]
+  float2* ml;      // [nsplit][2 halves][2 tiles][128 rows]
+  unsigned* done;  // [nsplit][2 tiles], zero at launch
+};
+
+// Named barrier 1 + i for the 128 threads of softmax warpgroup i (barrier 0
+// is the block-wide one).
+__device__ __forceinline__ void warpgroup_bar(int i) {
+  if (i == 0)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  else
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+}
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out, int t, int bh,
-                         float scale_log2) {
+                         int nfull, int nsplit, AttnSplitScratch split, float scale_log2) {
   constexpr int KC = D / 64;                     // 64-column chunks of a head row
   constexpr uint32_t TILE = KC * kChunkBytes;    // bytes of a 128 x D tile
   constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(128, 128, false);
@@ -240,6 +286,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bar_o[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int split_flag[2];  // per softmax warpgroup: decisions taken once for its 128 threads
 
   // Q0 | Q1 | K0 | K1 | V0 | V1, every tile 1024-byte aligned (addressed by
   // offset: arrays of pointers indexed at run time would live in local memory)
@@ -249,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto sV = [&](int b) { return base + (4 + b) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const AttnUnits units{t, bh, CAUSAL};
+  const AttnUnits units{t, bh, nfull, nsplit, CAUSAL};
   volatile int* abort = &abort_flag;
 
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
@@ -289,12 +336,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int nql = 0;                // Q loads issued
       bool ok = true;
       for (int round = 0; ok; ++round) {
-        const int u = units.unit(round);
-        if (u < 0) break;
-        const int nkv0 = units.nkv(u, 0), nkv1 = units.nkv(u, 1);
+        const AttnWork wk = units.work(round);
+        if (wk.u < 0) break;
+        const int nkv0 = units.nkv(wk, 0), nkv1 = units.nkv(wk, 1);
         const int nmax = nkv0 > nkv1 ? nkv0 : nkv1, ntiles = nkv1 > 0 ? 2 : 1;
-        const int row0 = units.slice(u) * t;  // first row of the slice in the [bh * t, D] view
-        const int pair = units.pair(u);
+        const int row0 = units.slice(wk.u) * t;  // first row of the slice in the [bh * t, D] view
+        const int krow0 = row0 + units.key0(wk) * kAttnBlock;
+        const int pair = units.pair(wk.u);
         if (round > 0 && !attn_wait(&bar_qfree, (round - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bar_q, ntiles * TILE);
         for (int i = 0; i < ntiles; ++i) {
@@ -312,7 +360,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_arrive_expect_tx(&bar_k[b], TILE);
 #pragma unroll
           for (int c = 0; c < KC; ++c)
-            tc::tma_load_2d(sK(b) + c * kChunkBytes, &tmk, &bar_k[b], c * 64, row0 + j * 128);
+            tc::tma_load_2d(sK(b) + c * kChunkBytes, &tmk, &bar_k[b], c * 64, krow0 + j * 128);
           nk = g + 1;
           if (g >= 2 && !attn_wait(&bar_vfree[b], ((g - 2) >> 1) & 1, abort)) {
             ok = false;
@@ -321,7 +369,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_arrive_expect_tx(&bar_v[b], TILE);
 #pragma unroll
           for (int c = 0; c < KC; ++c)
-            tc::tma_load_2d(sV(b) + c * kChunkBytes, &tmv, &bar_v[b], c * 64, row0 + j * 128);
+            tc::tma_load_2d(sV(b) + c * kChunkBytes, &tmv, &bar_v[b], c * 64, krow0 + j * 128);
           nv = g + 1;
         }
       }
@@ -357,9 +405,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int g0 = 0;          // tile counter of the unit's first K/V tile
       bool ok = true;
       for (int round = 0; ok; ++round) {
-        const int u = units.unit(round);
-        if (u < 0) break;
-        const int nkv0 = units.nkv(u, 0), nkv1 = units.nkv(u, 1);
+        const AttnWork wk = units.work(round);
+        if (wk.u < 0) break;
+        const int nkv0 = units.nkv(wk, 0), nkv1 = units.nkv(wk, 1);
         const int nmax = nkv0 > nkv1 ? nkv0 : nkv1, ntiles = nkv1 > 0 ? 2 : 1;
         int s_left = nkv0 + nkv1;  // S products of the unit still to issue
         auto last = [&](int j) { return j < nkv1 ? 1 : 0; };  // the tile that reads K_j and V_j last
@@ -431,10 +479,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tS = tmem + lane + i * 256, tO = tS + 128;
     int ns = 0, no = 0;  // S and O phases waited for (across units)
     for (int round = 0;; ++round) {
-      const int u = units.unit(round);
-      if (u < 0) break;
-      const int qb = 2 * units.pair(u) + i;
-      const int nkv_i = units.nkv(u, i);
+      const AttnWork wk = units.work(round);
+      if (wk.u < 0) break;
+      const int qb = 2 * units.pair(wk.u) + i;
+      const int nkv_i = units.nkv(wk, i);
       float m_i = -INFINITY, l_i = 0.0f;
       for (int j = 0; j < nkv_i; ++j, ++ns) {
         attn_wait(&bar_s[i], ns & 1, abort);
@@ -447,15 +495,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc::fence_before_sync();
         mbar_arrive(&bar_p[i]);
       }
-      if (nkv_i > 0) {
-        attn_wait(&bar_o[i], no & 1, abort);
-        ++no;
+      if (nkv_i == 0) continue;
+      attn_wait(&bar_o[i], no & 1, abort);
+      ++no;
+      // row r of the tile in the output
+      uint4* dst =
+          reinterpret_cast<uint4*>(out + (static_cast<size_t>(units.slice(wk.u)) * t + qb * kAttnBlock + r) * D);
+      if (wk.half < 0) {
         if (!__any_sync(0xffffffffu, *abort)) {
           tc::fence_after_sync();
-          // O / l, rounded to bf16: row r of the tile
+          // O / l, rounded to bf16
           const float inv = 1.0f / l_i;
-          uint4* dst =
-              reinterpret_cast<uint4*>(out + (static_cast<size_t>(units.slice(u)) * t + qb * kAttnBlock + r) * D);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float v[32];
@@ -467,12 +517,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                           pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
                                           pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
           }
-          // the next unit's first O product overwrites O: its tcgen05.ld
-          // reads have completed (tmem_ld32 waits for them) before this
-          // warpgroup's next arrival on P
-          tc::fence_before_sync();
+        }
+      } else {
+        // Half of a split unit.  Both halves store their rows' unnormalised
+        // O and (m, l); the half that finishes second (by an atomic count
+        // per unit and tile, taken after a fence) merges the other's with
+        // its own and writes the output.  Nothing waits on the other block.
+        // The warpgroup's 128 threads take each decision together (its named
+        // barrier), so that all of them pass the same barriers.
+        warpgroup_bar(i);
+        if (r == 0) split_flag[i] = *abort;
+        warpgroup_bar(i);
+        if (!split_flag[i]) {
+          const int su = wk.u - nfull;
+          const size_t mine = (static_cast<size_t>(su * 2 + wk.half) * 2 + i) * kAttnBlock + r;
+          const size_t other = (static_cast<size_t>(su * 2 + (1 - wk.half)) * 2 + i) * kAttnBlock + r;
+          tc::fence_after_sync();
+          float4* po = reinterpret_cast<float4*>(split.o + mine * D);
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tc::tmem_ld32(tO + c * 32, v);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) po[c * 8 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+          split.ml[mine] = make_float2(m_i, l_i);
+          __threadfence();
+          warpgroup_bar(i);
+          if (r == 0) split_flag[i] = static_cast<int>(atomicAdd(&split.done[su * 2 + i], 1u));
+          warpgroup_bar(i);
+          if (split_flag[i] == 1) {
+            __threadfence();
+            // the other half's (m, l) and O, read through L2 (written by another SM)
+            const float2 mlo = __ldcg(split.ml + other);
+            const float M = fmaxf(m_i, mlo.x);
+            const float fa = (m_i == M) ? 1.0f : ex2_ftz(m_i - M);
+            const float fb = (mlo.x == M) ? 1.0f : ex2_ftz(mlo.x - M);
+            const float inv = 1.0f / fmaf(l_i, fa, mlo.y * fb);
+            const float4* oo = reinterpret_cast<const float4*>(split.o + other * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              float v[32];
+              tc::tmem_ld32(tO + c * 32, v);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 w = __ldcg(oo + c * 8 + q);
+                v[4 * q] = fmaf(v[4 * q], fa, w.x * fb) * inv;
+                v[4 * q + 1] = fmaf(v[4 * q + 1], fa, w.y * fb) * inv;
+                v[4 * q + 2] = fmaf(v[4 * q + 2], fa, w.z * fb) * inv;
+                v[4 * q + 3] = fmaf(v[4 * q + 3], fa, w.w * fb) * inv;
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[c * 4 + q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            }
+          }
         }
       }
+      // the next unit's first O product overwrites O: this warpgroup's
+      // tcgen05.ld reads of it have completed (tmem_ld32 waits for them)
+      // before its next arrival on P
+      tc::fence_before_sync();
     }
   }
   tc::fence_before_sync();
@@ -513,6 +620,24 @@ bool make_map(CUtensorMap* m, const void* ptr, size_t rows, int d) {
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// How the units go to the persistent blocks: G blocks, the first nfull
+// units whole, the remaining nsplit units (the last, part-empty round of a
+// non-causal grid, when it fills at most half the blocks) in key halves.
+struct AttnGrid {
+  int blocks, nfull, nsplit;
+};
+
+AttnGrid attn_grid(size_t bh, size_t t, bool causal, int sm_count) {
+  const size_t nq = t / kAttnBlock;
+  const size_t nunits = bh * ((nq + 1) / 2);
+  const size_t sms = static_cast<size_t>(sm_count);
+  const size_t rounds = (nunits + sms - 1) / sms;
+  const size_t last = nunits - (rounds - 1) * sms;
+  if (!causal && nq >= 2 && 2 * last <= sms)
+    return AttnGrid{sm_count, static_cast<int>(nunits - last), static_cast<int>(last)};
+  return AttnGrid{static_cast<int>(nunits < sms ? nunits : sms), static_cast<int>(nunits), 0};
+}
+
 template <int D, bool CAUSAL>
 cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, size_t bh,
                         size_t t, float scale_log2, int sm_count, cudaStream_t s) {
@@ -530,12 +655,35 @@ cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (e != cudaSuccess) return e;
   // persistent blocks, one per SM (the kernel holds all of an SM's tensor
   // memory), each walking its units
-  const size_t nunits = bh * ((t / kAttnBlock + 1) / 2);
-  const size_t grid = nunits < static_cast<size_t>(sm_count) ? nunits : static_cast<size_t>(sm_count);
-  kernel<<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
-                                                                 static_cast<int>(t), static_cast<int>(bh),
-                                                                 scale_log2);
-  return cudaGetLastError();
+  const AttnGrid g = attn_grid(bh, t, CAUSAL, sm_count);
+  AttnSplitScratch split = {nullptr, nullptr, nullptr};
+  void* ws = nullptr;
+  if (g.nsplit > 0) {
+    // scratch for the split units, stream-ordered from the library's pool
+    const size_t rows = static_cast<size_t>(g.nsplit) * 2 * 2 * kAttnBlock;
+    const size_t o_bytes = rows * D * sizeof(float), ml_bytes = rows * sizeof(float2);
+    const size_t done_bytes = static_cast<size_t>(g.nsplit) * 2 * sizeof(unsigned);
+    e = workspace_alloc(&ws, o_bytes + ml_bytes + done_bytes, s);
+    if (e != cudaSuccess) return e;
+    char* base = static_cast<char*>(ws);
+    split.o = reinterpret_cast<float*>(base);
+    split.ml = reinterpret_cast<float2*>(base + o_bytes);
+    split.done = reinterpret_cast<unsigned*>(base + o_bytes + ml_bytes);
+    e = cudaMemsetAsync(split.done, 0, done_bytes, s);
+    if (e != cudaSuccess) {
+      (void)cudaFreeAsync(ws, s);
+      return e;
+    }
+  }
+  kernel<<<static_cast<unsigned>(g.blocks), kAttnThreads, smem, s>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(t), static_cast<int>(bh), g.nfull, g.nsplit, split,
+      scale_log2);
+  e = cudaGetLastError();
+  if (ws != nullptr) {
+    const cudaError_t f = cudaFreeAsync(ws, s);
+    if (e == cudaSuccess) e = f;
+  }
+  return e;
 }
 
 }  // namespace

@@ -121,6 +121,11 @@ cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const f
 // Workspace bytes a validated plan needs (0 except on the split path).
 size_t workspace_bytes(size_t rows, size_t cols, int dtype, const fk_softmax_plan& plan);
 
+// Stream-ordered device workspace of `bytes` from the library's private pool
+// on the current device (kept reserved across calls); release it with
+// cudaFreeAsync on the same stream after the kernels that use it.
+cudaError_t workspace_alloc(void** p, size_t bytes, cudaStream_t s);
+
 // ---- attention ------------------------------------------------------------
 // O = softmax(scale Q K^T, causal) V over bh slices of [t, d] bf16 rows
 // (validated: t % 128 == 0, d in {64, 128}, 16-byte aligned, bh * t < 2^31).

@@ -69,6 +69,20 @@ def test_parity(fk, torch_mod, bh, t, d, causal):
     assert fk.fk_wait_timeouts(reset=True) == 0
 
 
+@pytest.mark.parametrize("bh,t,d", [(40, 1024, 64), (230, 256, 64), (75, 384, 128), (148, 256, 64)])
+def test_persistent_grids(fk, torch_mod, bh, t, d):
+    """Non-causal grids of several rounds over the persistent blocks (one per
+    SM): a last round of 12 units split into key halves (40 x 1024), a last
+    round of 82 units too many to split (230 x 256), a single round of 150
+    units of which 2 spill into a split second round, odd query-tile counts
+    (75 x 384: the last pair of each slice has one tile), and a grid that
+    fills its rounds exactly (148 x 256).  Every slice against the oracle."""
+    q, k, v = inputs(bh, t, d, seed=bh * 7 + t)
+    scale = 1.0 / math.sqrt(d)
+    check(run(fk, torch_mod, q, k, v, False, scale), q, k, v, False, scale)
+    assert fk.fk_wait_timeouts(reset=True) == 0
+
+
 @pytest.mark.parametrize("sigma,scale", [(3.0, 0.125), (1.0, 1.0), (0.2, 0.05)])
 def test_score_ranges(fk, torch_mod, sigma, scale):
     """Peaked and flat attention: large scores (the running max moves often)
