@@ -874,7 +874,7 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
     """Same step through the C ABI from pinned host buffers: every step copies
     all inputs host->device and all outputs device->host inside the timed
     region.  Work is split into row chunks (about --e2e-chunk-mb of input
-    each) issued round-robin on two streams, so the host->device copy of one
+    each) issued round-robin on --e2e-streams streams, so the host->device copy of one
     chunk, the kernel of another and the device->host copy of a third
     overlap (the two copy directions use separate copy engines)."""
     import torch
@@ -904,13 +904,13 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
             per = max(1, per // a.shape[1]) * a.shape[1]  # whole query blocks per chunk
         for r0 in range(0, a.shape[0], per):
             chunks.append((n, r0, min(per, a.shape[0] - r0)))
-    streams = [stream, torch.cuda.Stream(device)]
+    streams = [stream] + [torch.cuda.Stream(device) for _ in range(max(1, args.e2e_streams) - 1)]
     raw_in = {n: (dev_in[n].view(torch.int16) if dev_in[n].dtype == torch.bfloat16 else dev_in[n]) for n in names}
     raw_out = {n: (dev_out[n].view(torch.int16) if dev_out[n].dtype == torch.bfloat16 else dev_out[n]) for n in names}
 
     def step():
         for i, (n, r0, cnt) in enumerate(chunks):
-            s = streams[i & 1]
+            s = streams[i % len(streams)]
             w = synth.WORKLOADS[n]
             with torch.cuda.stream(s):
                 raw_in[n][r0:r0 + cnt].copy_(pin_in[n][r0:r0 + cnt], non_blocking=True)
@@ -930,10 +930,12 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    streams[1].wait_stream(stream)
+    for s2 in streams[1:]:
+        s2.wait_stream(stream)
     for _ in range(steps):
         step()
-    stream.wait_stream(streams[1])
+    for s2 in streams[1:]:
+        stream.wait_stream(s2)
     b.record(stream)
     torch.cuda.synchronize(device)
     ms = max_over_ranks([a.elapsed_time(b)], world, device)[0]
@@ -942,7 +944,7 @@ def run_e2e(args, names, host, dev_in, dev_out, stream, device, world, bytes_ste
     assert torch.equal(pin_out[n0][r0:r0 + cnt], raw_out[n0][r0:r0 + cnt].cpu())
     return {"value": round(aggregate_value(bytes_step, steps, world, ms), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3), "chunks_per_step": len(chunks), "streams": 2}
+            "ms_per_step": round(ms / steps, 3), "chunks_per_step": len(chunks), "streams": len(streams)}
 
 
 # ---------------------------------------------------------------- unfused comparison
@@ -1106,6 +1108,7 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--e2e-chunk-mb", type=int, default=64,
                    help="input bytes per pipelined host<->device chunk in the e2e leg")
+    p.add_argument("--e2e-streams", type=int, default=2, help="streams the e2e leg's chunks rotate over")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-alone", action="store_true", help="skip the per-workload L2-clean leg")
     p.add_argument("--alone-reps", type=int, default=30, help="launches per workload in the L2-clean leg")
