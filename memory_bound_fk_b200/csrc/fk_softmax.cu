@@ -349,8 +349,16 @@ __global__ void __launch_bounds__(THREADS, (EPT * sizeof(T) <= 32 && THREADS <= 
 
 // A cluster of csize blocks per row; block `rank` holds vectors
 // [rank*per, (rank+1)*per) of the row in registers, per = ceil(nvec / csize).
+// With 64 values a thread the plain aligned kernel's register budget is held
+// to six 128-thread blocks an SM (three of 256): more clusters resident, so
+// that others stream while one waits at its exchange (80 vs 95 registers, no
+// spills; 512 x 131072 fp32 runs 80 instead of 86 us).  The scaled and the
+// unaligned forms would spill under that bound and keep the default.
+template <int THREADS, int EPT, bool PLAIN>
+constexpr int cluster_min_blocks() { return PLAIN && EPT == 64 && THREADS <= 256 ? 768 / THREADS : 1; }
+
 template <typename T, int THREADS, int EPT, bool ALIGNED, bool SC>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, cluster_min_blocks<THREADS, EPT, ALIGNED && !SC>())
     softmax_cluster_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = EPT / VEC;
