@@ -29,8 +29,8 @@ __device__ __forceinline__ float ex2_ftz(float v) {
   return r;
 }
 
-// 1/v with MUFU.RCP, at most 1 ulp off; v must be a normal number >= 1
-// (true for every softmax normaliser here).
+// 1/v with MUFU.RCP, at most 1 ulp off; results below 2^-126 flush to
+// zero and 1/inf is 0 (every softmax normaliser here is >= 1).
 __device__ __forceinline__ float rcp_approx(float v) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));

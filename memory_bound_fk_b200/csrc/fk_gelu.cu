@@ -15,16 +15,16 @@
 // The crossover is where input plus output stop fitting in L2 (the two tie
 // at 64 MiB, 128 MiB in all).
 //
-// tanh form (the notes, section 4.2).  With u = sqrt(2/pi) (x + 0.044715 x^3)
-// and t = exp(-2|u|) <= 1 (never overflows),
-//     0.5 x (1 + tanh u) = x * sigma(2u) = x / (1 + t)      for x >= 0,
-//                                        = x * t / (1 + t)  for x < 0
-// (sigma the logistic function; 1 + tanh u = 2 sigma(2u)).  One MUFU.EX2 for
-// t = 2^(-2|u| log2 e) and one MUFU.RCP for 1 / (1 + t); an IEEE division
-// here cost ~20 instructions per element and made the kernel issue-bound.
-// For large |x|, t underflows and y is x or the tiny x * t (kept as a
-// subnormal for bf16 outputs, whose smallest value is 2^-133); x = -inf is
-// mapped to the limit -0.
+// tanh form (the notes, section 4.2).  With u = sqrt(2/pi) (x + 0.044715 x^3),
+//     0.5 x (1 + tanh u) = x * sigma(2u) = x / (1 + exp(-2u))
+// (sigma the logistic function; 1 + tanh u = 2 sigma(2u)): one MUFU.EX2 for
+// exp(-2u) = 2^(-2u log2 e) and one MUFU.RCP for the quotient, with no
+// cancellation for either sign (for x < 0 the quotient is the small tail
+// itself); an IEEE division here cost ~20 instructions per element and made
+// the kernel issue-bound.  For large |x| the exponential overflows or
+// flushes and y is -0 or x; tails of bf16 outputs are kept down to their
+// smallest subnormal, 2^-133, by an exponent offset of 64 (fk_gelu.cuh);
+// inputs below -30, -inf among them, give -0, the correctly rounded value.
 //
 // Exact form: x Phi(x), Phi the standard normal distribution function, with
 // erfc in the form of Press et al. and coefficients fitted here (see

@@ -15,13 +15,53 @@ constexpr float kA = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.442695
 constexpr float kB = static_cast<float>(-2.0 * 0.79788456080286535588 * 1.44269504088896340736 * 0.044715);
 constexpr float kRsqrt2 = 0.70710678118654752440f;
 
+// Inputs below kGeluFloor are raised to it first, by a NaN-propagating max
+// (one instruction): both forms give -0 from there down, the correctly
+// rounded value (|GELU(x)| < 1e-49 for x <= -15, below every fp32 and bf16
+// subnormal), and x = -inf no longer meets inf * 0 on the way.
+constexpr float kGeluFloor = -30.0f;
+
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Exponent offset of the GELU tails.  bf16 outputs keep values down to
+// 2^-133, so their tail terms are taken 2^64 too large, where the
+// flush-to-zero MUFU units (one instruction each; the forms that keep
+// subnormal results take several) cannot flush them, and are scaled back by
+// 2^-64 in one rounding before the last product.  Folding the offset into
+// an exponent rounds it to 2^-18 absolute, a relative error under 2e-6 of
+// the exponential: far below a bf16 ulp.  fp32 outputs take the terms
+// flushed below 2^-126 (an absolute error under 1.2e-38 after the product).
+template <typename T>
+struct GeluScale {
+  static constexpr float kBias = 0.0f;
+  static constexpr float kUnbias = 1.0f;
+};
+template <>
+struct GeluScale<__nv_bfloat16> {
+  static constexpr float kBias = 64.0f;
+  static constexpr float kUnbias = 0x1p-64f;
+};
+
+// tanh form: 0.5 x (1 + tanh u) = x sigma(2u) = x / (1 + 2^a) with
+// a = -2u log2(e) (< 0 for x > 0).  For x < 0 the quotient is the small
+// tail itself, without cancellation; where 2^a overflows it is 0 and y is
+// -0, where 2^a flushes y is x.  One MUFU.EX2 and one MUFU.RCP.  With the
+// offset the sum is 2^-64 + 2^(a-64), whose reciprocal 2^64 / (1 + 2^a)
+// stays normal where 1 / (1 + 2^a) is subnormal (the flush-to-zero MUFU.RCP
+// would drop it); 2^-64 is applied to that reciprocal, not to x q, which
+// would overflow for x > 2^64.
 template <typename T>
 __device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float a = x * fmaf(kB, x * x, kA);  // -2u log2(e): <= 0 for x >= 0
-  const float t = Elem<T>::exp2(-fabsf(a)); // exp(-2|u|) in (0, 1]
-  const float r = rcp_approx(1.0f + t);
-  const float y = (a > 0.0f) ? x * t * r : x * r;
-  return (x == -INFINITY) ? -0.0f : y;
+  using S = GeluScale<T>;
+  x = max_nan(x, kGeluFloor);
+  const float p = fmaf(kB, x * x, kA);
+  const float e = ex2_ftz(S::kBias != 0.0f ? fmaf(x, p, -S::kBias) : x * p);  // 2^(a - bias)
+  const float q = rcp_approx(e + S::kUnbias) * S::kUnbias;                    // 1 / (1 + 2^a)
+  return x * q;
 }
 
 // Exact form, x Phi(x).  h = P(Z > |x|) = 0.5 erfc(w), w = |x| / sqrt 2,
@@ -54,12 +94,14 @@ __device__ __forceinline__ V erfc_poly(V t) {
 
 template <typename T>
 __device__ __forceinline__ float gelu_erf_f(float x) {
+  using S = GeluScale<T>;
+  x = max_nan(x, kGeluFloor);
   const float w = fabsf(x) * kRsqrt2;
   const float t = rcp_approx(fmaf(0.5f, w, 1.0f));
   const float p = erfc_poly(t);
-  const float h = 0.5f * t * Elem<T>::exp2(fmaf(-w, w, p) * kLog2e);
-  const float y = x * ((x >= 0.0f) ? 1.0f - h : h);
-  return (x == -INFINITY) ? -0.0f : y;
+  const float hb = ex2_ftz(fmaf(fmaf(-w, w, p), kLog2e, S::kBias));  // 2^bias erfc(w) / t
+  const float h = (0.5f * t * hb) * S::kUnbias;
+  return x * ((x >= 0.0f) ? 1.0f - h : h);
 }
 
 // The two forms on a pair of values: every lane takes the operations of the
@@ -68,31 +110,29 @@ __device__ __forceinline__ float gelu_erf_f(float x) {
 // with about half the arithmetic instructions.
 template <typename T>
 __device__ __forceinline__ float2 gelu_tanh_f2(float2 x) {
-  const float2 a = mul2(x, fma2(splat2(kB), mul2(x, x), splat2(kA)));
-  const float2 t = make_float2(Elem<T>::exp2(-fabsf(a.x)), Elem<T>::exp2(-fabsf(a.y)));
-  const float2 s = add2(splat2(1.0f), t);
-  const float2 r = make_float2(rcp_approx(s.x), rcp_approx(s.y));
-  const float2 yp = mul2(mul2(x, t), r);  // x t r, for a > 0
-  const float2 yn = mul2(x, r);
-  float2 y = make_float2(a.x > 0.0f ? yp.x : yn.x, a.y > 0.0f ? yp.y : yn.y);
-  y.x = (x.x == -INFINITY) ? -0.0f : y.x;
-  y.y = (x.y == -INFINITY) ? -0.0f : y.y;
-  return y;
+  using S = GeluScale<T>;
+  x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
+  const float2 p = fma2(splat2(kB), mul2(x, x), splat2(kA));
+  const float2 a = S::kBias != 0.0f ? fma2(x, p, splat2(-S::kBias)) : mul2(x, p);
+  const float2 s = add2(make_float2(ex2_ftz(a.x), ex2_ftz(a.y)), splat2(S::kUnbias));
+  float2 q = make_float2(rcp_approx(s.x), rcp_approx(s.y));
+  if constexpr (S::kBias != 0.0f) q = mul2(q, splat2(S::kUnbias));
+  return mul2(x, q);
 }
 
 template <typename T>
 __device__ __forceinline__ float2 gelu_erf_f2(float2 x) {
+  using S = GeluScale<T>;
+  x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
   const float2 w = mul2(make_float2(fabsf(x.x), fabsf(x.y)), splat2(kRsqrt2));
   const float2 q = fma2(splat2(0.5f), w, splat2(1.0f));
   const float2 t = make_float2(rcp_approx(q.x), rcp_approx(q.y));
   const float2 p = erfc_poly(t);
-  const float2 e = mul2(fma2(make_float2(-w.x, -w.y), w, p), splat2(kLog2e));
-  const float2 h = mul2(mul2(splat2(0.5f), t), make_float2(Elem<T>::exp2(e.x), Elem<T>::exp2(e.y)));
+  const float2 e = fma2(fma2(make_float2(-w.x, -w.y), w, p), splat2(kLog2e), splat2(S::kBias));
+  float2 h = mul2(mul2(splat2(0.5f), t), make_float2(ex2_ftz(e.x), ex2_ftz(e.y)));
+  if constexpr (S::kBias != 0.0f) h = mul2(h, splat2(S::kUnbias));
   const float2 om = add2(splat2(1.0f), make_float2(-h.x, -h.y));  // 1 - h
-  float2 y = mul2(x, make_float2(x.x >= 0.0f ? om.x : h.x, x.y >= 0.0f ? om.y : h.y));
-  y.x = (x.x == -INFINITY) ? -0.0f : y.x;
-  y.y = (x.y == -INFINITY) ? -0.0f : y.y;
-  return y;
+  return mul2(x, make_float2(x.x >= 0.0f ? om.x : h.x, x.y >= 0.0f ? om.y : h.y));
 }
 
 template <typename T, int KIND>

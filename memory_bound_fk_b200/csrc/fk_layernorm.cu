@@ -19,7 +19,8 @@
 //           d = a / cols corrects m1 (mean = m1 + d) and
 //           var = b / cols - d^2 (d is only m1's rounding error, so nothing
 //           cancels);
-//   output: y_j = ((x_j - m1) - d) * rsqrt(var + eps), affine, GELU.
+//   output: y_j = (x_j - m1) rstd - d rstd, rstd = rsqrt(var + eps) (one
+//           FMA; d rstd, a tiny term, is rounded once per row), affine, GELU.
 // x_j - m1 is exact to a rounding relative to itself, so the error of y does
 // not grow with |mean| / std the way a single fp32 mean's rounding would
 // make it.
@@ -155,22 +156,23 @@ __device__ __forceinline__ float2 epilogue2(float2 z) {
   }
 }
 
-// y = ((x - m1) - d) * rstd * gamma + beta, then the epilogue, stored chunk
-// by chunk (only one chunk's gamma / beta are live at a time).
+// y = ((x - m1) rstd - d rstd) * gamma + beta, then the epilogue, stored
+// chunk by chunk (only one chunk's gamma / beta are live at a time).
 template <typename T, int VPT, int TEAM, bool ALIGNED, int EPI, typename Idx>
 __device__ __forceinline__ void normalise_store(T* yr, const uint4* raw, float m1, float d, float rstd,
                                                 const float* gamma, const float* beta, Idx vfirst, Idx ve,
                                                 Idx cols, int t) {
   constexpr int VEC = Elem<T>::VEC;
+  const float ndr = -d * rstd;
   store_chunks_fn<T, VPT, TEAM, ALIGNED, Idx>(yr, vfirst, ve, cols, t, [&](int c, float* o) {
     float g[VEC], b[VEC];
     load_affine<T, TEAM, ALIGNED, Idx>(gamma, 1.0f, vfirst, c, cols, t, g);
     load_affine<T, TEAM, ALIGNED, Idx>(beta, 0.0f, vfirst, c, cols, t, b);
-    // pairs of columns, each lane as ((x - m1) - d) * rstd * gamma + beta
+    // pairs of columns, each lane as ((x - m1) rstd - d rstd) * gamma + beta
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) {
       float2 z = add2(make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1)), splat2(-m1));
-      z = mul2(add2(z, splat2(-d)), splat2(rstd));
+      z = fma2(z, splat2(rstd), splat2(ndr));
       z = epilogue2<EPI>(fma2(z, make_float2(g[k], g[k + 1]), make_float2(b[k], b[k + 1])));
       o[k] = z.x;
       o[k + 1] = z.y;
