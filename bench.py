@@ -784,6 +784,12 @@ def run_attention(args) -> dict | None:
     max_ms = max_over_ranks([a.elapsed_time(b)], world, device)[0]
     tflops = flops * args.steps * world / (max_ms * 1e-3) / 1e12
 
+    # context: torch's fused attention on the same q, k, v and stream, timed
+    # the same way right after (rank 0 of a single-GPU run only)
+    library = None
+    if rank == 0 and world == 1 and not args.no_library:
+        library = library_attention(qkv, o, bh, t, d, causal, scale, flops, args.steps, args.warmup, stream, gpu_id)
+
     # end to end: q, k, v from pinned host memory in, o back out, every step
     e2e = None
     if not args.no_e2e:
@@ -841,7 +847,47 @@ def run_attention(args) -> dict | None:
                      "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": 4 * bh * t * d * 2},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+        "library_context": library,
     }
+
+
+def library_attention(qkv, o, bh, t, d, causal, scale, flops, steps, warmup, stream, gpu_id) -> dict:
+    """torch.nn.functional.scaled_dot_product_attention on the same inputs,
+    once per backend that runs on this GPU: W warm-ups, then K calls between
+    two CUDA events on the same stream, with the SM clocks sampled meanwhile.
+    A reference point for the kernel's speed, not part of this library."""
+    import torch
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    q4, k4, v4 = (qkv[i].view(1, bh, t, d) for i in range(3))
+    ours = o.view(1, bh, t, d).float()
+    out = {"what": "torch.nn.functional.scaled_dot_product_attention, same q, k, v, scale and mask, timed right "
+                   "after the kernel (context only)", "torch": torch.__version__, "backends": {}}
+    for be in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION):
+        try:
+            with sdpa_kernel(be):
+                def call():
+                    return torch.nn.functional.scaled_dot_product_attention(q4, k4, v4, is_causal=causal,
+                                                                            scale=scale)
+                ref = call()
+                for _ in range(warmup):
+                    call()
+                torch.cuda.synchronize()
+                sampler = ClockSampler(gpu_id)
+                time.sleep(0.25)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(steps):
+                    call()
+                b.record(stream)
+                torch.cuda.synchronize()
+                clocks = sampler.stop()
+                ms = a.elapsed_time(b) / steps
+                out["backends"][be.name] = {"TFLOP_s": round(flops / ms / 1e9, 1), "ms": round(ms, 5),
+                                            "max_abs_diff_vs_this_kernel": float((ref.float() - ours).abs().max()),
+                                            "clocks": clocks}
+        except RuntimeError as e:
+            out["backends"][be.name] = {"unavailable": str(e).splitlines()[0][:160]}
+    return out
 
 
 def copy_reference(fk, src, dst, stream, device, world, reps: int = 7) -> dict | None:
@@ -1111,6 +1157,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-streams", type=int, default=2, help="streams the e2e leg's chunks rotate over")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-alone", action="store_true", help="skip the per-workload L2-clean leg")
+    p.add_argument("--no-library", action="store_true",
+                   help="attention workloads: skip timing torch's scaled_dot_product_attention beside the kernel")
     p.add_argument("--alone-reps", type=int, default=30, help="launches per workload in the L2-clean leg")
     p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     p.add_argument("--reference-budget", type=float, default=120.0,
