@@ -101,6 +101,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// max(a, b, c) in one instruction (sm_100); a NaN operand is ignored, as by
+// fmaxf.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Two fp32 lanes per instruction (sm_100 packed arithmetic), each rounded as
 // the scalar operation would be.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
@@ -140,13 +148,15 @@ __device__ __forceinline__ void softmax_block(uint32_t tS, uint32_t tO, int d_co
 #pragma unroll
     for (int i = 0; i < 128; ++i) sr[i] = (i > r) ? 0xff800000u : sr[i];
   }
+  // eight running maxima, two values folded in per three-input max
   float mx8[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+  for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
 #pragma unroll
-  for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i]));
-  const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+  for (int i = 16; i < 128; i += 16)  // values i .. i + 15 (the last group ends at 127)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx8[k] = max3(mx8[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + 8 + k]));
+  const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) *
                    scale_log2;
   const bool upd = mx > m_i + kLazyRescale;  // always for the first block (m_i = -inf)
   const float m_new = upd ? mx : m_i;

@@ -55,11 +55,16 @@ template <typename T, int KIND>
 struct GeluOp {
   __device__ __forceinline__ uint4 vec(uint4 v) const {
     constexpr int VEC = Elem<T>::VEC;
+    constexpr bool BF16 = sizeof(T) == 2;
+    if constexpr (BF16) {  // clamped while packed
+      v = make_uint4(max_nan_floor_bf16x2(v.x), max_nan_floor_bf16x2(v.y), max_nan_floor_bf16x2(v.z),
+                     max_nan_floor_bf16x2(v.w));
+    }
     float f[VEC];
     Elem<T>::unpack(v, f);
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) {
-      const float2 g = gelu_f2<T, KIND>(make_float2(f[k], f[k + 1]));
+      const float2 g = gelu_f2<T, KIND, BF16>(make_float2(f[k], f[k + 1]));
       f[k] = g.x;
       f[k + 1] = g.y;
     }

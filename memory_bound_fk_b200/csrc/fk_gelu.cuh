@@ -27,6 +27,13 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return r;
 }
 
+// The same on a packed bf16 pair (-30 is exact in bf16: 0xc1f0).
+__device__ __forceinline__ uint32_t max_nan_floor_bf16x2(uint32_t w) {
+  uint32_t r;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xc1f0c1f0u));
+  return r;
+}
+
 // Exponent offset of the GELU tails.  bf16 outputs keep values down to
 // 2^-133, so their tail terms are taken 2^64 too large, where the
 // flush-to-zero MUFU units (one instruction each; the forms that keep
@@ -75,7 +82,8 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 // nine FMAs and one MUFU.EX2, against ~45 instructions for erfcf; P - w^2
 // is a single FMA, so w^2 is not rounded on its own.  Errors: under 4e-7
 // absolute on [-20, 20] for fp32, and a relative error of h below 2e-5
-// where h is tiny (the fp32 rounding of the exponent, up to ~100).
+// where h is tiny (the fp32 rounding of the exponent, up to ~100).  bf16
+// outputs use a degree-7 fit (below).
 // The fitted P(t), by Horner's rule, for one value or a pair.
 template <typename V>
 __device__ __forceinline__ V erfc_poly(V t) {
@@ -92,26 +100,60 @@ __device__ __forceinline__ V erfc_poly(V t) {
   return p;
 }
 
+// The degree-7 fit (fit_erfc.py 7: largest error 2.9e-6, a relative error of
+// erfc) for bf16 outputs, whose half ulp is 2^-9: two FMAs fewer.
+template <typename V>
+__device__ __forceinline__ V erfc_poly7(V t) {
+  V p = splat_v<V>(-1.661221087e-01f);
+  p = fma_v(p, t, 6.685151458e-01f);
+  p = fma_v(p, t, -8.729041219e-01f);
+  p = fma_v(p, t, 2.482906431e-01f);
+  p = fma_v(p, t, 4.035713617e-03f);
+  p = fma_v(p, t, 3.840898573e-01f);
+  p = fma_v(p, t, 9.996045828e-01f);
+  p = fma_v(p, t, -1.265509248e+00f);
+  return p;
+}
+
+template <typename T, typename V>
+__device__ __forceinline__ V erfc_poly_for(V t) {
+  if constexpr (sizeof(T) == 2)
+    return erfc_poly7(t);
+  else
+    return erfc_poly(t);
+}
+
+// Phi(x) from the tail h: 1 - h for x >= 0, h for x < 0, as
+// fma(s, h, (1 - s) / 2) with s = -1 or +1 taken from the sign bit of x
+// (one logic instruction; -0 counts as negative, which gives the same -0
+// output).  1 - h is rounded once, h is exact: the values of the select.
+__device__ __forceinline__ float phi_sign(float x) {
+  return __uint_as_float((__float_as_uint(x) & 0x80000000u) ^ 0xbf800000u);
+}
+
 template <typename T>
 __device__ __forceinline__ float gelu_erf_f(float x) {
   using S = GeluScale<T>;
   x = max_nan(x, kGeluFloor);
   const float w = fabsf(x) * kRsqrt2;
   const float t = rcp_approx(fmaf(0.5f, w, 1.0f));
-  const float p = erfc_poly(t);
+  const float p = erfc_poly_for<T>(t);
   const float hb = ex2_ftz(fmaf(fmaf(-w, w, p), kLog2e, S::kBias));  // 2^bias erfc(w) / t
   const float h = (0.5f * t * hb) * S::kUnbias;
-  return x * ((x >= 0.0f) ? 1.0f - h : h);
+  const float sg = phi_sign(x);
+  return x * fmaf(sg, h, fmaf(sg, -0.5f, 0.5f));
 }
 
 // The two forms on a pair of values: every lane takes the operations of the
 // scalar functions above in the same order (packed fp32 arithmetic rounds
 // each lane as the scalar instruction does), so the results are identical,
 // with about half the arithmetic instructions.
-template <typename T>
+// CLAMPED: the caller has already raised x to kGeluFloor (bf16 inputs are
+// clamped while still packed, one instruction per pair).
+template <typename T, bool CLAMPED = false>
 __device__ __forceinline__ float2 gelu_tanh_f2(float2 x) {
   using S = GeluScale<T>;
-  x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
+  if (!CLAMPED) x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
   const float2 p = fma2(splat2(kB), mul2(x, x), splat2(kA));
   const float2 a = S::kBias != 0.0f ? fma2(x, p, splat2(-S::kBias)) : mul2(x, p);
   const float2 s = add2(make_float2(ex2_ftz(a.x), ex2_ftz(a.y)), splat2(S::kUnbias));
@@ -120,24 +162,24 @@ __device__ __forceinline__ float2 gelu_tanh_f2(float2 x) {
   return mul2(x, q);
 }
 
-template <typename T>
+template <typename T, bool CLAMPED = false>
 __device__ __forceinline__ float2 gelu_erf_f2(float2 x) {
   using S = GeluScale<T>;
-  x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
+  if (!CLAMPED) x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
   const float2 w = mul2(make_float2(fabsf(x.x), fabsf(x.y)), splat2(kRsqrt2));
   const float2 q = fma2(splat2(0.5f), w, splat2(1.0f));
   const float2 t = make_float2(rcp_approx(q.x), rcp_approx(q.y));
-  const float2 p = erfc_poly(t);
+  const float2 p = erfc_poly_for<T>(t);
   const float2 e = fma2(fma2(make_float2(-w.x, -w.y), w, p), splat2(kLog2e), splat2(S::kBias));
   float2 h = mul2(mul2(splat2(0.5f), t), make_float2(ex2_ftz(e.x), ex2_ftz(e.y)));
   if constexpr (S::kBias != 0.0f) h = mul2(h, splat2(S::kUnbias));
-  const float2 om = add2(splat2(1.0f), make_float2(-h.x, -h.y));  // 1 - h
-  return mul2(x, make_float2(x.x >= 0.0f ? om.x : h.x, x.y >= 0.0f ? om.y : h.y));
+  const float2 sg = make_float2(phi_sign(x.x), phi_sign(x.y));
+  return mul2(x, fma2(sg, h, fma2(sg, splat2(-0.5f), splat2(0.5f))));
 }
 
-template <typename T, int KIND>
+template <typename T, int KIND, bool CLAMPED = false>
 __device__ __forceinline__ float2 gelu_f2(float2 x) {
-  return KIND == FK_GELU_TANH ? gelu_tanh_f2<T>(x) : gelu_erf_f2<T>(x);
+  return KIND == FK_GELU_TANH ? gelu_tanh_f2<T, CLAMPED>(x) : gelu_erf_f2<T, CLAMPED>(x);
 }
 
 template <typename T, int KIND>

@@ -99,6 +99,26 @@ __device__ __forceinline__ float val(const uint4& w, int k) {
   }
 }
 
+// (x_k + c, x_k+1 + c) for the pair of values k, k + 1 (k even) of a packed
+// word, each rounded once to fp32.  bf16: two sm_100 mixed-precision adds
+// (add.f32.bf16 takes the bf16 half of the word as it is), one instruction
+// per value where widening first took two per pair more.  The results are
+// those of widening (exact) and adding.
+template <typename T>
+__device__ __forceinline__ float2 add_pair(const uint4& w, int k, float2 c) {
+  if constexpr (sizeof(T) == 4) {
+    return add2(make_float2(val<T>(w, k), val<T>(w, k + 1)), c);
+  } else {
+    const uint32_t u = k < 2 ? w.x : k < 4 ? w.y : k < 6 ? w.z : w.w;
+    float2 d;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %3;\n\tadd.rn.f32.bf16 %1, hi, %4;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "r"(u), "f"(c.x), "f"(c.y));
+    return d;
+  }
+}
+
 // 16-byte read-only load that stays in program order with the row's
 // (volatile) stores, so the compiler fetches each chunk's parameters just
 // before that chunk is stored instead of hoisting every chunk's parameters
@@ -171,7 +191,7 @@ __device__ __forceinline__ void normalise_store(T* yr, const uint4* raw, float m
     // pairs of columns, each lane as ((x - m1) rstd - d rstd) * gamma + beta
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) {
-      float2 z = add2(make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1)), splat2(-m1));
+      float2 z = add_pair<T>(raw[c], k, splat2(-m1));
       z = fma2(z, splat2(rstd), splat2(ndr));
       z = epilogue2<EPI>(fma2(z, make_float2(g[k], g[k + 1]), make_float2(b[k], b[k + 1])));
       o[k] = z.x;
@@ -190,18 +210,18 @@ __device__ __forceinline__ float sum_raw(const uint4* raw) {
   for (int c = 0; c < VPT; ++c)
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) {
-      const float2 v = make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1));
       if (k & 2)
-        s23 = add2(s23, v);
+        s23 = add_pair<T>(raw[c], k, s23);
       else
-        s01 = add2(s01, v);
+        s01 = add_pair<T>(raw[c], k, s01);
     }
   return (s01.x + s01.y) + (s23.x + s23.y);
 }
 
 // Pass-2 partial sums of one thread: sum (x - m1) and sum (x - m1)^2 over
-// its columns of the row (padding excluded).
-template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx>
+// its columns of the row (padding excluded).  FULL: every value the thread
+// holds is a column of the row (no padding to mask).
+template <typename T, int VPT, int TEAM, bool ALIGNED, typename Idx, bool FULL = false>
 __device__ __forceinline__ float2 centred_sums(const uint4* raw, float m1, Idx vfirst, Idx cols, int t) {
   constexpr int VEC = Elem<T>::VEC;
   // two accumulators each (even and odd columns), one packed pair
@@ -210,9 +230,11 @@ __device__ __forceinline__ float2 centred_sums(const uint4* raw, float m1, Idx v
   for (int c = 0; c < VPT; ++c) {
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) {
-      float2 z = add2(make_float2(val<T>(raw[c], k), val<T>(raw[c], k + 1)), splat2(-m1));
-      z.x = in_row<T, TEAM, ALIGNED>(vfirst, c, k, t, cols) ? z.x : 0.0f;
-      z.y = in_row<T, TEAM, ALIGNED>(vfirst, c, k + 1, t, cols) ? z.y : 0.0f;
+      float2 z = add_pair<T>(raw[c], k, splat2(-m1));
+      if (!FULL) {
+        z.x = in_row<T, TEAM, ALIGNED>(vfirst, c, k, t, cols) ? z.x : 0.0f;
+        z.y = in_row<T, TEAM, ALIGNED>(vfirst, c, k + 1, t, cols) ? z.y : 0.0f;
+      }
       a = add2(a, z);
       b = fma2(z, z, b);
     }
@@ -275,7 +297,11 @@ __global__ void __launch_bounds__(THREADS)
     for (int w = 1; w < NW; ++w) s += red1[w];
     const float m1 = s * inv_n;
 
-    float2 ab = centred_sums<T, VPT, THREADS, ALIGNED, int>(raw, m1, 0, cols, t);
+    // bf16 rows that fill every thread's vectors exactly need no padding
+    // masks (issue-bound rows; fp32 rows keep one code path)
+    float2 ab = (sizeof(T) == 2 && ALIGNED && nvec == VPT * THREADS)
+                    ? centred_sums<T, VPT, THREADS, ALIGNED, int, true>(raw, m1, 0, cols, t)
+                    : centred_sums<T, VPT, THREADS, ALIGNED, int>(raw, m1, 0, cols, t);
     ab.x = warp_sum(ab.x);
     ab.y = warp_sum(ab.y);
     if (lane == 0) red2[warp] = ab;
