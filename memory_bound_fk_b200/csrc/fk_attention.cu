@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bar_vfree[i], 1);
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_o[i], 1);
-      mbar_init(&bar_p[i], kAttnTileThreads);
+      mbar_init(&bar_p[i], kAttnTileThreads / 32);  // one arrival per softmax warp
     }
     mbar_init(&bar_drain, 1);
     abort_flag = 0;
@@ -502,8 +502,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           else
             softmax_block<false>(tS, tO, D, r, j, scale_log2, m_i, l_i);
         }
+        // each thread's P stores are complete (tcgen05.wait::st); one lane
+        // per warp arrives once the warp has synchronised
         tc::fence_before_sync();
-        mbar_arrive(&bar_p[i]);
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(&bar_p[i]);
       }
       if (nkv_i == 0) continue;
       attn_wait(&bar_o[i], no & 1, abort);
