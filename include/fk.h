@@ -259,6 +259,19 @@ FK_API fk_status fk_softmax_rows_noalloc(const void *x, void *y, size_t rows, si
                                          void *stream);
 
 /*
+ * fk_softmax_rows_noalloc_cap -- fk_softmax_rows_noalloc using only the
+ * first capacity_pairs (max, sum) pairs of the library's array (1 ..
+ * 131072), so that the batching can be exercised on inputs of a few GB: rows
+ * run in batches of floor(capacity_pairs / chunks) rows.  A capacity that
+ * cannot hold one row's chunks, or the chunks of the full batch or of the
+ * shorter last batch as each is planned, returns FK_ERR_INVALID_ARG before
+ * anything is enqueued; capacity_pairs outside 1 .. 131072 likewise.
+ * Otherwise as fk_softmax_rows_noalloc (same array, same ordering rules).
+ */
+FK_API fk_status fk_softmax_rows_noalloc_cap(const void *x, void *y, size_t rows, size_t cols, int dtype,
+                                             size_t capacity_pairs, void *stream);
+
+/*
  * fk_softmax_rows_causal -- scaled, causally masked row softmax: the score
  * step of causal attention (lecture 6, "GPU Kernels and Triton", section 8:
  * scores times 1/sqrt(d_k), -inf where the key position is after the query

@@ -276,6 +276,18 @@ def fk_softmax_rows_noalloc(x: int, y: int, rows: int, cols: int, dtype: int, st
     return f(x, y, rows, cols, dtype, stream)
 
 
+def fk_softmax_rows_noalloc_cap(x: int, y: int, rows: int, cols: int, dtype: int, capacity_pairs: int,
+                                stream: int = 0) -> int:
+    """fk_softmax_rows_noalloc on the first capacity_pairs entries of the
+    library's scratch array (more batches on smaller inputs)."""
+    f = lib().fk_softmax_rows_noalloc_cap
+    if f.argtypes is None:
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        f.argtypes = [vp, vp, sz, sz, ctypes.c_int, sz, vp]
+        f.restype = ctypes.c_int
+    return f(x, y, rows, cols, dtype, capacity_pairs, stream)
+
+
 def make_plan(path: int, threads: int = 0, vpt: int = 0, cluster: int = 0, chunks: int = 0) -> SoftmaxPlan:
     return SoftmaxPlan(path, threads, vpt, cluster, chunks)
 
@@ -463,7 +475,7 @@ __all__ = [
     "FK_ERR_CUDA", "FK_F32", "FK_BF16", "FK_GELU_TANH", "FK_GELU_ERF", "FK_PATH_AUTO", "FK_PATH_WARP", "FK_PATH_CTA",
     "FK_PATH_CLUSTER", "FK_PATH_TWOPHASE", "FK_PATH_SPLIT", "FkError", "SoftmaxPlan", "lib", "header_functions",
     "fk_gelu_tanh", "fk_gelu", "fk_copy", "fk_softmax_rows", "fk_softmax_rows_ex", "fk_softmax_rows_plan",
-    "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc",
+    "fk_softmax_rows_workspace", "fk_softmax_rows_ws", "fk_softmax_rows_noalloc", "fk_softmax_rows_noalloc_cap",
     "fk_softmax_rows_causal", "fk_softmax_rows_causal_ex", "softmax_causal", "FK_SOFTMAX_SKIP_MASKED",
     "fk_layernorm_rows", "fk_layernorm_rows_ex", "fk_layernorm_rows_plan", "layernorm",
     "fk_attention_fwd", "attention", "FK_EPILOGUE_NONE", "FK_EPILOGUE_GELU_TANH",

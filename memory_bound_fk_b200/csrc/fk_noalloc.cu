@@ -57,48 +57,73 @@ void* scratch_address(int dev, cudaError_t* err) {
 }  // namespace
 }  // namespace fk
 
-extern "C" fk_status fk_softmax_rows_noalloc(const void* x, void* y, size_t rows, size_t cols, int dtype,
-                                             void* stream) {
+namespace fk {
+namespace {
+
+// The allocation-free call with a scratch of `capacity` (max, sum) pairs
+// (at most the array's).  Rows run in batches of floor(capacity / chunks)
+// rows, chunks as planned for all rows; each batch plans its own chunking
+// for its row count, so the two batch sizes that occur (the full batch and
+// the shorter last one) are checked against the capacity before anything
+// is enqueued.
+fk_status noalloc_batched(const void* x, void* y, size_t rows, size_t cols, int dtype, size_t capacity,
+                          void* stream) {
   if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED_DTYPE;
   if (rows == 0 || cols == 0) return FK_OK;
   if (rows > SIZE_MAX / cols) return FK_ERR_INVALID_ARG;
   fk_softmax_plan plan;
-  fk_status st = fk::plan_softmax(rows, cols, dtype, FK_PATH_AUTO, &plan);
+  fk_status st = plan_softmax(rows, cols, dtype, FK_PATH_AUTO, &plan);
   if (st != FK_OK) return st;
   if (plan.path != FK_PATH_SPLIT) {
     // every other path keeps its state on chip: nothing to allocate
     return fk_softmax_rows_ws(x, y, rows, cols, dtype, &plan, nullptr, 0, stream);
   }
-  // The split path in batches of rows whose partials fit the scratch array;
-  // a single row with more chunks than the array holds (more than 2^35
-  // elements) is refused.  The whole of x and y is checked before the first
-  // batch is enqueued, so a rejected call writes nothing.
-  const fk::SplitGeometry g = fk::split_geometry(rows, cols, dtype);
-  if (g.nchunks > fk::kNoAllocPartials) return FK_ERR_INVALID_ARG;
+  // A single row with more chunks than the scratch holds (for the whole
+  // array: more than 2^35 elements) is refused.  The whole of x and y is
+  // checked before the first batch is enqueued, so a rejected call writes
+  // nothing.
+  const SplitGeometry g = split_geometry(rows, cols, dtype);
+  if (g.nchunks > capacity) return FK_ERR_INVALID_ARG;
+  const size_t rows_per_batch = capacity / g.nchunks;
+  const size_t last = rows % rows_per_batch;
+  const size_t cap_bytes = capacity * sizeof(float2);
+  if (split_geometry(rows < rows_per_batch ? rows : rows_per_batch, cols, dtype).ws_bytes > cap_bytes ||
+      (last != 0 && split_geometry(last, cols, dtype).ws_bytes > cap_bytes))
+    return FK_ERR_INVALID_ARG;
   const size_t esize = dtype == FK_F32 ? 4 : 2;
-  st = fk::validate_call(x, y, rows * cols, esize);
+  st = validate_call(x, y, rows * cols, esize);
   if (st != FK_OK) return st;
-  const size_t rows_per_batch = fk::kNoAllocPartials / g.nchunks;
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= fk::kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     (void)cudaGetLastError();
     return FK_ERR_UNSUPPORTED_DEVICE;
   }
   cudaError_t err = cudaSuccess;
-  void* scratch = fk::scratch_address(dev, &err);
+  void* scratch = scratch_address(dev, &err);
   if (scratch == nullptr) return FK_ERR_CUDA;
   const char* xb = static_cast<const char*>(x);
   char* yb = static_cast<char*>(y);
   for (size_t r0 = 0; r0 < rows; r0 += rows_per_batch) {
     const size_t n = (rows - r0 < rows_per_batch) ? rows - r0 : rows_per_batch;
-    // each batch plans its own chunking for its rows; its partials fit the
-    // array (n * chunks(n) <= 131072 for every n up to rows_per_batch)
     fk_softmax_plan p = plan;
     p.chunks = 0;
     const size_t off = r0 * cols * esize;
-    st = fk_softmax_rows_ws(xb + off, yb + off, n, cols, dtype, &p, scratch, fk::kNoAllocPartials * sizeof(float2),
-                            stream);
+    st = fk_softmax_rows_ws(xb + off, yb + off, n, cols, dtype, &p, scratch, cap_bytes, stream);
     if (st != FK_OK) return st;
   }
   return FK_OK;
+}
+
+}  // namespace
+}  // namespace fk
+
+extern "C" fk_status fk_softmax_rows_noalloc(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                                             void* stream) {
+  return fk::noalloc_batched(x, y, rows, cols, dtype, fk::kNoAllocPartials, stream);
+}
+
+extern "C" fk_status fk_softmax_rows_noalloc_cap(const void* x, void* y, size_t rows, size_t cols, int dtype,
+                                                 size_t capacity_pairs, void* stream) {
+  if (capacity_pairs == 0 || capacity_pairs > fk::kNoAllocPartials) return FK_ERR_INVALID_ARG;
+  return fk::noalloc_batched(x, y, rows, cols, dtype, capacity_pairs, stream);
 }

@@ -80,3 +80,39 @@ def test_noalloc_on_the_other_paths_and_arguments(fk, cuda_device):
     assert torch.equal(y, fk.softmax_rows(x))
     assert _noalloc(fk, 0, 0, 0, 4096, fk.FK_F32, s) == fk.FK_OK
     assert _noalloc(fk, x.data_ptr(), y.data_ptr(), 64, 4096, 7, s) == fk.FK_ERR_UNSUPPORTED_DTYPE
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_noalloc_batches_rows_when_the_scratch_is_small(fk, cuda_device, dtype):
+    """With 1200 of the array's pairs, 80 split-path rows of 2^22 columns run
+    as a batch of 75 rows (16 chunks each) and a last batch of 5 (171 chunks
+    each, planned for 5 rows): every row against the oracle, the rows at the
+    batch boundary among them.  A capacity that cannot hold a batch is
+    refused before anything is written."""
+    import torch
+    code = fk.FK_F32 if dtype == "f32" else fk.FK_BF16
+    rows, cols, cap = 80, 1 << 22, 1200
+    assert fk.fk_softmax_rows_plan(rows, cols, code).as_dict()["path"] == "split"
+    s = torch.cuda.current_stream().cuda_stream
+    host = synth.softmax_input(rows, cols, dtype, sigma=3.0, neg_inf_frac=0.01, seed=44)
+    if dtype == "f32":
+        x = torch.from_numpy(host).cuda()
+    else:
+        x = torch.from_numpy(host.view(np.int16)).cuda()
+    y = torch.full_like(x, 7)
+    assert fk.fk_softmax_rows_noalloc_cap(x.data_ptr(), y.data_ptr(), rows, cols, code, 100, s) == \
+        fk.FK_ERR_INVALID_ARG
+    assert fk.fk_softmax_rows_noalloc_cap(x.data_ptr(), y.data_ptr(), rows, cols, code, 0, s) == \
+        fk.FK_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert bool((y == 7).all()), "a refused call wrote output"
+    assert fk.fk_softmax_rows_noalloc_cap(x.data_ptr(), y.data_ptr(), rows, cols, code, cap, s) == fk.FK_OK
+    torch.cuda.synchronize()
+    got = y.cpu().numpy()
+    for r in (0, 1, 37, 74, 75, 76, 79):
+        if dtype == "f32":
+            ref = oracle.softmax_rows_f32(host[r:r + 1])[0]
+            assert np.max(np.abs(got[r].astype(np.float64) - ref)) <= 1e-6, r
+        else:
+            ref = oracle.softmax_rows_bf16(host[r:r + 1])[0]
+            assert np.max(np.abs(_ordinal(got[r].view(np.uint16)) - _ordinal(ref))) <= 1, r
