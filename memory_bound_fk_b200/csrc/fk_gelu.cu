@@ -57,8 +57,8 @@ struct GeluOp {
     constexpr int VEC = Elem<T>::VEC;
     constexpr bool BF16 = sizeof(T) == 2;
     if constexpr (BF16) {  // clamped while packed
-      v = make_uint4(max_nan_floor_bf16x2(v.x), max_nan_floor_bf16x2(v.y), max_nan_floor_bf16x2(v.z),
-                     max_nan_floor_bf16x2(v.w));
+      v = make_uint4(max_nan_floor_bf16x2<KIND>(v.x), max_nan_floor_bf16x2<KIND>(v.y),
+                     max_nan_floor_bf16x2<KIND>(v.z), max_nan_floor_bf16x2<KIND>(v.w));
     }
     float f[VEC];
     Elem<T>::unpack(v, f);

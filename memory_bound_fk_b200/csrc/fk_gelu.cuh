@@ -27,11 +27,36 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return r;
 }
 
-// The same on a packed bf16 pair (-30 is exact in bf16: 0xc1f0).
+// The same on a packed bf16 pair, to the floor of the form used for bf16
+// outputs (both exact in bf16: -30 = 0xc1f0, -11 = 0xc130).
+template <int KIND>
 __device__ __forceinline__ uint32_t max_nan_floor_bf16x2(uint32_t w) {
+  constexpr uint32_t kFloorPair = KIND == FK_GELU_TANH ? 0xc130c130u : 0xc1f0c1f0u;
   uint32_t r;
-  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xc1f0c1f0u));
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(kFloorPair));
   return r;
+}
+
+// 1/s on the FMA pipes, for s in [2^-125, 2^125]: an estimate from the bits,
+// K - bits(s) with K = 0x7ef311c0 (the constant of smallest largest relative
+// error over a scan of the mantissa, 5.1%), then two Newton steps
+// r <- r + r (1 - s r), each squaring the relative error: under 1e-5, far
+// below a bf16 half ulp (2^-9).  Four FMAs and an integer subtraction in
+// place of one MUFU.RCP, for kernels that MUFU limits.
+constexpr uint32_t kRecipMagic = 0x7ef311c0u;
+
+__device__ __forceinline__ float recip_newton(float s) {
+  float r = __uint_as_float(kRecipMagic - __float_as_uint(s));
+  r = fmaf(r, fmaf(-s, r, 1.0f), r);
+  return fmaf(r, fmaf(-s, r, 1.0f), r);
+}
+
+__device__ __forceinline__ float2 recip_newton2(float2 s) {
+  const float2 ns = make_float2(-s.x, -s.y);
+  float2 r = make_float2(__uint_as_float(kRecipMagic - __float_as_uint(s.x)),
+                         __uint_as_float(kRecipMagic - __float_as_uint(s.y)));
+  r = fma2(r, fma2(ns, r, splat2(1.0f)), r);
+  return fma2(r, fma2(ns, r, splat2(1.0f)), r);
 }
 
 // Exponent offset of the GELU tails.  bf16 outputs keep values down to
@@ -42,15 +67,25 @@ __device__ __forceinline__ uint32_t max_nan_floor_bf16x2(uint32_t w) {
 // an exponent rounds it to 2^-18 absolute, a relative error under 2e-6 of
 // the exponential: far below a bf16 ulp.  fp32 outputs take the terms
 // flushed below 2^-126 (an absolute error under 1.2e-38 after the product).
+//
+// bf16 outputs of the tanh form take their reciprocal on the FMA pipes
+// (recip_newton: the elementwise bf16 kernel is bound by MUFU, two
+// operations per value), which wants a finite sum: inputs are raised to -11
+// instead of -30 (2^(a - 64) <= 2^98 there; every x <= -10.4 gives -0
+// already, the correctly rounded bf16 value).
 template <typename T>
 struct GeluScale {
   static constexpr float kBias = 0.0f;
   static constexpr float kUnbias = 1.0f;
+  static constexpr float kTanhFloor = kGeluFloor;
+  static constexpr bool kNewtonRecip = false;
 };
 template <>
 struct GeluScale<__nv_bfloat16> {
   static constexpr float kBias = 64.0f;
   static constexpr float kUnbias = 0x1p-64f;
+  static constexpr float kTanhFloor = -11.0f;
+  static constexpr bool kNewtonRecip = true;
 };
 
 // tanh form: 0.5 x (1 + tanh u) = x sigma(2u) = x / (1 + 2^a) with
@@ -64,10 +99,11 @@ struct GeluScale<__nv_bfloat16> {
 template <typename T>
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   using S = GeluScale<T>;
-  x = max_nan(x, kGeluFloor);
+  x = max_nan(x, S::kTanhFloor);
   const float p = fmaf(kB, x * x, kA);
   const float e = ex2_ftz(S::kBias != 0.0f ? fmaf(x, p, -S::kBias) : x * p);  // 2^(a - bias)
-  const float q = rcp_approx(e + S::kUnbias) * S::kUnbias;                    // 1 / (1 + 2^a)
+  const float sum = e + S::kUnbias;
+  const float q = (S::kNewtonRecip ? recip_newton(sum) : rcp_approx(sum)) * S::kUnbias;  // 1 / (1 + 2^a)
   return x * q;
 }
 
@@ -153,11 +189,15 @@ __device__ __forceinline__ float gelu_erf_f(float x) {
 template <typename T, bool CLAMPED = false>
 __device__ __forceinline__ float2 gelu_tanh_f2(float2 x) {
   using S = GeluScale<T>;
-  if (!CLAMPED) x = make_float2(max_nan(x.x, kGeluFloor), max_nan(x.y, kGeluFloor));
+  if (!CLAMPED) x = make_float2(max_nan(x.x, S::kTanhFloor), max_nan(x.y, S::kTanhFloor));
   const float2 p = fma2(splat2(kB), mul2(x, x), splat2(kA));
   const float2 a = S::kBias != 0.0f ? fma2(x, p, splat2(-S::kBias)) : mul2(x, p);
   const float2 s = add2(make_float2(ex2_ftz(a.x), ex2_ftz(a.y)), splat2(S::kUnbias));
-  float2 q = make_float2(rcp_approx(s.x), rcp_approx(s.y));
+  float2 q;
+  if constexpr (S::kNewtonRecip)
+    q = recip_newton2(s);
+  else
+    q = make_float2(rcp_approx(s.x), rcp_approx(s.y));
   if constexpr (S::kBias != 0.0f) q = mul2(q, splat2(S::kUnbias));
   return mul2(x, q);
 }
