@@ -25,6 +25,9 @@
 // flushes and y is -0 or x; tails of bf16 outputs are kept down to their
 // smallest subnormal, 2^-133, by an exponent offset of 64 (fk_gelu.cuh);
 // inputs below -30, -inf among them, give -0, the correctly rounded value.
+// For bf16 outputs, where MUFU limits the kernel, the reciprocal is taken on
+// the FMA pipes instead (a bit estimate and two Newton steps) and inputs are
+// raised to -11, below which the result is -0 already.
 //
 // Exact form: x Phi(x), Phi the standard normal distribution function, with
 // erfc in the form of Press et al. and coefficients fitted here (see
