@@ -271,8 +271,13 @@ __global__ void __launch_bounds__(kWarpThreads)
 
 // ---------------------------------------------------------------- block path
 
+// bf16 rows of 128-thread blocks fit 64 registers without spills: eight
+// blocks (rows in flight) per SM instead of seven.
+template <typename T, int THREADS>
+constexpr int ln_block_min_blocks() { return sizeof(T) == 2 && THREADS == 128 ? 8 : 1; }
+
 template <typename T, int THREADS, int EPT, bool ALIGNED, int EPI>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, ln_block_min_blocks<T, THREADS>())
     layernorm_block_kernel(const T* x, T* y, const float* gamma, const float* beta, size_t rows, int cols,
                            float eps) {
   constexpr int VEC = Elem<T>::VEC;
