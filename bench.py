@@ -252,6 +252,17 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def wait_ready(self, timeout_s: float = 3.0) -> None:
+        """Block until nvidia-smi has written its first reading (it takes a
+        few hundred ms to start), so that a short timed region still has a
+        reading next to it."""
+        t0 = time.monotonic()
+        while self.proc is not None and time.monotonic() - t0 < timeout_s:
+            self.out.flush()
+            if os.path.getsize(self.out.name) > 0:
+                return
+            time.sleep(0.02)
+
     def stop(self) -> dict | None:
         if self.proc is None:
             return None
@@ -537,7 +548,8 @@ def run_ours(args) -> dict | None:
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     barrier()
     sampler = ClockSampler(gpu_id) if rank == 0 else None
-    time.sleep(0.25 if sampler else 0)  # let the sampler take its first reading
+    if sampler:
+        sampler.wait_ready()  # its first reading before the timed region
     # the timed region: K steps, events only at its ends
     total_ms, _ = timed_steps(calls, args.steps, per_kernel=False)
     # per-kernel breakdown: K more steps with an event between every two kernels
@@ -772,7 +784,8 @@ def run_attention(args) -> dict | None:
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     barrier()
     sampler = ClockSampler(gpu_id) if rank == 0 else None
-    time.sleep(0.25 if sampler else 0)
+    if sampler:
+        sampler.wait_ready()
     barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
@@ -873,7 +886,7 @@ def library_attention(qkv, o, bh, t, d, causal, scale, flops, steps, warmup, str
                     call()
                 torch.cuda.synchronize()
                 sampler = ClockSampler(gpu_id)
-                time.sleep(0.25)
+                sampler.wait_ready()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 for _ in range(steps):
