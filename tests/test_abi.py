@@ -194,6 +194,28 @@ def test_noalloc_batches_fit_its_scratch_array(fk, dtype):
     assert P.fk_softmax_rows_plan(1, (1 << 35) + 1, dtype, P.FK_PATH_SPLIT).as_dict()["chunks"] > NOALLOC_PAIRS
 
 
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_noalloc_capacity_is_checked_before_the_device(fk, dtype):
+    """fk_softmax_rows_noalloc_cap refuses a capacity outside 1 .. 131072,
+    or one that cannot hold a batch as it is planned, before it looks at the
+    pointers or the device (so null pointers are enough here)."""
+    P = fk
+    rows, cols = 80, 1 << 22
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, rows, cols, dtype, 0, 0) == P.FK_ERR_INVALID_ARG
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, rows, cols, dtype, NOALLOC_PAIRS + 1, 0) == P.FK_ERR_INVALID_ARG
+    chunks = P.fk_softmax_rows_plan(rows, cols, dtype).as_dict()["chunks"]
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, rows, cols, dtype, chunks - 1, 0) == P.FK_ERR_INVALID_ARG
+    # a capacity that holds the batch size as planned for all rows, but not
+    # the batch as its own row count plans it (fewer rows, more chunks each)
+    split = P.make_plan(P.FK_PATH_SPLIT)
+    rows2, cap = 112, 592
+    per = cap // P.fk_softmax_rows_plan(rows2, cols, dtype).as_dict()["chunks"]
+    assert per >= 1 and P.fk_softmax_rows_workspace(per, cols, dtype, split) > cap * 8
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, rows2, cols, dtype, cap, 0) == P.FK_ERR_INVALID_ARG
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, rows, cols, 9, 1200, 0) == P.FK_ERR_UNSUPPORTED_DTYPE
+    assert P.fk_softmax_rows_noalloc_cap(0, 0, 0, cols, dtype, 1200, 0) == P.FK_OK  # empty: no-op
+
+
 def _layernorm_rule(cols, dtype):
     """The documented LayerNorm plan: one warp per row up to 1024 columns;
     one block per row up to 32768 (16 values per thread up to 2048 columns,
