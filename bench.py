@@ -875,9 +875,13 @@ def library_attention(qkv, o, bh, t, d, causal, scale, flops, steps, warmup, str
     ours = o.view(1, bh, t, d).float()
     out = {"what": "torch.nn.functional.scaled_dot_product_attention, same q, k, v, scale and mask, timed right "
                    "after the kernel (context only)", "torch": torch.__version__, "backends": {}}
-    for be in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION):
+    import contextlib
+    # torch's own choice of backend first (what a caller gets by default),
+    # then each fused backend forced
+    for label, be in (("DEFAULT", None), ("CUDNN_ATTENTION", SDPBackend.CUDNN_ATTENTION),
+                      ("FLASH_ATTENTION", SDPBackend.FLASH_ATTENTION)):
         try:
-            with sdpa_kernel(be):
+            with (sdpa_kernel(be) if be is not None else contextlib.nullcontext()):
                 def call():
                     return torch.nn.functional.scaled_dot_product_attention(q4, k4, v4, is_causal=causal,
                                                                             scale=scale)
@@ -895,11 +899,11 @@ def library_attention(qkv, o, bh, t, d, causal, scale, flops, steps, warmup, str
                 torch.cuda.synchronize()
                 clocks = sampler.stop()
                 ms = a.elapsed_time(b) / steps
-                out["backends"][be.name] = {"TFLOP_s": round(flops / ms / 1e9, 1), "ms": round(ms, 5),
-                                            "max_abs_diff_vs_this_kernel": float((ref.float() - ours).abs().max()),
-                                            "clocks": clocks}
+                out["backends"][label] = {"TFLOP_s": round(flops / ms / 1e9, 1), "ms": round(ms, 5),
+                                          "max_abs_diff_vs_this_kernel": float((ref.float() - ours).abs().max()),
+                                          "clocks": clocks}
         except RuntimeError as e:
-            out["backends"][be.name] = {"unavailable": str(e).splitlines()[0][:160]}
+            out["backends"][label] = {"unavailable": str(e).splitlines()[0][:160]}
     return out
 
 
