@@ -5,8 +5,10 @@
 //
 // Two ways of moving the data, chosen by size (measured on B200, fp32, L2
 // cleaned or left full of another kernel's dirty lines before each launch):
-//   * when input and output together fit in L2, a persistent pipeline
-//     through shared memory fed by the bulk-copy engine (cp.async.bulk):
+//   * when input and output together fit in L2 (and the input holds at
+//     least 8 MiB; smaller arrays take one wave through registers), a
+//     persistent pipeline through shared memory fed by the bulk-copy engine
+//     (cp.async.bulk):
 //     32 MiB in 11.5 us clean and 12.7 us after a dirty predecessor, against
 //     13.5 and 17.0 us for loads and stores through registers;
 //   * beyond that, one batch of two 16-byte loads per thread straight into
@@ -231,8 +233,14 @@ cudaError_t allow_stage_smem(K kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kStageSmem));
 }
 
-// The shared-memory pipeline while input and output together fit in L2.
-bool use_bulk(size_t bytes, size_t l2_bytes) { return bytes > 0 && 2 * bytes <= l2_bytes; }
+// The shared-memory pipeline while input and output together fit in L2 and
+// the input holds at least kBulkMinBytes: below that, one wave through
+// registers has less fixed latency (measured alone with L2 cleaned, fp32
+// tanh GELU: 1 MB 6.2 us against 8.1, 4 MB 6.6 against 8.1, 16 MB equal;
+// the copy is equal either way up to 4 MB and faster through shared memory
+// at 16 MB).
+constexpr size_t kBulkMinBytes = size_t{8} << 20;
+bool use_bulk(size_t bytes, size_t l2_bytes) { return bytes >= kBulkMinBytes && 2 * bytes <= l2_bytes; }
 
 // ---------------------------------------------------------------- kernels
 

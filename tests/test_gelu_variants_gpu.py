@@ -202,15 +202,16 @@ def test_tensor_wrapper_and_errors(fk, torch_mod):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_both_data_paths_around_the_l2_switch(fk, torch_mod, dtype, kind):
     """Arrays whose input and output together fit in L2 stream through shared
-    memory (bulk copies, persistent blocks, a short last chunk); larger ones
-    go through registers.  Both sides of the switch, with ragged tails and a
-    misaligned head, against the oracle."""
+    memory (bulk copies, persistent blocks, a short last chunk); larger ones,
+    and inputs under 8 MiB, go through registers.  Both sides of both
+    switches, with ragged tails and a misaligned head, against the oracle."""
     l2 = torch_mod.cuda.get_device_properties(0).L2_cache_size
     esize = 4 if dtype == "f32" else 2
     code = fk.FK_F32 if dtype == "f32" else fk.FK_BF16
     limit = l2 // (2 * esize)  # elements at which input + output fill L2
     g = np.random.default_rng(101)
-    for n, off in ((limit - 9, 0), (limit + 13, 0), (limit - 40, 3)):
+    small = (8 << 20) // esize  # elements at which the input reaches 8 MiB
+    for n, off in ((limit - 9, 0), (limit + 13, 0), (limit - 40, 3), (small - 5, 0), (small + 7, 1)):
         x = (g.standard_normal(n) * 5).astype(np.float32)
         if dtype == "f32":
             _check_f32(_run(fk, torch_mod, x, code, kind, xoff=off, yoff=off), x, kind)
