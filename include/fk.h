@@ -167,7 +167,9 @@ typedef enum fk_softmax_path {
                              number of rows, needs workspace */
 } fk_softmax_path;
 
-/* A resolved launch plan.  `threads` = threads per block; `vpt` = 16-byte
+/* A resolved launch plan.  `threads` = threads per block (on FK_PATH_WARP,
+ * 32 x the rows one block takes: 32, 64, 128 or 256, chosen from the row
+ * count so that few rows still reach every multiprocessor); `vpt` = 16-byte
  * vectors per thread per step; `cluster` = blocks per row for the cluster
  * paths (1 otherwise); `chunks` = blocks per row on the split path (derived
  * from the shape; 1 otherwise). */
@@ -195,7 +197,8 @@ FK_API fk_status fk_softmax_rows_plan(size_t rows, size_t cols, int dtype, int p
  * fk_softmax_rows_ex -- fk_softmax_rows with an explicit plan (tests and
  * tuning).  plan == NULL or plan->path == FK_PATH_AUTO behaves like
  * fk_softmax_rows.  Otherwise every field is validated against the compiled
- * kernel set (threads in {128,256,512,1024} for block paths; cluster in
+ * kernel set (threads in {32,64,128,256} for the warp path and
+ * {128,256,512,1024} for block paths; cluster in
  * 1..16; vpt fixed per dtype and path) and FK_ERR_INVALID_ARG is returned
  * for a plan that is not built or cannot hold `cols`.  Zero fields take the
  * path's defaults.

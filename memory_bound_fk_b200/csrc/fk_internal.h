@@ -42,7 +42,7 @@ cudaError_t launch_copy(const void* src, void* dst, size_t bytes, const DeviceIn
 cudaError_t read_gelu_wait_timeouts(unsigned* out, bool reset);
 
 // ---- softmax -----------------------------------------------------------
-constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path
+constexpr int kWarpRowsPerBlock = 8;        // warps (= rows) per block on the warp path, at most
 constexpr int kWarpThreads = 32 * kWarpRowsPerBlock;
 constexpr int kBlockEptSmall = 16;          // register-resident elements per thread (CTA/cluster)
 constexpr int kBlockEptLarge = 32;

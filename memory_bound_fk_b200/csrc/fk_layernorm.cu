@@ -252,9 +252,9 @@ __global__ void __launch_bounds__(kWarpThreads)
   const int lane = threadIdx.x & 31;
   const int nvec = (cols + VEC - 1) / VEC;
   const float inv_n = 1.0f / static_cast<float>(cols);
-  const size_t stride = static_cast<size_t>(gridDim.x) * kWarpRowsPerBlock;
-  for (size_t row = static_cast<size_t>(blockIdx.x) * kWarpRowsPerBlock + (threadIdx.x >> 5); row < rows;
-       row += stride) {
+  const unsigned rpb = blockDim.x >> 5;  // rows (= warps) per block
+  const size_t stride = static_cast<size_t>(gridDim.x) * rpb;
+  for (size_t row = static_cast<size_t>(blockIdx.x) * rpb + (threadIdx.x >> 5); row < rows; row += stride) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
     uint4 raw[VPT];
@@ -457,18 +457,19 @@ struct LnArgs {
 };
 
 template <typename T, bool ALIGNED, int EPI>
-cudaError_t launch_ln_warp(const LnArgs& a, int vpt, cudaStream_t s) {
-  size_t blocks = (a.rows + kWarpRowsPerBlock - 1) / kWarpRowsPerBlock;
+cudaError_t launch_ln_warp(const LnArgs& a, int threads, int vpt, cudaStream_t s) {
+  const size_t rpb = static_cast<size_t>(threads) / 32;
+  size_t blocks = (a.rows + rpb - 1) / rpb;
   if (blocks > kLnMaxGrid) blocks = kLnMaxGrid;
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
   const int c = static_cast<int>(a.cols);
   const unsigned g = static_cast<unsigned>(blocks);
   switch (vpt) {
-    case 1: layernorm_warp_kernel<T, 1, ALIGNED, EPI><<<g, kWarpThreads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
-    case 2: layernorm_warp_kernel<T, 2, ALIGNED, EPI><<<g, kWarpThreads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
-    case 4: layernorm_warp_kernel<T, 4, ALIGNED, EPI><<<g, kWarpThreads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
-    case 8: layernorm_warp_kernel<T, 8, ALIGNED, EPI><<<g, kWarpThreads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
+    case 1: layernorm_warp_kernel<T, 1, ALIGNED, EPI><<<g, threads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
+    case 2: layernorm_warp_kernel<T, 2, ALIGNED, EPI><<<g, threads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
+    case 4: layernorm_warp_kernel<T, 4, ALIGNED, EPI><<<g, threads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
+    case 8: layernorm_warp_kernel<T, 8, ALIGNED, EPI><<<g, threads, 0, s>>>(x, y, a.gamma, a.beta, a.rows, c, a.eps); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -493,7 +494,7 @@ cudaError_t launch_ln_block_ept(const LnArgs& a, int threads, cudaStream_t s) {
 template <typename T, bool ALIGNED, int EPI>
 cudaError_t launch_ln_plan(const LnArgs& a, const fk_softmax_plan& p, cudaStream_t s) {
   switch (p.path) {
-    case FK_PATH_WARP: return launch_ln_warp<T, ALIGNED, EPI>(a, p.vpt, s);
+    case FK_PATH_WARP: return launch_ln_warp<T, ALIGNED, EPI>(a, p.threads, p.vpt, s);
     case FK_PATH_CTA:
       switch (p.vpt * Elem<T>::VEC) {
         case 16: return launch_ln_block_ept<T, 16, ALIGNED, EPI>(a, p.threads, s);

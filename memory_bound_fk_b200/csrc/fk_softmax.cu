@@ -233,9 +233,9 @@ __global__ void __launch_bounds__(kWarpThreads)
   const int lane = threadIdx.x & 31;
   const int nvec = (cols + VEC - 1) / VEC;
   const float k = SC ? sc.k : kLog2e;
-  const size_t stride = static_cast<size_t>(gridDim.x) * kWarpRowsPerBlock;
-  for (size_t row = static_cast<size_t>(blockIdx.x) * kWarpRowsPerBlock + (threadIdx.x >> 5);
-       row < rows; row += stride) {
+  const unsigned rpb = blockDim.x >> 5;  // rows (= warps) per block
+  const size_t stride = static_cast<size_t>(gridDim.x) * rpb;
+  for (size_t row = static_cast<size_t>(blockIdx.x) * rpb + (threadIdx.x >> 5); row < rows; row += stride) {
     const T* xr = x + row * static_cast<size_t>(cols);
     T* yr = y + row * static_cast<size_t>(cols);
     uint4 raw[VPT];
@@ -626,16 +626,17 @@ cudaError_t launch(void (*kernel)(KArgs...), size_t blocks, int threads, int clu
 constexpr size_t kMaxGrid = 0x7fffffffu;
 
 template <typename T, bool ALIGNED, bool SC>
-cudaError_t launch_warp(const T* xp, T* yp, size_t rows, size_t cols, int vpt, SoftmaxScaling sc,
+cudaError_t launch_warp(const T* xp, T* yp, size_t rows, size_t cols, int threads, int vpt, SoftmaxScaling sc,
                         cudaStream_t s) {
-  size_t blocks = (rows + kWarpRowsPerBlock - 1) / kWarpRowsPerBlock;
+  const size_t rpb = static_cast<size_t>(threads) / 32;
+  size_t blocks = (rows + rpb - 1) / rpb;
   if (blocks > kMaxGrid) blocks = kMaxGrid;
   const int c = static_cast<int>(cols);
   switch (vpt) {
-    case 1: return launch(softmax_warp_kernel<T, 1, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
-    case 2: return launch(softmax_warp_kernel<T, 2, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
-    case 4: return launch(softmax_warp_kernel<T, 4, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
-    case 8: return launch(softmax_warp_kernel<T, 8, ALIGNED, SC>, blocks, kWarpThreads, 1, s, xp, yp, rows, c, sc);
+    case 1: return launch(softmax_warp_kernel<T, 1, ALIGNED, SC>, blocks, threads, 1, s, xp, yp, rows, c, sc);
+    case 2: return launch(softmax_warp_kernel<T, 2, ALIGNED, SC>, blocks, threads, 1, s, xp, yp, rows, c, sc);
+    case 4: return launch(softmax_warp_kernel<T, 4, ALIGNED, SC>, blocks, threads, 1, s, xp, yp, rows, c, sc);
+    case 8: return launch(softmax_warp_kernel<T, 8, ALIGNED, SC>, blocks, threads, 1, s, xp, yp, rows, c, sc);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -753,7 +754,7 @@ cudaError_t launch_typed(const void* x, void* y, size_t rows, size_t cols, const
   const T* xp = static_cast<const T*>(x);
   T* yp = static_cast<T*>(y);
   switch (p.path) {
-    case FK_PATH_WARP: return launch_warp<T, ALIGNED, SC>(xp, yp, rows, cols, p.vpt, sc, s);
+    case FK_PATH_WARP: return launch_warp<T, ALIGNED, SC>(xp, yp, rows, cols, p.threads, p.vpt, sc, s);
     case FK_PATH_CTA: return launch_block<T, ALIGNED, SC>(xp, yp, rows, cols, p.threads, p.vpt, sc, s);
     case FK_PATH_CLUSTER:
       return launch_cluster<T, ALIGNED, SC>(xp, yp, rows, cols, p.threads, p.vpt, p.cluster, sc, s);

@@ -71,7 +71,7 @@ def check_softmax_bf16(y_bits: np.ndarray, ref_bits: np.ndarray, x_bits: np.ndar
 def forced_plans(fk, cols, dtype):
     """Every compiled softmax plan that can hold `cols` columns of `dtype`
     ("f32" or "bf16"): CTA and cluster shapes, two-phase with 1..16 blocks,
-    split, and the warp path where a row fits a warp."""
+    split, and the warp path (1 to 8 rows per block) where a row fits a warp."""
     plans = []
     vec = 4 if dtype == "f32" else 8
     for ept in (16, 32):
@@ -88,5 +88,6 @@ def forced_plans(fk, cols, dtype):
         plans.append(fk.make_plan(fk.FK_PATH_TWOPHASE, cluster=k))
     plans.append(fk.make_plan(fk.FK_PATH_SPLIT))
     if cols <= (1024 if dtype == "f32" else 2048):
-        plans.append(fk.make_plan(fk.FK_PATH_WARP, vpt=8))
+        for t in (32, 64, 128, 256):  # 1, 2, 4 and 8 rows per block
+            plans.append(fk.make_plan(fk.FK_PATH_WARP, threads=t, vpt=8))
     return plans

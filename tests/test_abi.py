@@ -24,17 +24,21 @@ def test_version_and_status_strings(fk):
 
 
 @pytest.mark.parametrize("rows,cols,dtype,expect", [
-    (256, 1000, 0, ("warp", 256, 8, 1)),        # 256x1000 fp32
+    (256, 1000, 0, ("warp", 64, 8, 1)),         # 256x1000 fp32: two rows per block
     (8192, 4096, 0, ("cta", 128, 8, 1)),        # 8192x4096 fp32
     (1 << 20, 2048, 1, ("cta", 128, 2, 1)),     # bf16 attention rows
     (512, 131072, 0, ("cluster", 128, 16, 16)), # vocab-sized rows
-    (4, 1, 0, ("warp", 256, 1, 1)),
-    (4, 128, 0, ("warp", 256, 1, 1)),
-    (4, 129, 0, ("warp", 256, 2, 1)),
-    (4, 1024, 0, ("warp", 256, 8, 1)),
+    (4, 1, 0, ("warp", 64, 1, 1)),
+    (4, 128, 0, ("warp", 64, 1, 1)),
+    (4, 129, 0, ("warp", 64, 2, 1)),
+    (4, 1024, 0, ("warp", 64, 8, 1)),
+    (588, 1000, 0, ("warp", 64, 8, 1)),         # 147 blocks of 4 rows leave an SM idle
+    (589, 1000, 0, ("warp", 128, 8, 1)),
+    (1176, 1000, 0, ("warp", 128, 8, 1)),
+    (1177, 1000, 0, ("warp", 256, 8, 1)),       # 148 blocks of 8 rows
     (4, 1025, 0, ("cta", 128, 8, 1)),
     (4, 2049, 1, ("cta", 256, 2, 1)),
-    (4, 1024, 1, ("warp", 256, 4, 1)),
+    (4, 1024, 1, ("warp", 64, 4, 1)),
     (4, 16385, 1, ("cta", 1024, 4, 1)),
     (4, 32768, 0, ("cta", 1024, 8, 1)),
     (4, 32769, 0, ("cluster", 128, 16, 5)),
@@ -109,7 +113,8 @@ def test_valid_looking_arguments_without_a_usable_device_are_rejected(fk):
 
 
 def test_explicit_plan_validation(fk):
-    bad = [fk.make_plan(fk.FK_PATH_WARP, threads=128),
+    bad = [fk.make_plan(fk.FK_PATH_WARP, threads=96),
+           fk.make_plan(fk.FK_PATH_WARP, threads=512),
            fk.make_plan(fk.FK_PATH_WARP, vpt=3),
            fk.make_plan(fk.FK_PATH_CTA, threads=96),
            fk.make_plan(fk.FK_PATH_CLUSTER, cluster=17),

@@ -121,7 +121,8 @@ def _plans(fk, cols, dtype):
             if t * ept >= cols:
                 plans.append(fk.make_plan(fk.FK_PATH_CTA, threads=t, vpt=ept // vec))
     if cols <= 32 * 8 * vec:
-        plans.append(fk.make_plan(fk.FK_PATH_WARP, vpt=8))
+        for t in (32, 64, 128, 256):  # 1, 2, 4 and 8 rows per block
+            plans.append(fk.make_plan(fk.FK_PATH_WARP, threads=t, vpt=8))
     return plans
 
 
