@@ -267,7 +267,8 @@ struct AttnUnits {
 // query tile, every row's unnormalised O (fp32) and its (reference max m,
 // sum l), and per split unit and tile a counter of the halves that finished.
 struct AttnSplitScratch {
-  float* o;        // [nsplit][2 halves][2 tiles][128 rows][D]
+  float* o;        // [nsplit][2 halves][2 tiles][D / 4 column quads][128 rows][4]: a warp's
+                   // 32 rows of one quad are 512 contiguous bytes
   float2* ml;      // [nsplit][2 halves][2 tiles][128 rows]
   unsigned* done;  // [nsplit][2 tiles], zero at launch
 };
@@ -531,8 +532,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                           pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
           }
         }
-      } else {
-        // Half of a split unit.  Both halves store their rows' unnormalised
+      } else if constexpr (!CAUSAL) {
+        // Half of a split unit (non-causal grids only).  Both halves store their rows' unnormalised
         // O and (m, l); the half that finishes second (by an atomic count
         // per unit and tile, taken after a fence) merges the other's with
         // its own and writes the output.  Nothing waits on the other block.
@@ -543,16 +544,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         warpgroup_bar(i);
         if (!split_flag[i]) {
           const int su = wk.u - nfull;
-          const size_t mine = (static_cast<size_t>(su * 2 + wk.half) * 2 + i) * kAttnBlock + r;
-          const size_t other = (static_cast<size_t>(su * 2 + (1 - wk.half)) * 2 + i) * kAttnBlock + r;
+          const size_t tmine = static_cast<size_t>(su * 2 + wk.half) * 2 + i;
+          const size_t tother = static_cast<size_t>(su * 2 + (1 - wk.half)) * 2 + i;
+          const size_t mine = tmine * kAttnBlock + r, other = tother * kAttnBlock + r;
           tc::fence_after_sync();
-          float4* po = reinterpret_cast<float4*>(split.o + mine * D);
+          float4* po = reinterpret_cast<float4*>(split.o) + tmine * kAttnBlock * (D / 4) + r;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float v[32];
             tc::tmem_ld32(tO + c * 32, v);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) po[c * 8 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int q = 0; q < 8; ++q)
+              po[(c * 8 + q) * kAttnBlock] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           }
           split.ml[mine] = make_float2(m_i, l_i);
           __threadfence();
@@ -561,20 +564,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           warpgroup_bar(i);
           if (split_flag[i] == 1) {
             __threadfence();
-            // the other half's (m, l) and O, read through L2 (written by another SM)
+            // the other half's (m, l) and O, read through L2 (written by
+            // another SM), all of the row's loads in flight at once
+            const float4* oo = reinterpret_cast<const float4*>(split.o) + tother * kAttnBlock * (D / 4) + r;
             const float2 mlo = __ldcg(split.ml + other);
+            float4 wo[D / 4];
+#pragma unroll
+            for (int q = 0; q < D / 4; ++q) wo[q] = __ldcg(oo + q * kAttnBlock);
             const float M = fmaxf(m_i, mlo.x);
             const float fa = (m_i == M) ? 1.0f : ex2_ftz(m_i - M);
             const float fb = (mlo.x == M) ? 1.0f : ex2_ftz(mlo.x - M);
             const float inv = 1.0f / fmaf(l_i, fa, mlo.y * fb);
-            const float4* oo = reinterpret_cast<const float4*>(split.o + other * D);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               float v[32];
               tc::tmem_ld32(tO + c * 32, v);
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
-                const float4 w = __ldcg(oo + c * 8 + q);
+                const float4 w = wo[c * 8 + q];
                 v[4 * q] = fmaf(v[4 * q], fa, w.x * fb) * inv;
                 v[4 * q + 1] = fmaf(v[4 * q + 1], fa, w.y * fb) * inv;
                 v[4 * q + 2] = fmaf(v[4 * q + 2], fa, w.z * fb) * inv;
