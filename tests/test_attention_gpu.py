@@ -83,6 +83,19 @@ def test_persistent_grids(fk, torch_mod, bh, t, d):
     assert fk.fk_wait_timeouts(reset=True) == 0
 
 
+@pytest.mark.parametrize("bh,t,d", [(100, 512, 64), (120, 384, 64), (60, 640, 128)])
+def test_persistent_causal_grids(fk, torch_mod, bh, t, d):
+    """Causal grids of two rounds over the persistent blocks, the longest
+    pairs first: the first S products of a block's next unit go out while its
+    current unit's second tile still runs (a pair's first tile has one key
+    block fewer), and units of a single query tile (odd query-tile counts,
+    384 and 640) shift the three Q slots.  Every slice against the oracle."""
+    q, k, v = inputs(bh, t, d, seed=bh * 5 + t + d)
+    scale = 1.0 / math.sqrt(d)
+    check(run(fk, torch_mod, q, k, v, True, scale), q, k, v, True, scale)
+    assert fk.fk_wait_timeouts(reset=True) == 0
+
+
 @pytest.mark.parametrize("sigma,scale", [(3.0, 0.125), (1.0, 1.0), (0.2, 0.05)])
 def test_score_ranges(fk, torch_mod, sigma, scale):
     """Peaked and flat attention: large scores (the running max moves often)
