@@ -241,7 +241,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_power_cap"]
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_id: str, period_ms: int = 100):
+    def __init__(self, gpu_id: str, period_ms: int = 20):
         self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         self.proc = None
         try:
