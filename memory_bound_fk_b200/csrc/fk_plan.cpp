@@ -2,7 +2,8 @@
 //
 // The capacities follow from the kernels' register budgets:
 //   warp     : 32 lanes x VPT 16-byte vectors, VPT in {1, 2, 4, 8}
-//              -> up to 1024 fp32 / 2048 bf16 columns
+//              -> up to 1024 fp32 / 2048 bf16 columns; 1 to 8 rows (warps)
+//              per block, 2 to 8 by default (see warp_threads_for)
 //   block    : 16 or 32 elements per thread (EPT), threads in
 //              {128, 256, 512, 1024} -> up to 32768 columns
 //   cluster  : 2..16 blocks of 128..512 threads holding 64 values each
