@@ -350,15 +350,20 @@ __global__ void __launch_bounds__(THREADS, (EPT * sizeof(T) <= 32 && THREADS <= 
 // A cluster of csize blocks per row; block `rank` holds vectors
 // [rank*per, (rank+1)*per) of the row in registers, per = ceil(nvec / csize).
 // With 64 values a thread the plain aligned kernel's register budget is held
-// to six 128-thread blocks an SM (three of 256): more clusters resident, so
-// that others stream while one waits at its exchange (80 vs 95 registers, no
-// spills; 512 x 131072 fp32 runs 80 instead of 86 us).  The scaled and the
-// unaligned forms would spill under that bound and keep the default.
-template <int THREADS, int EPT, bool PLAIN>
-constexpr int cluster_min_blocks() { return PLAIN && EPT == 64 && THREADS <= 256 ? 768 / THREADS : 1; }
+// so that more clusters are resident, and others stream while one waits at
+// its exchange: fp32 to six 128-thread blocks an SM (three of 256; 80 vs 95
+// registers, no spills; 512 x 131072 fp32 runs 80 instead of 86 us, and 7%
+// slower again at seven), bf16 to eight (four of 256; 64 registers, no
+// spills; 4096 x 65536 bf16 204 -> 191 us, 1024 x 131072 119 -> 107).  The
+// scaled and the unaligned forms would spill under that bound and keep the
+// default.
+template <typename T, int THREADS, int EPT, bool PLAIN>
+constexpr int cluster_min_blocks() {
+  return PLAIN && EPT == 64 && THREADS <= 256 ? (sizeof(T) == 2 ? 1024 : 768) / THREADS : 1;
+}
 
 template <typename T, int THREADS, int EPT, bool ALIGNED, bool SC>
-__global__ void __launch_bounds__(THREADS, cluster_min_blocks<THREADS, EPT, ALIGNED && !SC>())
+__global__ void __launch_bounds__(THREADS, cluster_min_blocks<T, THREADS, EPT, ALIGNED && !SC>())
     softmax_cluster_kernel(const T* x, T* y, size_t rows, int cols, SoftmaxScaling sc) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int VPT = EPT / VEC;
