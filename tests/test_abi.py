@@ -57,6 +57,20 @@ def test_auto_plans(fk, rows, cols, dtype, expect):
     assert (p["path"], p["threads"], p["vpt"], p["cluster"]) == expect
 
 
+def test_warp_rows_per_block_follow_the_rule(fk):
+    """The warp path's rows per block (threads / 32): the largest of 8, 4, 2
+    whose grid still gives each of the B200's 148 SMs a block, 2 at the
+    least, for every row count and both dtypes (LayerNorm takes the same)."""
+    for dtype in (0, 1):
+        for rows in list(range(1, 1300, 7)) + [1183, 1184, 1185, 4096, 1 << 20]:
+            t = fk.fk_softmax_rows_plan(rows, 1000, dtype).as_dict()["threads"]
+            want = 8
+            while want > 2 and -(-rows // want) < 148:
+                want //= 2
+            assert t == 32 * want, (dtype, rows, t)
+            assert fk.fk_layernorm_rows_plan(rows, 1000, dtype).as_dict()["threads"] == t
+
+
 def test_forced_plans_and_capacity_errors(fk):
     P = fk
     assert P.fk_softmax_rows_plan(2, 100, 0, P.FK_PATH_TWOPHASE).as_dict()["cluster"] == 1
