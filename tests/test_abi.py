@@ -37,10 +37,14 @@ def test_version_and_status_strings(fk):
     (1176, 1000, 0, ("warp", 128, 8, 1)),
     (1177, 1000, 0, ("warp", 256, 8, 1)),       # 148 blocks of 8 rows
     (4, 1025, 0, ("cta", 128, 8, 1)),
-    (4, 2049, 1, ("cta", 256, 2, 1)),
+    (4, 2049, 1, ("cta", 128, 4, 1)),        # bf16 past 2048 columns: 32 values a thread
+    (4, 8192, 0, ("cta", 256, 8, 1)),
+    (4, 8193, 0, ("cluster", 128, 16, 2)),     # wider rows: clusters of 128-thread blocks
+    (4, 8192, 1, ("cta", 256, 4, 1)),
+    (4, 8193, 1, ("cluster", 128, 8, 2)),
     (4, 1024, 1, ("warp", 64, 4, 1)),
-    (4, 16385, 1, ("cta", 1024, 4, 1)),
-    (4, 32768, 0, ("cta", 1024, 8, 1)),
+    (4, 16385, 1, ("cluster", 128, 8, 3)),
+    (4, 32768, 0, ("cluster", 128, 16, 4)),
     (4, 32769, 0, ("cluster", 128, 16, 5)),
     (4, 131073, 0, ("cluster", 256, 16, 9)),
     (4, 524288, 0, ("cluster", 512, 16, 16)),
