@@ -75,6 +75,54 @@ def test_warp_rows_per_block_follow_the_rule(fk):
             assert fk.fk_layernorm_rows_plan(rows, 1000, dtype).as_dict()["threads"] == t
 
 
+def _softmax_rule(rows, cols, dtype):
+    """The documented automatic softmax plan, restated: a warp per row up to
+    1024 columns; one block per row up to 8192 (bf16 rows of up to 2048
+    columns 16 values a thread, every other row 32; the fewest threads from
+    128 that hold the row); clusters of blocks with 64 values a thread up to
+    524288 (the smallest block from 128 threads whose cluster of at most 16
+    holds the row, at least 2 blocks); past that the split path for fewer
+    than 4 rows or 4M columns and more, else the two-phase path."""
+    vec = 4 if dtype == 0 else 8
+    if cols <= 1024:
+        vpt = 1
+        while 32 * vpt * vec < cols:
+            vpt *= 2
+        return ("warp", vpt, 1)
+    if cols <= 8192:
+        ept = 16 if dtype == 1 and cols <= 2048 else 32
+        t = 128
+        while t * ept < cols:
+            t *= 2
+        return ("cta", t, ept // vec, 1)
+    if cols <= 16 * 512 * 64:
+        t = 128
+        k = -(-cols // (t * 64))
+        while k > 16:
+            t *= 2
+            k = -(-cols // (t * 64))
+        return ("cluster", t, 64 // vec, max(k, 2))
+    return ("split",) if rows < 4 or cols >= 1 << 22 else ("twophase",)
+
+
+def test_softmax_auto_plans_follow_the_rule(fk):
+    widths = sorted({1, 7, 64, 100, 128, 129, 513, 1000, 1024, 1025, 2047, 2048, 2049, 4095, 4096, 4097,
+                     8191, 8192, 8193, 16384, 16385, 32768, 32769, 65536, 131072, 131073, 262144, 262145,
+                     524288, 524289, 1 << 21, (1 << 22) - 1, 1 << 22})
+    for dtype in (0, 1):
+        for rows in (1, 3, 4, 5000):
+            for cols in widths:
+                p = fk.fk_softmax_rows_plan(rows, cols, dtype).as_dict()
+                want = _softmax_rule(rows, cols, dtype)
+                got = (p["path"],) + ((p["vpt"], p["cluster"]) if p["path"] == "warp" else
+                                       (p["threads"], p["vpt"], p["cluster"]) if p["path"] in ("cta", "cluster")
+                                       else ())
+                assert got == want, (rows, cols, dtype, p, want)
+                # whatever the path, a row is held (or streamed) whole
+                if p["path"] in ("cta", "cluster"):
+                    assert p["threads"] * p["vpt"] * (4 if dtype == 0 else 8) * p["cluster"] >= cols
+
+
 def test_forced_plans_and_capacity_errors(fk):
     P = fk
     assert P.fk_softmax_rows_plan(2, 100, 0, P.FK_PATH_TWOPHASE).as_dict()["cluster"] == 1
